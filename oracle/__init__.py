@@ -1,0 +1,153 @@
+"""fp64 CPU oracle for the generalized-causal GQA attention with 2D RoPE.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the ``cpu_baseline`` / reference leg of ``bench.py``.  The product path
+(``joint_text_image_b200``) never imports it.  The arithmetic lives in
+``oracle.c`` (plain C, fp64); this module only marshals numpy arrays.
+
+Every function cites its passage in ``oracle.c``.  Parity pins live in
+``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (plain gcc, IEEE fp64, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c11",
+                               "-D_GNU_SOURCE", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        D = ctypes.c_double
+        lib.oracle_mask.argtypes = [I, I, P, P, P, P, P]
+        lib.oracle_positions.argtypes = [I, I, P, P, P, P, P, P]
+        lib.oracle_rope_tables.argtypes = [I, I, I, P, P, P, P, D, P, P]
+        lib.oracle_rope_apply.argtypes = [I, I, I, I, P, P, P, P, D, I, P, P]
+        lib.oracle_attn_fwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, D, D, I, P, I, P, P, P, I]
+        lib.oracle_attn_bwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, D, D, I, P, P, P, P, I]
+        _lib = lib
+    return _lib
+
+
+def _geom(samples):
+    """samples: list of (prefix, img_h, img_w, suffix) -> four int32 arrays."""
+    a = np.asarray(samples, dtype=np.int32).reshape(-1, 4)
+    return [np.ascontiguousarray(a[:, i]) for i in range(4)]
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def mask(samples, S: int) -> np.ndarray:
+    """uint8 [B, S, S] indexed [b, query, key] from the literal rule."""
+    g = _geom(samples)
+    out = np.zeros((len(g[0]), S, S), dtype=np.uint8)
+    if _load().oracle_mask(len(g[0]), S, *map(_p, g), _p(out)) != 0:
+        raise ValueError("bad sample geometry")
+    return out
+
+
+def positions(samples, S: int):
+    """(x, y) int64 [B, S] 2D RoPE positions."""
+    g = _geom(samples)
+    B = len(g[0])
+    x = np.zeros((B, S), dtype=np.int64)
+    y = np.zeros((B, S), dtype=np.int64)
+    if _load().oracle_positions(B, S, *map(_p, g), _p(x), _p(y)) != 0:
+        raise ValueError("bad sample geometry")
+    return x, y
+
+
+def rope_tables(samples, S: int, D: int, base: float = 10000.0):
+    """(cos, sin) fp64 [B, S, D]."""
+    g = _geom(samples)
+    B = len(g[0])
+    c = np.zeros((B, S, D))
+    s = np.zeros((B, S, D))
+    if _load().oracle_rope_tables(B, S, D, *map(_p, g), float(base), _p(c), _p(s)) != 0:
+        raise ValueError("bad arguments")
+    return c, s
+
+
+def rope_apply(samples, x: np.ndarray, base: float = 10000.0, inverse: bool = False):
+    """R x (or R^T x) for x fp64 [B, S, H, D]."""
+    g = _geom(samples)
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    B, S, H, D = x.shape
+    y = np.zeros_like(x)
+    if _load().oracle_rope_apply(B, S, H, D, *map(_p, g), float(base), int(inverse), _p(x), _p(y)) != 0:
+        raise ValueError("bad arguments")
+    return y
+
+
+def attn_fwd(samples, q, k, v, scale=None, base=10000.0, rotate=True, rows=None,
+             groups=None, nthreads=0):
+    """Forward: returns (o [B,S,Hq,D], lse [B,Hq,S], threads_used).
+
+    q [B,S,Hq,D], k/v [B,S,Hkv,D] as fp64 (exact copies of the bf16 inputs).
+    rows: optional int list of query rows; groups: optional bool [B, Hkv]."""
+    g = _geom(samples)
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    gs = None if groups is None else np.ascontiguousarray(groups, dtype=np.uint8).reshape(-1)
+    o = np.zeros((B, S, Hq, D))
+    lse = np.zeros((B, Hq, S))
+    used = _load().oracle_attn_fwd(B, S, Hq, Hkv, D, *map(_p, g), _p(q), _p(k), _p(v),
+                                   float(scale), float(base), int(rotate), _p(r),
+                                   0 if r is None else len(r), _p(gs), _p(o), _p(lse),
+                                   int(nthreads))
+    if used < 0:
+        raise ValueError("bad arguments")
+    return o, lse, used
+
+
+def attn_bwd(samples, q, k, v, dout, scale=None, base=10000.0, rotate=True, groups=None,
+             nthreads=0):
+    """Backward: returns (dq [B,S,Hq,D], dk, dv [B,S,Hkv,D], threads_used)."""
+    g = _geom(samples)
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    dout = np.ascontiguousarray(dout, dtype=np.float64)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    gs = None if groups is None else np.ascontiguousarray(groups, dtype=np.uint8).reshape(-1)
+    dq = np.zeros((B, S, Hq, D))
+    dk = np.zeros((B, S, Hkv, D))
+    dv = np.zeros((B, S, Hkv, D))
+    used = _load().oracle_attn_bwd(B, S, Hq, Hkv, D, *map(_p, g), _p(q), _p(k), _p(v), _p(dout),
+                                   float(scale), float(base), int(rotate), _p(gs), _p(dq),
+                                   _p(dk), _p(dv), int(nthreads))
+    if used < 0:
+        raise ValueError("bad arguments")
+    return dq, dk, dv, used

@@ -1,0 +1,440 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle for the generalized-causal GQA
+ * self-attention with the generalized 2D RoPE (HunyuanImage-3.0).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this file's library.  It shares no
+ * code, header, table or constant with the CUDA path, and it never reads a
+ * value produced by the CUDA path.
+ *
+ * Sources (page title, section / API item):
+ *   - "HunyuanImage-3.0" model-coverage page, Cache Contract: the sequence is
+ *     prefix (ending in <timestep>) + <img> * (h*w) + suffix, right-padded.
+ *   - nemo_automodel ... hunyuan_image3.model, build_joint_attention_mask:
+ *     boolean [batch,1,seq,seq] mask indexed [b,1,query,key]: causal text,
+ *     bidirectional image span, padded keys masked out.
+ *   - HunyuanImage 3.0 Technical Report summary, 3.1.2 Generalized Causal
+ *     Attention and 3.1.3 Position Embedding.
+ *   - Paper review (xllm-io), 3.3 generalized causal attention and 3.4
+ *     generalized 2D RoPE: 1D RoPE [cos n t0, cos n t1, ..., sin n t0, ...];
+ *     2D [cos x t0, cos y t1, ..., sin x t0, sin y t1, ...]; text on the
+ *     diagonal x = y = n; image positions reshaped to h x w between the text
+ *     segments; exact reduction to 1D RoPE with no image.
+ *   - nemo_automodel ... hunyuan_image3.layers, HunyuanImage3Attention:
+ *     fused KV-head-grouped QKV (query head h uses kv head h / q_per_kv);
+ *     cos/sin tables are fp32 [batch, seq, head_dim].
+ *   - ... layers, UNetDown.forward: image tokens in row-major (height, width)
+ *     order.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *   - padded query rows (q >= L) are ordinary rows that see keys [0, L-1];
+ *   - a row with no visible key (only when L == 0) has O = 0, LSE = -inf and
+ *     zero gradients;
+ *   - theta_j = base^(-2j/D), j < D/2; channel pair (j, j + D/2) is rotated by
+ *     angle_j (half-split layout);
+ *   - image token i (row r = i / w, column c = i % w) sits at x = I0 + c,
+ *     y = I0 + r; even j use x, odd j use y; every other token (text, suffix,
+ *     padding) sits at x = y = n, its sequence index;
+ *   - scores are scale * <R q, R k>, with scale passed in (1/sqrt(D)).
+ *
+ * Parity pins: every function here is pinned by the CPU tests (hand-written
+ * masks, closed-form pair counts, the 1D-RoPE library routine, relative
+ * position invariance, a library attention routine, finite differences).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+/* ------------------------------------------------------------------------ */
+/* Sample geometry                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* One sample: prefix P (text incl. <timestep>), image h x w, suffix s.
+ * I0 = P, I1 = P + h*w, L = I1 + s.  Padding is [L, S). */
+typedef struct {
+    int64_t I0, I1, L, w;
+} osample;
+
+static osample make_sample(int32_t prefix, int32_t h, int32_t w, int32_t suffix) {
+    osample s;
+    s.I0 = prefix;
+    s.I1 = (int64_t)prefix + (int64_t)h * (int64_t)w;
+    s.L = s.I1 + suffix;
+    s.w = w;
+    return s;
+}
+
+/* The literal mask rule (build_joint_attention_mask; 3.1.2; 3.3):
+ *   key k visible from query q  <=>  k < L  and  ( k <= q  or
+ *                                   (I0 <= q < I1 and I0 <= k < I1) ). */
+static int visible(const osample* s, int64_t q, int64_t k) {
+    if (k >= s->L) return 0;
+    if (k <= q) return 1;
+    if (s->I0 <= q && q < s->I1 && s->I0 <= k && k < s->I1) return 1;
+    return 0;
+}
+
+/* mask: uint8 [B, S, S] indexed [b, q, k]. */
+int oracle_mask(int B, int S, const int32_t* prefix, const int32_t* img_h,
+                const int32_t* img_w, const int32_t* suffix, uint8_t* mask) {
+    for (int b = 0; b < B; ++b) {
+        osample s = make_sample(prefix[b], img_h[b], img_w[b], suffix[b]);
+        if (s.L > S) return -1;
+        for (int64_t q = 0; q < S; ++q)
+            for (int64_t k = 0; k < S; ++k)
+                mask[((int64_t)b * S + q) * S + k] = (uint8_t)visible(&s, q, k);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Generalized 2D RoPE (3.4 of the paper review)                             */
+/* ------------------------------------------------------------------------ */
+
+/* 2D position (x, y) of token n of sample s. */
+static void position(const osample* s, int64_t n, double* x, double* y) {
+    if (s->I0 <= n && n < s->I1) {
+        int64_t i = n - s->I0;
+        int64_t r = i / s->w, c = i % s->w;
+        *x = (double)(s->I0 + c);
+        *y = (double)(s->I0 + r);
+    } else {
+        *x = (double)n;
+        *y = (double)n;
+    }
+}
+
+/* angle_j of token n: (j even ? x : y) * base^(-2j/D). */
+static double angle(const osample* s, int64_t n, int j, int D, double base) {
+    double x, y;
+    position(s, n, &x, &y);
+    double theta = pow(base, -2.0 * (double)j / (double)D);
+    return ((j % 2 == 0) ? x : y) * theta;
+}
+
+/* positions: int64 [B, S] x and y. */
+int oracle_positions(int B, int S, const int32_t* prefix, const int32_t* img_h,
+                     const int32_t* img_w, const int32_t* suffix, int64_t* xs, int64_t* ys) {
+    for (int b = 0; b < B; ++b) {
+        osample s = make_sample(prefix[b], img_h[b], img_w[b], suffix[b]);
+        if (s.L > S) return -1;
+        for (int64_t n = 0; n < S; ++n) {
+            double x, y;
+            position(&s, n, &x, &y);
+            xs[(int64_t)b * S + n] = (int64_t)x;
+            ys[(int64_t)b * S + n] = (int64_t)y;
+        }
+    }
+    return 0;
+}
+
+/* cos, sin fp64 [B, S, D]: entry j and j + D/2 both hold angle_j. */
+int oracle_rope_tables(int B, int S, int D, const int32_t* prefix, const int32_t* img_h,
+                       const int32_t* img_w, const int32_t* suffix, double base,
+                       double* cos_t, double* sin_t) {
+    if (D % 2) return -1;
+    for (int b = 0; b < B; ++b) {
+        osample s = make_sample(prefix[b], img_h[b], img_w[b], suffix[b]);
+        if (s.L > S) return -1;
+        for (int64_t n = 0; n < S; ++n)
+            for (int j = 0; j < D / 2; ++j) {
+                double a = angle(&s, n, j, D, base);
+                int64_t o = ((int64_t)b * S + n) * D;
+                cos_t[o + j] = cos(a);
+                cos_t[o + j + D / 2] = cos(a);
+                sin_t[o + j] = sin(a);
+                sin_t[o + j + D / 2] = sin(a);
+            }
+    }
+    return 0;
+}
+
+/* R(n) v: (Rv)_j = v_j cos a_j - v_{j+D/2} sin a_j,
+ *         (Rv)_{j+D/2} = v_{j+D/2} cos a_j + v_j sin a_j.
+ * (v * cos + rotate_half(v) * sin, rotate_half(v) = [-v_hi, v_lo].) */
+static void rotate(const osample* s, int64_t n, int D, double base, const double* v, double* out) {
+    for (int j = 0; j < D / 2; ++j) {
+        double a = angle(s, n, j, D, base);
+        double c = cos(a), sn = sin(a);
+        double lo = v[j], hi = v[j + D / 2];
+        out[j] = lo * c - hi * sn;
+        out[j + D / 2] = hi * c + lo * sn;
+    }
+}
+
+/* R(n)^T v, the inverse rotation (R is orthogonal). */
+static void rotate_t(const osample* s, int64_t n, int D, double base, const double* v, double* out) {
+    for (int j = 0; j < D / 2; ++j) {
+        double a = angle(s, n, j, D, base);
+        double c = cos(a), sn = sin(a);
+        double lo = v[j], hi = v[j + D / 2];
+        out[j] = lo * c + hi * sn;
+        out[j + D / 2] = hi * c - lo * sn;
+    }
+}
+
+/* Apply R (inverse = 0) or R^T (inverse = 1) to x [B, S, H, D] in place of y. */
+int oracle_rope_apply(int B, int S, int H, int D, const int32_t* prefix, const int32_t* img_h,
+                      const int32_t* img_w, const int32_t* suffix, double base, int inverse,
+                      const double* x, double* y) {
+    if (D % 2) return -1;
+    for (int b = 0; b < B; ++b) {
+        osample s = make_sample(prefix[b], img_h[b], img_w[b], suffix[b]);
+        if (s.L > S) return -1;
+        for (int64_t n = 0; n < S; ++n)
+            for (int h = 0; h < H; ++h) {
+                int64_t o = (((int64_t)b * S + n) * H + h) * D;
+                if (inverse) rotate_t(&s, n, D, base, x + o, y + o);
+                else rotate(&s, n, D, base, x + o, y + o);
+            }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Attention: naive S x S scores with the explicit mask, fp64 softmax.        */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int B, S, Hq, Hkv, D;
+    const int32_t *prefix, *img_h, *img_w, *suffix;
+    const double *q, *k, *v, *dout;
+    double scale, base;
+    int rotate_inputs;          /* 1: apply R to q, k here; 0: inputs already rotated */
+    const int32_t* rows;        /* query rows to compute, or NULL for all */
+    int n_rows;
+    const uint8_t* group_sel;   /* [B * Hkv] 1 = compute this (b, kv head) group; NULL = all */
+    double *o, *lse;            /* fwd outputs */
+    double *dq, *dk_h, *dv_h;   /* bwd outputs; dk_h, dv_h per q head [B,S,Hq,D] */
+    int n_tasks;
+    int next_task;
+    pthread_mutex_t lock;
+} job_t;
+
+static double dot(const double* a, const double* b, int D) {
+    double s = 0.0;
+    for (int d = 0; d < D; ++d) s += a[d] * b[d];
+    return s;
+}
+
+/* Rotated copy of head h of tensor x [B,S,H,D] for sample b: out [S, D]. */
+static void gather_head(const job_t* J, const double* x, int H, int b, int h, int rot, double* out) {
+    osample s = make_sample(J->prefix[b], J->img_h[b], J->img_w[b], J->suffix[b]);
+    for (int64_t n = 0; n < J->S; ++n) {
+        const double* src = x + (((int64_t)b * J->S + n) * H + h) * J->D;
+        if (rot) rotate(&s, n, J->D, J->base, src, out + n * J->D);
+        else memcpy(out + n * J->D, src, sizeof(double) * J->D);
+    }
+}
+
+/* Forward for one (b, h): o [B,S,Hq,D], lse [B,Hq,S] (natural log of the sum
+ * of exp(scaled score)). */
+static void fwd_task(job_t* J, int b, int h) {
+    const int S = J->S, D = J->D, g = J->Hq / J->Hkv;
+    osample s = make_sample(J->prefix[b], J->img_h[b], J->img_w[b], J->suffix[b]);
+    double* qr = malloc(sizeof(double) * (size_t)S * D);
+    double* kr = malloc(sizeof(double) * (size_t)S * D);
+    double* vv = malloc(sizeof(double) * (size_t)S * D);
+    double* sc = malloc(sizeof(double) * (size_t)S);
+    gather_head(J, J->q, J->Hq, b, h, J->rotate_inputs, qr);
+    gather_head(J, J->k, J->Hkv, b, h / g, J->rotate_inputs, kr);
+    gather_head(J, J->v, J->Hkv, b, h / g, 0, vv);
+    int nr = J->rows ? J->n_rows : S;
+    for (int ri = 0; ri < nr; ++ri) {
+        int64_t q = J->rows ? J->rows[ri] : ri;
+        double m = -INFINITY;
+        for (int64_t k = 0; k < S; ++k) {
+            sc[k] = visible(&s, q, k) ? J->scale * dot(qr + q * D, kr + k * D, D) : -INFINITY;
+            if (sc[k] > m) m = sc[k];
+        }
+        double* orow = J->o + (((int64_t)b * S + q) * J->Hq + h) * D;
+        double* lrow = J->lse + ((int64_t)b * J->Hq + h) * S + q;
+        for (int d = 0; d < D; ++d) orow[d] = 0.0;
+        if (m == -INFINITY) { *lrow = -INFINITY; continue; }
+        double l = 0.0;
+        for (int64_t k = 0; k < S; ++k) {
+            if (sc[k] == -INFINITY) continue;
+            double p = exp(sc[k] - m);
+            l += p;
+            for (int d = 0; d < D; ++d) orow[d] += p * vv[k * D + d];
+        }
+        for (int d = 0; d < D; ++d) orow[d] /= l;
+        *lrow = m + log(l);
+    }
+    free(qr); free(kr); free(vv); free(sc);
+}
+
+/* Backward for one (b, h).  Recomputes the forward in fp64, then
+ *   dP = dO V^T,  Dq = dO . O,  dS = P (dP - Dq),
+ *   dQr = scale dS Kr,  dKr += scale dS^T Qr,  dV += P^T dO,
+ * and returns dQ = R^T dQr; dk_h/dv_h hold this head's R^T dKr and dV
+ * contributions (summed over the heads of a group by the caller). */
+static void bwd_task(job_t* J, int b, int h) {
+    const int S = J->S, D = J->D, g = J->Hq / J->Hkv;
+    osample s = make_sample(J->prefix[b], J->img_h[b], J->img_w[b], J->suffix[b]);
+    size_t SD = (size_t)S * D;
+    double* qr = malloc(sizeof(double) * SD);
+    double* kr = malloc(sizeof(double) * SD);
+    double* vv = malloc(sizeof(double) * SD);
+    double* dkr = calloc(SD, sizeof(double));
+    double* dvv = calloc(SD, sizeof(double));
+    double* dqr = malloc(sizeof(double) * D);
+    double* orow = malloc(sizeof(double) * D);
+    double* sc = malloc(sizeof(double) * (size_t)S);
+    gather_head(J, J->q, J->Hq, b, h, J->rotate_inputs, qr);
+    gather_head(J, J->k, J->Hkv, b, h / g, J->rotate_inputs, kr);
+    gather_head(J, J->v, J->Hkv, b, h / g, 0, vv);
+    for (int64_t q = 0; q < S; ++q) {
+        const double* dorow = J->dout + (((int64_t)b * S + q) * J->Hq + h) * D;
+        double* dqout = J->dq + (((int64_t)b * S + q) * J->Hq + h) * D;
+        double m = -INFINITY;
+        for (int64_t k = 0; k < S; ++k) {
+            sc[k] = visible(&s, q, k) ? J->scale * dot(qr + q * D, kr + k * D, D) : -INFINITY;
+            if (sc[k] > m) m = sc[k];
+        }
+        if (m == -INFINITY) { for (int d = 0; d < D; ++d) dqout[d] = 0.0; continue; }
+        double l = 0.0;
+        for (int d = 0; d < D; ++d) orow[d] = 0.0;
+        for (int64_t k = 0; k < S; ++k) {
+            if (sc[k] == -INFINITY) { sc[k] = 0.0; continue; }
+            sc[k] = exp(sc[k] - m);          /* unnormalised P */
+            l += sc[k];
+            for (int d = 0; d < D; ++d) orow[d] += sc[k] * vv[k * D + d];
+        }
+        for (int d = 0; d < D; ++d) orow[d] /= l;
+        double Dq = dot(dorow, orow, D);
+        for (int d = 0; d < D; ++d) dqr[d] = 0.0;
+        for (int64_t k = 0; k < S; ++k) {
+            if (sc[k] == 0.0) continue;
+            double p = sc[k] / l;
+            double dp = dot(dorow, vv + k * D, D);
+            double ds = p * (dp - Dq);
+            for (int d = 0; d < D; ++d) {
+                dqr[d] += J->scale * ds * kr[k * D + d];
+                dkr[k * D + d] += J->scale * ds * qr[q * D + d];
+                dvv[k * D + d] += p * dorow[d];
+            }
+        }
+        if (J->rotate_inputs) rotate_t(&s, q, D, J->base, dqr, dqout);
+        else memcpy(dqout, dqr, sizeof(double) * D);
+    }
+    for (int64_t k = 0; k < S; ++k) {
+        double* dko = J->dk_h + (((int64_t)b * S + k) * J->Hq + h) * D;
+        double* dvo = J->dv_h + (((int64_t)b * S + k) * J->Hq + h) * D;
+        if (J->rotate_inputs) rotate_t(&s, k, D, J->base, dkr + k * D, dko);
+        else memcpy(dko, dkr + k * D, sizeof(double) * D);
+        memcpy(dvo, dvv + k * D, sizeof(double) * D);
+    }
+    free(qr); free(kr); free(vv); free(dkr); free(dvv); free(dqr); free(orow); free(sc);
+}
+
+static int task_selected(const job_t* J, int t) {
+    int b = t / J->Hq, h = t % J->Hq, g = J->Hq / J->Hkv;
+    return J->group_sel == NULL || J->group_sel[b * J->Hkv + h / g];
+}
+
+typedef struct { job_t* J; int is_bwd; } worker_arg;
+
+static void* worker(void* p) {
+    worker_arg* a = (worker_arg*)p;
+    job_t* J = a->J;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int t = J->next_task++;
+        pthread_mutex_unlock(&J->lock);
+        if (t >= J->n_tasks) break;
+        if (!task_selected(J, t)) continue;
+        if (a->is_bwd) bwd_task(J, t / J->Hq, t % J->Hq);
+        else fwd_task(J, t / J->Hq, t % J->Hq);
+    }
+    return NULL;
+}
+
+static int run_job(job_t* J, int is_bwd, int nthreads) {
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 1024) nthreads = 1024;
+    J->n_tasks = J->B * J->Hq;
+    J->next_task = 0;
+    pthread_mutex_init(&J->lock, NULL);
+    pthread_t* th = malloc(sizeof(pthread_t) * nthreads);
+    worker_arg a = {J, is_bwd};
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, worker, &a);
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J->lock);
+    return nthreads;
+}
+
+static int check_geom(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
+                      const int32_t* img_h, const int32_t* img_w, const int32_t* suffix) {
+    if (B < 0 || S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || D % 2) return -1;
+    for (int b = 0; b < B; ++b) {
+        if (prefix[b] < 0 || img_h[b] < 0 || img_w[b] < 0 || suffix[b] < 0) return -1;
+        if ((img_h[b] == 0) != (img_w[b] == 0)) return -1;
+        if (make_sample(prefix[b], img_h[b], img_w[b], suffix[b]).L > S) return -1;
+    }
+    return 0;
+}
+
+/* Forward.  q [B,S,Hq,D], k, v [B,S,Hkv,D] (fp64, exact copies of the bf16
+ * inputs); o [B,S,Hq,D]; lse [B,Hq,S].  rows/n_rows restrict the query rows;
+ * group_sel [B*Hkv] restricts the (b, kv head) groups.  Returns the number of
+ * threads used, or -1 on bad arguments. */
+int oracle_attn_fwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
+                    const int32_t* img_h, const int32_t* img_w, const int32_t* suffix,
+                    const double* q, const double* k, const double* v, double scale,
+                    double base, int rotate_inputs, const int32_t* rows, int n_rows,
+                    const uint8_t* group_sel, double* o, double* lse, int nthreads) {
+    if (check_geom(B, S, Hq, Hkv, D, prefix, img_h, img_w, suffix)) return -1;
+    job_t J;
+    memset(&J, 0, sizeof(J));
+    J.B = B; J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.D = D;
+    J.prefix = prefix; J.img_h = img_h; J.img_w = img_w; J.suffix = suffix;
+    J.q = q; J.k = k; J.v = v; J.scale = scale; J.base = base;
+    J.rotate_inputs = rotate_inputs; J.rows = rows; J.n_rows = n_rows;
+    J.group_sel = group_sel; J.o = o; J.lse = lse;
+    return run_job(&J, 0, nthreads);
+}
+
+/* Backward.  dq [B,S,Hq,D]; dk, dv [B,S,Hkv,D].  group_sel as above (dq of
+ * unselected groups and their dk/dv are left untouched). */
+int oracle_attn_bwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
+                    const int32_t* img_h, const int32_t* img_w, const int32_t* suffix,
+                    const double* q, const double* k, const double* v, const double* dout,
+                    double scale, double base, int rotate_inputs, const uint8_t* group_sel,
+                    double* dq, double* dk, double* dv, int nthreads) {
+    if (check_geom(B, S, Hq, Hkv, D, prefix, img_h, img_w, suffix)) return -1;
+    size_t n = (size_t)B * S * Hq * D;
+    job_t J;
+    memset(&J, 0, sizeof(J));
+    J.B = B; J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.D = D;
+    J.prefix = prefix; J.img_h = img_h; J.img_w = img_w; J.suffix = suffix;
+    J.q = q; J.k = k; J.v = v; J.dout = dout; J.scale = scale; J.base = base;
+    J.rotate_inputs = rotate_inputs; J.group_sel = group_sel; J.dq = dq;
+    J.dk_h = calloc(n ? n : 1, sizeof(double));
+    J.dv_h = calloc(n ? n : 1, sizeof(double));
+    int used = run_job(&J, 1, nthreads);
+    int g = Hq / Hkv;
+    for (int b = 0; b < B; ++b)
+        for (int hk = 0; hk < Hkv; ++hk) {
+            if (group_sel && !group_sel[b * Hkv + hk]) continue;
+            for (int64_t s = 0; s < S; ++s)
+                for (int d = 0; d < D; ++d) {
+                    double ak = 0.0, av = 0.0;
+                    for (int i = 0; i < g; ++i) {
+                        int64_t o = (((int64_t)b * S + s) * Hq + hk * g + i) * D + d;
+                        ak += J.dk_h[o];
+                        av += J.dv_h[o];
+                    }
+                    dk[(((int64_t)b * S + s) * Hkv + hk) * D + d] = ak;
+                    dv[(((int64_t)b * S + s) * Hkv + hk) * D + d] = av;
+                }
+        }
+    free(J.dk_h);
+    free(J.dv_h);
+    return used;
+}
