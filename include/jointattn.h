@@ -1,0 +1,199 @@
+/*
+ * jointattn.h -- C ABI of libjointattn: the generalized-causal GQA
+ * self-attention of a unified text+image decoder (HunyuanImage-3.0), with the
+ * generalized 2D RoPE applied to Q and K, forward and recompute backward, for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Conventions for every entry point
+ *   - Return value: an hia_status (HIA_OK = 0).  All argument checks run on the
+ *     host before anything is launched; on error nothing is launched and no
+ *     output is touched.
+ *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *     default stream).  Every device call is asynchronous on that stream; the
+ *     library never synchronizes the device and never allocates inside
+ *     hia_attn_fwd / hia_attn_bwd (the caller passes the workspace).
+ *   - Ownership: the caller owns every device buffer (tensors, tables,
+ *     workspace).  The library owns only hia_segments objects, which the
+ *     caller frees with hia_segments_destroy.
+ *   - Dtypes: bf16 for q, k, v, o, dout, dq, dk, dv; fp32 for cos, sin, lse.
+ *   - Shapes: B samples, padded length S, Hq query heads, Hkv key/value heads
+ *     (Hq % Hkv == 0, g = Hq / Hkv query heads per kv head), head_dim D in
+ *     {64, 128}.
+ *
+ * Citations name the page title and the section or API item they come from.
+ */
+#ifndef JOINTATTN_H
+#define JOINTATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HIA_OK = 0,
+    HIA_ERR_INVALID_ARG = 1,    /* null pointer, negative size, bad geometry, short workspace */
+    HIA_ERR_UNSUPPORTED = 2,    /* D not in {64,128}, Hq % Hkv != 0, misaligned pointer/stride */
+    HIA_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed */
+    HIA_ERR_DEVICE_TIMEOUT = 4, /* a kernel's bounded wait expired (see hia_get_device_status) */
+    HIA_ERR_NOT_ON_DEVICE = 5   /* hia_segments used on the device before hia_segments_upload */
+} hia_status;
+
+/* One sample of the batch.  Layout (HunyuanImage-3.0 coverage page, Cache
+ * Contract; hunyuan_image3.model HunyuanImage3ForCausalMM.forward, input_ids):
+ *   [0, prefix_len)                 text, ending in the <timestep> token
+ *   [prefix_len, prefix_len + h*w)  image tokens, row-major (h, w) order
+ *   [.., L = prefix + h*w + suffix) suffix text (e.g. <eoi>)
+ *   [L, S)                          right padding
+ * img_h = img_w = 0 is a text-only sample.  Equivalent to the reference
+ * mask builder's arguments with image_starts = prefix_len, num_image_tokens =
+ * h*w (here allowed to differ per sample) and valid_lengths = L. */
+typedef struct {
+    int32_t prefix_len;
+    int32_t img_h;
+    int32_t img_w;
+    int32_t suffix_len;
+} hia_sample;
+
+/* A strided [B, S, heads, D] bf16 (or fp32) device tensor.  Strides are in
+ * elements; the last dimension is contiguous.  For a tensor with Hq heads,
+ * head h lives at ptr + (h / g) * stride_hkv + (h % g) * stride_hq, which
+ * covers both a plain [B,S,Hq,D] tensor (stride_hkv = g*D, stride_hq = D) and
+ * the fused KV-head-grouped QKV projection output [B,S,Hkv,g+2,D]
+ * (hunyuan_image3.layers HunyuanImage3Attention: per kv head, its g query
+ * heads then one key and one value head).  For a tensor with Hkv heads, head
+ * h lives at ptr + h * stride_hkv and stride_hq is ignored.  Every stride in
+ * bytes and the pointer must be multiples of 16. */
+typedef struct {
+    void* ptr;
+    int64_t stride_b;
+    int64_t stride_s;
+    int64_t stride_hkv;
+    int64_t stride_hq;
+} hia_tensor;
+
+/* Opaque segment descriptor, owned by the library. */
+typedef struct hia_segments hia_segments;
+
+/* Summary numbers of a descriptor. */
+typedef struct {
+    int32_t B, S;
+    int64_t visible_pairs;       /* sum over b and query rows q < S of (e_b(q) + 1) */
+    int32_t fwd_q_tiles;         /* ceil(S / 128) */
+    int32_t fwd_kv_tiles;        /* ceil(S / 128) */
+    int64_t fwd_tiles_full;      /* (b, q-tile, kv-tile) triples, 128 x 128 tiles */
+    int64_t fwd_tiles_partial;
+    int64_t fwd_tiles_skipped;   /* fully masked, incl. padded keys: never loaded */
+    int32_t bwd_q_tiles;         /* ceil(S / 64) */
+    int32_t bwd_kv_tiles;        /* ceil(S / 128) */
+} hia_segments_info_t;
+
+/* Tile classes reported by hia_segments_tile_classes. */
+enum {
+    HIA_TILE_SKIP = 0,       /* every pair masked (causal future or image-block edge) */
+    HIA_TILE_FULL = 1,       /* every pair visible: no predicate evaluated */
+    HIA_TILE_PARTIAL = 2,    /* mixed: per-pair predicate k <= e(q) in registers */
+    HIA_TILE_PADDED = 3      /* keys all at or beyond L (right padding): skipped */
+};
+
+/* Build the segment descriptor that replaces the dense [B,1,S,S] boolean
+ * mask (hunyuan_image3.model build_joint_attention_mask: causal text,
+ * bidirectional image span, padded keys masked out; technical report summary
+ * 3.1.2; paper review 3.3).  With I0 = prefix_len, I1 = I0 + h*w and
+ * L = I1 + suffix_len, key k is visible from query q iff k <= e(q) where
+ *   e(q) = min(L - 1, (I0 <= q < I1) ? I1 - 1 : q),
+ * a non-decreasing row bound (padded query rows see every real key).  From it
+ * the builder classifies every (q-tile, kv-tile) as FULL, PARTIAL or skipped
+ * and orders the work heaviest first.  Host only: no CUDA call is made.
+ * samples: host array of B entries.  S >= max L.  On success *out receives a
+ * new object.  Errors: HIA_ERR_INVALID_ARG (null, B < 0, S < 0, negative
+ * lengths, exactly one of img_h/img_w zero, L > S, S >= 2^24). */
+int hia_segments_build(const hia_sample* samples, int B, int S, hia_segments** out);
+
+/* Copy the per-sample bounds, tile tables and work lists to the current
+ * device (allocated once per object; asynchronous on `stream`).  Must
+ * precede hia_rope2d_tables / hia_attn_fwd / hia_attn_bwd. */
+int hia_segments_upload(hia_segments* seg, void* stream);
+
+/* Free the object and its device copies (the device copies are freed with
+ * cudaFree, which synchronizes).  NULL is a no-op. */
+void hia_segments_destroy(hia_segments* seg);
+
+int hia_segments_info(const hia_segments* seg, hia_segments_info_t* info);
+
+/* Host copies for tests and inspection.  row_bound: int32 [B, S] e_b(q)
+ * (-1 for a sample with L = 0).  mask: uint8 [B, S, S] (1 = visible) rendered
+ * from e, for a bit-exact comparison with the reference rule.  classes:
+ * uint8 [B, fwd_q_tiles, fwd_kv_tiles] with HIA_TILE_* values. */
+int hia_segments_row_bound(const hia_segments* seg, int32_t* row_bound);
+int hia_segments_mask(const hia_segments* seg, uint8_t* mask);
+int hia_segments_tile_classes(const hia_segments* seg, uint8_t* classes);
+
+/* Generalized 2D RoPE tables (paper review 3.4 and Figure 5; technical report
+ * summary 3.1.3): cos, sin fp32 [B, S, D] device buffers written on `stream`.
+ * Token n of a sample sits at (x, y) = (n, n) unless it is image token
+ * i = n - I0, which sits at x = I0 + (i % w), y = I0 + (i / w).  For
+ * j < D/2, angle_j = (j even ? x : y) * base^(-2j/D), and
+ * cos[b,n,j] = cos[b,n,j+D/2] = cos(angle_j), likewise sin (the cos block /
+ * sin block layout of the [B, S, head_dim] tables taken by
+ * HunyuanImage3Attention.forward).  Angles and cos/sin are evaluated in fp64
+ * and rounded once to fp32, so a text-only sample gives exactly the 1D RoPE
+ * tables.  D even, 2 <= D <= 256, base > 0. */
+int hia_rope2d_tables(const hia_segments* seg, int D, double base, float* cos_out,
+                      float* sin_out, void* stream);
+
+/* Bytes of device workspace hia_attn_fwd needs (256-byte aligned pointer). */
+size_t hia_attn_fwd_workspace_bytes(const hia_segments* seg, int Hq, int Hkv, int D);
+
+/* Forward of the masked GQA attention with RoPE applied to q and k
+ * (HunyuanImage3Attention.forward: q_r = q*cos + rotate_half(q)*sin, the same
+ * for k; rotate_half(v) = [-v[D/2:], v[:D/2]]; v is not rotated; scores
+ * scale * q_r . k_r over visible pairs; softmax; output P v).
+ *   q [B,S,Hq,D], k, v [B,S,Hkv,D], o [B,S,Hq,D] (bf16, hia_tensor strides);
+ *   cos, sin fp32 [B,S,D] (from hia_rope2d_tables or the caller's own);
+ *   lse fp32 [B,Hq,S] contiguous: natural-log sum of exp(scaled scores) per
+ *   row (-inf, with o = 0, for a row with no visible key, i.e. L = 0);
+ *   scale: usually 1/sqrt(D).  Padded query rows are computed like any row.
+ * Q and K are rotated once into the workspace (bf16, [B,H,S,D]) by a
+ * bandwidth-bound pre-pass; the attention kernel streams them with TMA into
+ * tcgen05 MMAs.  Errors: HIA_ERR_INVALID_ARG, HIA_ERR_UNSUPPORTED,
+ * HIA_ERR_NOT_ON_DEVICE, HIA_ERR_CUDA (launch failure). */
+int hia_attn_fwd(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                 hia_tensor v, const float* cos_t, const float* sin_t, float scale,
+                 hia_tensor o, float* lse, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/* Bytes of device workspace hia_attn_bwd needs. */
+size_t hia_attn_bwd_workspace_bytes(const hia_segments* seg, int Hq, int Hkv, int D);
+
+/* Recompute backward of hia_attn_fwd: given o and lse from the forward and
+ * dout = dL/do, writes dq [B,S,Hq,D], dk, dv [B,S,Hkv,D] (bf16), i.e. the
+ * gradients w.r.t. the un-rotated q and k (dq = R^T dq_r, dk = R^T dk_r) and
+ * v, summed over the g query heads of each kv head.  Same conventions and
+ * errors as hia_attn_fwd. */
+int hia_attn_bwd(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                 hia_tensor v, const float* cos_t, const float* sin_t, float scale,
+                 hia_tensor o, const float* lse, hia_tensor dout, hia_tensor dq,
+                 hia_tensor dk, hia_tensor dv, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/* Read and clear the device status word of the current device (synchronizes
+ * `stream`).  Returns HIA_OK, HIA_ERR_DEVICE_TIMEOUT if any kernel's bounded
+ * wait expired since the last call, or HIA_ERR_CUDA. */
+int hia_get_device_status(void* stream);
+
+/* Test hook for the bounded-wait machinery: launches one block that waits on
+ * an mbarrier nothing ever arrives on, with the given limit in nanoseconds;
+ * the wait expires, records HIA_ERR_DEVICE_TIMEOUT in the status word and the
+ * kernel returns normally.  timeout_ns in [1, 10^9]. */
+int hia_debug_wait_timeout(uint64_t timeout_ns, void* stream);
+
+const char* hia_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JOINTATTN_H */

@@ -1,0 +1,259 @@
+"""libjointattn: generalized-causal GQA attention with generalized 2D RoPE
+(HunyuanImage-3.0) for B200 / sm_100a.
+
+Thin ctypes binding over the C ABI in ``include/jointattn.h``: these functions
+only marshal arguments (torch tensors -> pointers and strides, the current
+torch CUDA stream); every step runs in the library's CUDA kernels.  There is no
+CPU fallback: if ``libjointattn.so`` is missing or fails to load, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "HiaError", "Segments", "lib", "hia_segments_build", "hia_rope2d_tables", "hia_attn_fwd",
+    "hia_attn_bwd", "hia_attn_fwd_workspace_bytes", "hia_attn_bwd_workspace_bytes",
+    "hia_get_device_status", "hia_debug_wait_timeout", "LIB_PATH", "EXPORTED_SYMBOLS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libjointattn.so")
+
+EXPORTED_SYMBOLS = (
+    "hia_segments_build", "hia_segments_upload", "hia_segments_destroy", "hia_segments_info",
+    "hia_segments_row_bound", "hia_segments_mask", "hia_segments_tile_classes", "hia_rope2d_tables",
+    "hia_attn_fwd_workspace_bytes", "hia_attn_fwd", "hia_attn_bwd_workspace_bytes", "hia_attn_bwd",
+    "hia_get_device_status", "hia_debug_wait_timeout", "hia_status_string",
+)
+
+
+class HiaError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__(f"{what}: {_status_string(code)} (status {code})")
+
+
+class _Sample(ctypes.Structure):
+    _fields_ = [("prefix_len", ctypes.c_int32), ("img_h", ctypes.c_int32),
+                ("img_w", ctypes.c_int32), ("suffix_len", ctypes.c_int32)]
+
+
+class _Tensor(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("stride_b", ctypes.c_int64), ("stride_s", ctypes.c_int64),
+                ("stride_hkv", ctypes.c_int64), ("stride_hq", ctypes.c_int64)]
+
+
+class SegmentsInfo(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("S", ctypes.c_int32), ("visible_pairs", ctypes.c_int64),
+                ("fwd_q_tiles", ctypes.c_int32), ("fwd_kv_tiles", ctypes.c_int32),
+                ("fwd_tiles_full", ctypes.c_int64), ("fwd_tiles_partial", ctypes.c_int64),
+                ("fwd_tiles_skipped", ctypes.c_int64), ("bwd_q_tiles", ctypes.c_int32),
+                ("bwd_kv_tiles", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libjointattn.so (raises if it is missing: no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
+                              "or python joint_text_image_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, Z, T = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, _Tensor
+        L.hia_segments_build.argtypes = [ctypes.POINTER(_Sample), I, I, ctypes.POINTER(P)]
+        L.hia_segments_upload.argtypes = [P, P]
+        L.hia_segments_destroy.argtypes = [P]
+        L.hia_segments_destroy.restype = None
+        L.hia_segments_info.argtypes = [P, ctypes.POINTER(SegmentsInfo)]
+        L.hia_segments_row_bound.argtypes = [P, P]
+        L.hia_segments_mask.argtypes = [P, P]
+        L.hia_segments_tile_classes.argtypes = [P, P]
+        L.hia_rope2d_tables.argtypes = [P, I, ctypes.c_double, P, P, P]
+        L.hia_attn_fwd_workspace_bytes.argtypes = [P, I, I, I]
+        L.hia_attn_fwd_workspace_bytes.restype = Z
+        L.hia_attn_bwd_workspace_bytes.argtypes = [P, I, I, I]
+        L.hia_attn_bwd_workspace_bytes.restype = Z
+        L.hia_attn_fwd.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, T, P, P, Z, P]
+        L.hia_attn_bwd.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, T, P, T, T, T, T, P, Z, P]
+        L.hia_get_device_status.argtypes = [P]
+        L.hia_debug_wait_timeout.argtypes = [ctypes.c_uint64, P]
+        L.hia_status_string.argtypes = [I]
+        L.hia_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _status_string(code):
+    try:
+        return lib().hia_status_string(int(code)).decode()
+    except Exception:  # library missing: still report the code
+        return "status"
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise HiaError(rc, what)
+
+
+def _stream(device=None):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+class Segments:
+    """Owner of a library hia_segments object (host tables + device copies)."""
+
+    def __init__(self, samples, S):
+        arr = (_Sample * max(1, len(samples)))(*[_Sample(*map(int, s)) for s in samples])
+        h = ctypes.c_void_p()
+        _check(lib().hia_segments_build(arr, len(samples), int(S), ctypes.byref(h)), "hia_segments_build")
+        self.handle = h
+        self.samples = [tuple(map(int, s)) for s in samples]
+        self.B, self.S = len(samples), int(S)
+        self.on_device = False
+
+    def upload(self):
+        _check(lib().hia_segments_upload(self.handle, _stream()), "hia_segments_upload")
+        self.on_device = True
+        return self
+
+    def info(self) -> SegmentsInfo:
+        out = SegmentsInfo()
+        _check(lib().hia_segments_info(self.handle, ctypes.byref(out)), "hia_segments_info")
+        return out
+
+    def row_bound(self):
+        import numpy as np
+        e = np.zeros((self.B, self.S), dtype=np.int32)
+        _check(lib().hia_segments_row_bound(self.handle, e.ctypes.data_as(ctypes.c_void_p)), "row_bound")
+        return e
+
+    def mask(self):
+        import numpy as np
+        m = np.zeros((self.B, self.S, self.S), dtype=np.uint8)
+        _check(lib().hia_segments_mask(self.handle, m.ctypes.data_as(ctypes.c_void_p)), "mask")
+        return m
+
+    def tile_classes(self):
+        import numpy as np
+        inf = self.info()
+        c = np.zeros((self.B, inf.fwd_q_tiles, inf.fwd_kv_tiles), dtype=np.uint8)
+        _check(lib().hia_segments_tile_classes(self.handle, c.ctypes.data_as(ctypes.c_void_p)), "tile_classes")
+        return c
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.hia_segments_destroy(h)
+            self.handle = None
+
+
+def hia_segments_build(samples, S, upload=True) -> Segments:
+    """Segment descriptor for samples [(prefix, img_h, img_w, suffix)] padded to S."""
+    seg = Segments(samples, S)
+    return seg.upload() if upload else seg
+
+
+def _t(x, q_heads, g):
+    """hia_tensor from a [B,S,H,D] torch view (or a [B,S,Hkv,g+2,D] fused slice)."""
+    if x is None:
+        return _Tensor(None, 0, 0, 0, 0)
+    if x.dim() == 4:
+        sb, ss, sh, sd = x.stride()
+        if sd != 1:
+            raise ValueError("last dimension must be contiguous")
+        return _Tensor(x.data_ptr(), sb, ss, sh * g if q_heads else sh, sh if q_heads else 0)
+    if x.dim() == 5:  # [B, S, Hkv, g, D] grouped view
+        sb, ss, shkv, shq, sd = x.stride()
+        if sd != 1:
+            raise ValueError("last dimension must be contiguous")
+        return _Tensor(x.data_ptr(), sb, ss, shkv, shq)
+    raise ValueError("expected a 4-D [B,S,H,D] or 5-D [B,S,Hkv,g,D] tensor")
+
+
+def _heads(x):
+    return x.shape[2] * (x.shape[3] if x.dim() == 5 else 1)
+
+
+def hia_rope2d_tables(seg: Segments, D: int, base: float = 10000.0, out=None):
+    """fp32 cos, sin [B, S, D] on the current CUDA device."""
+    import torch
+    if out is None:
+        out = (torch.empty(seg.B, seg.S, D, device="cuda", dtype=torch.float32),
+               torch.empty(seg.B, seg.S, D, device="cuda", dtype=torch.float32))
+    c, s = out
+    _check(lib().hia_rope2d_tables(seg.handle, int(D), float(base), c.data_ptr(), s.data_ptr(), _stream()),
+           "hia_rope2d_tables")
+    return c, s
+
+
+def hia_attn_fwd_workspace_bytes(seg: Segments, Hq, Hkv, D):
+    return int(lib().hia_attn_fwd_workspace_bytes(seg.handle, Hq, Hkv, D))
+
+
+def hia_attn_bwd_workspace_bytes(seg: Segments, Hq, Hkv, D):
+    return int(lib().hia_attn_bwd_workspace_bytes(seg.handle, Hq, Hkv, D))
+
+
+def _ws(nbytes, workspace):
+    import torch
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError("workspace too small")
+        return workspace
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device="cuda")
+
+
+def hia_attn_fwd(seg: Segments, q, k, v, cos, sin, scale=None, o=None, lse=None, workspace=None):
+    """Forward.  q [B,S,Hq,D], k, v [B,S,Hkv,D] bf16 CUDA tensors (or grouped
+    5-D views).  Returns (o [B,S,Hq,D] bf16, lse [B,Hq,S] fp32)."""
+    import torch
+    Hq, Hkv, D = _heads(q), _heads(k), q.shape[-1]
+    g = Hq // Hkv
+    if scale is None:
+        scale = D ** -0.5
+    if o is None:
+        o = torch.empty(seg.B, seg.S, Hq, D, device=q.device, dtype=torch.bfloat16)
+    if lse is None:
+        lse = torch.empty(seg.B, Hq, seg.S, device=q.device, dtype=torch.float32)
+    nb = hia_attn_fwd_workspace_bytes(seg, Hq, Hkv, D)
+    ws = _ws(nb, workspace)
+    _check(lib().hia_attn_fwd(seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1),
+                              cos.data_ptr(), sin.data_ptr(), float(scale), _t(o, True, g), lse.data_ptr(),
+                              ws.data_ptr(), nb, _stream()), "hia_attn_fwd")
+    return o, lse
+
+
+def hia_attn_bwd(seg: Segments, q, k, v, cos, sin, o, lse, dout, scale=None, dq=None, dk=None, dv=None,
+                 workspace=None):
+    """Recompute backward.  Returns (dq, dk, dv) bf16."""
+    import torch
+    Hq, Hkv, D = _heads(q), _heads(k), q.shape[-1]
+    g = Hq // Hkv
+    if scale is None:
+        scale = D ** -0.5
+    if dq is None:
+        dq = torch.empty(seg.B, seg.S, Hq, D, device=q.device, dtype=torch.bfloat16)
+    if dk is None:
+        dk = torch.empty(seg.B, seg.S, Hkv, D, device=q.device, dtype=torch.bfloat16)
+    if dv is None:
+        dv = torch.empty(seg.B, seg.S, Hkv, D, device=q.device, dtype=torch.bfloat16)
+    nb = hia_attn_bwd_workspace_bytes(seg, Hq, Hkv, D)
+    ws = _ws(nb, workspace)
+    _check(lib().hia_attn_bwd(seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1),
+                              cos.data_ptr(), sin.data_ptr(), float(scale), _t(o, True, g), lse.data_ptr(),
+                              _t(dout, True, g), _t(dq, True, g), _t(dk, False, 1), _t(dv, False, 1),
+                              ws.data_ptr(), nb, _stream()), "hia_attn_bwd")
+    return dq, dk, dv
+
+
+def hia_get_device_status():
+    return int(lib().hia_get_device_status(_stream()))
+
+
+def hia_debug_wait_timeout(timeout_ns: int):
+    _check(lib().hia_debug_wait_timeout(int(timeout_ns), _stream()), "hia_debug_wait_timeout")

@@ -1,0 +1,326 @@
+// api.cu -- the C ABI of libjointattn: argument checks, device copies of the
+// segment descriptor, TMA tensor maps, workspace layout and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.h"
+
+namespace {
+
+using hia::SampleDev;
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per barrier wait
+
+__device__ int g_status;  // per-device status word (HIA_OK or HIA_ERR_DEVICE_TIMEOUT)
+
+int* status_ptr() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static std::mutex mu;
+  static int* ptrs[64] = {};
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle and a box of 64 x rows along dims 0/`row_dim`.
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+              const uint32_t* box) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[5], s[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) s[i] = strides_bytes[i];
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cuuint32_t(rank), const_cast<void*>(base), d, s, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows = S][D] per (b, head) slab of a [B*H][S][D] workspace tensor.
+bool make_ws_map(CUtensorMap* m, const void* base, int D, int S, int BH) {
+  uint64_t dims[3] = {uint64_t(D), uint64_t(S), uint64_t(BH)};
+  uint64_t st[2] = {uint64_t(D) * 2, uint64_t(S) * D * 2};
+  uint32_t box[3] = {64, 128, 1};
+  return make_map(m, base, 3, dims, st, box);
+}
+
+// User tensor with Hkv heads: dims (D, Hkv, S, B), box rows along S.
+bool make_kv_map(CUtensorMap* m, const hia_tensor& t, int D, int Hkv, int S, int B, uint32_t rows) {
+  uint64_t dims[4] = {uint64_t(D), uint64_t(Hkv), uint64_t(S), uint64_t(B)};
+  uint64_t st[3] = {uint64_t(t.stride_hkv) * 2, uint64_t(t.stride_s) * 2, uint64_t(t.stride_b) * 2};
+  uint32_t box[4] = {64, 1, rows, 1};
+  return make_map(m, t.ptr, 4, dims, st, box);
+}
+
+// User tensor with Hq heads: dims (D, g, Hkv, S, B), box rows along S.
+bool make_q_map(CUtensorMap* m, const hia_tensor& t, int D, int g, int Hkv, int S, int B, uint32_t rows) {
+  uint64_t dims[5] = {uint64_t(D), uint64_t(g), uint64_t(Hkv), uint64_t(S), uint64_t(B)};
+  uint64_t st[4] = {uint64_t(t.stride_hq) * 2, uint64_t(t.stride_hkv) * 2, uint64_t(t.stride_s) * 2,
+                    uint64_t(t.stride_b) * 2};
+  uint32_t box[5] = {64, 1, 1, rows, 1};
+  return make_map(m, t.ptr, 5, dims, st, box);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Checks shared by fwd and bwd.  heads_g: g for Hq-head tensors, 1 for Hkv-head tensors.
+int check_tensor(const hia_tensor& t, bool q_heads, int B, int S, int g) {
+  if (!t.ptr) return (B == 0 || S == 0) ? HIA_OK : HIA_ERR_INVALID_ARG;
+  if (t.stride_b < 0 || t.stride_s < 0 || t.stride_hkv < 0 || t.stride_hq < 0) return HIA_ERR_INVALID_ARG;
+  if (!aligned16(t.ptr)) return HIA_ERR_UNSUPPORTED;
+  if ((t.stride_b * 2) % 16 || (t.stride_s * 2) % 16 || (t.stride_hkv * 2) % 16) return HIA_ERR_UNSUPPORTED;
+  if (q_heads && g > 1 && (t.stride_hq * 2) % 16) return HIA_ERR_UNSUPPORTED;
+  return HIA_OK;
+}
+
+int check_common(const hia_segments* seg, int Hq, int Hkv, int D, const float* c, const float* s) {
+  if (!seg || Hq <= 0 || Hkv <= 0) return HIA_ERR_INVALID_ARG;
+  if (Hq % Hkv) return HIA_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return HIA_ERR_UNSUPPORTED;
+  if (seg->B == 0 || seg->S == 0) return HIA_OK;
+  if (!c || !s) return HIA_ERR_INVALID_ARG;
+  if (!aligned16(c) || !aligned16(s)) return HIA_ERR_UNSUPPORTED;
+  if (seg->device < 0) return HIA_ERR_NOT_ON_DEVICE;
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != seg->device) return HIA_ERR_NOT_ON_DEVICE;
+  return HIA_OK;
+}
+
+struct FwdWs {
+  size_t q_off, k_off, total;
+};
+FwdWs fwd_ws(const hia_segments* seg, int Hq, int Hkv, int D) {
+  FwdWs w{};
+  const size_t BS = size_t(seg->B) * seg->S;
+  w.q_off = 0;
+  w.k_off = align256(BS * Hq * D * 2);
+  w.total = w.k_off + align256(BS * Hkv * D * 2);
+  return w;
+}
+
+int S_pad64(int S) { return (S + 63) / 64 * 64; }
+
+struct BwdWs {
+  size_t q_off, k_off, lse_off, delta_off, dq_off, total;
+};
+BwdWs bwd_ws(const hia_segments* seg, int Hq, int Hkv, int D) {
+  BwdWs w{};
+  const size_t BS = size_t(seg->B) * seg->S;
+  const size_t BSp = size_t(seg->B) * S_pad64(seg->S);
+  w.q_off = 0;
+  w.k_off = align256(BS * Hq * D * 2);
+  w.lse_off = w.k_off + align256(BS * Hkv * D * 2);
+  w.delta_off = w.lse_off + align256(BSp * Hq * 4);
+  w.dq_off = w.delta_off + align256(BSp * Hq * 4);
+  w.total = w.dq_off + align256(BSp * Hq * D * 4);
+  return w;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? HIA_OK : HIA_ERR_CUDA; }
+
+void rotate_into(const hia_tensor& src, int H, int g, const float* c, const float* s, __nv_bfloat16* dst,
+                 const hia_segments* seg, int D, cudaStream_t st) {
+  hia::RotateArgs a{};
+  a.src = src.ptr;
+  a.src_sb = src.stride_b;
+  a.src_ss = src.stride_s;
+  a.src_shkv = src.stride_hkv;
+  a.src_shq = src.stride_hq;
+  a.g = g;
+  a.cos_t = c;
+  a.sin_t = s;
+  a.dst = dst;
+  a.B = seg->B;
+  a.S = seg->S;
+  a.H = H;
+  hia::launch_rope_rotate(a, D, st);
+}
+
+}  // namespace
+
+extern "C" int hia_segments_upload(hia_segments* g, void* stream) {
+  if (!g) return HIA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HIA_ERR_CUDA;
+  if (g->dbuf && g->device != dev) return HIA_ERR_INVALID_ARG;
+  const size_t n_s = g->samples.size() * sizeof(SampleDev);
+  const size_t n_ft = g->fwd_tiles.size() * 4, n_fw = g->fwd_work.size() * 4;
+  const size_t n_bt = g->bwd_tiles.size() * 4, n_bw = g->bwd_work.size() * 4;
+  const size_t o_s = 0, o_ft = align256(n_s), o_fw = o_ft + align256(n_ft), o_bt = o_fw + align256(n_fw),
+               o_bw = o_bt + align256(n_bt), total = o_bw + align256(n_bw) + 256;
+  if (!g->dbuf) {
+    if (cudaMalloc(&g->dbuf, total) != cudaSuccess) {
+      g->dbuf = nullptr;
+      return HIA_ERR_CUDA;
+    }
+  }
+  char* base = static_cast<char*>(g->dbuf);
+  cudaError_t e = cudaSuccess;
+  if (n_s) e = cudaMemcpyAsync(base + o_s, g->samples.data(), n_s, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && n_ft) e = cudaMemcpyAsync(base + o_ft, g->fwd_tiles.data(), n_ft, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && n_fw) e = cudaMemcpyAsync(base + o_fw, g->fwd_work.data(), n_fw, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && n_bt) e = cudaMemcpyAsync(base + o_bt, g->bwd_tiles.data(), n_bt, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && n_bw) e = cudaMemcpyAsync(base + o_bw, g->bwd_work.data(), n_bw, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return HIA_ERR_CUDA;
+  g->device = dev;
+  g->d_samples = reinterpret_cast<const SampleDev*>(base + o_s);
+  g->d_fwd_tiles = reinterpret_cast<const int32_t*>(base + o_ft);
+  g->d_fwd_work = reinterpret_cast<const int32_t*>(base + o_fw);
+  g->d_bwd_tiles = reinterpret_cast<const int32_t*>(base + o_bt);
+  g->d_bwd_work = reinterpret_cast<const int32_t*>(base + o_bw);
+  return HIA_OK;
+}
+
+extern "C" void hia_segments_destroy(hia_segments* g) {
+  if (!g) return;
+  if (g->dbuf) {
+    int cur = 0;
+    cudaGetDevice(&cur);
+    if (cur != g->device) cudaSetDevice(g->device);
+    cudaFree(g->dbuf);
+    if (cur != g->device) cudaSetDevice(cur);
+  }
+  delete g;
+}
+
+extern "C" int hia_rope2d_tables(const hia_segments* g, int D, double base, float* c, float* s, void* stream) {
+  if (!g || D < 2 || D > 256 || (D & 1) || !(base > 0.0) || !std::isfinite(base)) return HIA_ERR_INVALID_ARG;
+  if (g->B == 0 || g->S == 0) return HIA_OK;
+  if (!c || !s) return HIA_ERR_INVALID_ARG;
+  if (g->device < 0) return HIA_ERR_NOT_ON_DEVICE;
+  hia::launch_rope2d_tables(g->d_samples, g->B, g->S, D, base, c, s, static_cast<cudaStream_t>(stream));
+  return cuda_status(cudaGetLastError());
+}
+
+extern "C" size_t hia_attn_fwd_workspace_bytes(const hia_segments* g, int Hq, int Hkv, int D) {
+  if (!g || Hq <= 0 || Hkv <= 0 || D <= 0) return 0;
+  return fwd_ws(g, Hq, Hkv, D).total;
+}
+
+extern "C" size_t hia_attn_bwd_workspace_bytes(const hia_segments* g, int Hq, int Hkv, int D) {
+  if (!g || Hq <= 0 || Hkv <= 0 || D <= 0) return 0;
+  return bwd_ws(g, Hq, Hkv, D).total;
+}
+
+extern "C" int hia_attn_fwd(const hia_segments* g, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                            hia_tensor v, const float* c, const float* s, float scale, hia_tensor o, float* lse,
+                            void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_common(g, Hq, Hkv, D, c, s);
+  if (rc) return rc;
+  if (g->B == 0 || g->S == 0) return HIA_OK;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return HIA_ERR_INVALID_ARG;
+  const int gq = Hq / Hkv;
+  if ((rc = check_tensor(q, true, g->B, g->S, gq)) || (rc = check_tensor(k, false, g->B, g->S, 1)) ||
+      (rc = check_tensor(v, false, g->B, g->S, 1)) || (rc = check_tensor(o, true, g->B, g->S, gq)))
+    return rc;
+  if (!q.ptr || !k.ptr || !v.ptr || !o.ptr || !lse || !ws) return HIA_ERR_INVALID_ARG;
+  const FwdWs w = fwd_ws(g, Hq, Hkv, D);
+  if (ws_bytes < w.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return HIA_ERR_INVALID_ARG;
+  int* status = status_ptr();
+  if (!status) return HIA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* wb = static_cast<char*>(ws);
+  __nv_bfloat16* qr = reinterpret_cast<__nv_bfloat16*>(wb + w.q_off);
+  __nv_bfloat16* kr = reinterpret_cast<__nv_bfloat16*>(wb + w.k_off);
+
+  CUtensorMap tq, tk, tv;
+  if (!make_ws_map(&tq, qr, D, g->S, g->B * Hq) || !make_ws_map(&tk, kr, D, g->S, g->B * Hkv) ||
+      !make_kv_map(&tv, v, D, Hkv, g->S, g->B, 128))
+    return HIA_ERR_CUDA;
+
+  rotate_into(q, Hq, gq, c, s, qr, g, D, st);
+  rotate_into(k, Hkv, 1, c, s, kr, g, D, st);
+
+  hia::FwdParams p{};
+  p.samples = g->d_samples;
+  p.tiles = g->d_fwd_tiles;
+  p.work = g->d_fwd_work;
+  p.B = g->B;
+  p.S = g->S;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.g = gq;
+  p.nQT = g->nQT;
+  p.n_hp = (gq + 1) / 2;
+  p.o = static_cast<__nv_bfloat16*>(o.ptr);
+  p.o_sb = o.stride_b;
+  p.o_ss = o.stride_s;
+  p.o_shkv = o.stride_hkv;
+  p.o_shq = o.stride_hq;
+  p.lse = lse;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  const int64_t n_blocks = int64_t(g->B) * g->nQT * Hkv * p.n_hp;
+  if (n_blocks > (1ll << 31) - 1) return HIA_ERR_UNSUPPORTED;
+  return cuda_status(hia::launch_attn_fwd(tq, tk, tv, p, int(n_blocks), D, st));
+}
+
+extern "C" int hia_get_device_status(void* stream) {
+  int* sp = status_ptr();
+  if (!sp) return HIA_ERR_CUDA;
+  int h = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, sp, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return HIA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return HIA_ERR_CUDA;
+  if (h != 0) {
+    const int z = 0;
+    if (cudaMemcpyAsync(sp, &z, sizeof(int), cudaMemcpyHostToDevice, st) != cudaSuccess) return HIA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return HIA_ERR_CUDA;
+  }
+  return h == 0 ? HIA_OK : HIA_ERR_DEVICE_TIMEOUT;
+}
+
+extern "C" int hia_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
+  if (timeout_ns < 1 || timeout_ns > 1000000000ull) return HIA_ERR_INVALID_ARG;
+  int* sp = status_ptr();
+  if (!sp) return HIA_ERR_CUDA;
+  return cuda_status(hia::launch_wait_probe(sp, timeout_ns, static_cast<cudaStream_t>(stream)));
+}
+
+extern "C" int hia_attn_bwd(const hia_segments* g, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                            hia_tensor v, const float* c, const float* s, float scale, hia_tensor o,
+                            const float* lse, hia_tensor dout, hia_tensor dq, hia_tensor dk, hia_tensor dv,
+                            void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_common(g, Hq, Hkv, D, c, s);
+  if (rc) return rc;
+  if (g->B == 0 || g->S == 0) return HIA_OK;
+  (void)q; (void)k; (void)v; (void)scale; (void)o; (void)lse; (void)dout; (void)dq; (void)dk; (void)dv;
+  (void)ws; (void)ws_bytes; (void)stream;
+  return HIA_ERR_UNSUPPORTED;
+}

@@ -1,0 +1,319 @@
+// attn_fwd.cu -- forward of the generalized-causal GQA attention on sm_100a.
+//
+// Definition (hunyuan_image3.layers HunyuanImage3Attention.forward with the
+// mask of hunyuan_image3.model build_joint_attention_mask): for every query
+// row q and head h, O = softmax(scale * q_r . k_r over visible keys) V with
+// q_r, k_r the RoPE-rotated rows and kv head h / g (grouped QKV).
+//
+// One CTA owns 128 query rows of two query heads of the same kv head (two
+// M = 128 tiles), so every K/V tile it streams feeds two MMAs.  It walks the
+// kv tiles the segment builder marked visible for that query tile: FULL tiles
+// run without a mask, PARTIAL ones apply the predicate k <= e(q) in
+// registers, fully masked and padded tiles are never loaded.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q tiles once, then K/V tiles into a 2-stage ring
+//   warp 1      TMEM owner and single-thread tcgen05.mma issuer
+//   warps 4-7   softmax / correction / epilogue of tile 0 (one row per thread)
+//   warps 8-11  the same for tile 1
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 after it;
+// P_t is written as packed bf16 over the first 64 columns of S_t and fed to
+// the PV MMA straight from TMEM.  MMA order per kv tile j:
+//   PV0(j), QK0(j+1), PV1(j), QK1(j+1)
+// so the commit that publishes S_t(j+1) also proves PV_t(j) finished: the
+// softmax warps may then rescale O_t and overwrite P_t without extra barriers.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace hia {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kTileElems = 128 * D;
+  alignas(1024) __nv_bfloat16 q[2][kTileElems];
+  alignas(1024) __nv_bfloat16 k[2][kTileElems];
+  alignas(1024) __nv_bfloat16 v[2][kTileElems];
+  uint64_t bar_q;
+  uint64_t bar_k_full[2];
+  uint64_t bar_v_full[2];
+  uint64_t bar_kv_empty[2];
+  uint64_t bar_s_full[2];
+  uint64_t bar_p_ready[2];
+  uint64_t bar_o_final[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t tS, const __nv_bfloat16* q, const __nv_bfloat16* k) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+  const uint32_t qa = smem_u32(q), ka = smem_u32(k);
+#pragma unroll
+  for (int kb = 0; kb < D / 16; ++kb) {
+    const uint32_t off = uint32_t(kb >> 2) * 16384u + uint32_t(kb & 3) * 32u;
+    mma_ss(tS, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc, kb > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, const __nv_bfloat16* v, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+  const uint32_t va = smem_u32(v);
+#pragma unroll
+  for (int kb = 0; kb < 8; ++kb) {
+    // V tile: [128 keys][D], 64-wide D blocks 16 KB apart; 16 keys = 2 KB.
+    const uint64_t bd = sdesc_sw128(va + uint32_t(kb) * 2048u, 16384, 1024);
+    mma_ts(tO, tP + uint32_t(kb) * 8u, bd, idesc, (accumulate || kb > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  FwdSmem<D>& sm =
+      *reinterpret_cast<FwdSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work item: (b, q tile) heaviest first, then kv head, then head pair
+  int bid = blockIdx.x;
+  const int hp = bid % p.n_hp;
+  bid /= p.n_hp;
+  const int hkv = bid % p.Hkv;
+  bid /= p.Hkv;
+  const int b = p.work[2 * bid], qt = p.work[2 * bid + 1];
+  const int n_full = p.tiles[2 * (b * p.nQT + qt)];
+  const int n_vis = p.tiles[2 * (b * p.nQT + qt) + 1];
+  const int h0 = hkv * p.g + 2 * hp;
+  const int n_tiles = (2 * hp + 1 < p.g) ? 2 : 1;
+  const SampleDev smp = p.samples[b];
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.bar_k_full[i], 1);
+      mbar_init(&sm.bar_v_full[i], 1);
+      mbar_init(&sm.bar_kv_empty[i], 1);
+      mbar_init(&sm.bar_s_full[i], 1);
+      mbar_init(&sm.bar_p_ready[i], 128);
+      mbar_init(&sm.bar_o_final[i], 1);
+    }
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtx wc{&sm.abort_flag, p.status, p.timeout_ns};
+
+  if (warp == 0) {
+    // =============================== TMA producer
+    if (lane == 0 && n_vis > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      constexpr uint32_t tile_bytes = 128 * D * 2;
+      mbar_arrive_expect_tx(&sm.bar_q, tile_bytes * n_tiles);
+      for (int t = 0; t < n_tiles; ++t)
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(&sm.q[t][c * 128 * 64], &tm_q, &sm.bar_q, c * 64, qt * 128, b * p.Hq + h0 + t);
+      int issued = 0;
+      for (int j = 0; j < n_vis; ++j) {
+        const int s = j & 1;
+        if (j >= 2 && !mbar_wait(&sm.bar_kv_empty[s], ((j >> 1) - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&sm.bar_k_full[s], tile_bytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(&sm.k[s][c * 128 * 64], &tm_k, &sm.bar_k_full[s], c * 64, j * 128, b * p.Hkv + hkv);
+        mbar_arrive_expect_tx(&sm.bar_v_full[s], tile_bytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(&sm.v[s][c * 128 * 64], &tm_v, &sm.bar_v_full[s], c * 64, hkv, j * 128, b);
+        issued = j + 1;
+      }
+      // Drain: the copies this CTA issued must land before its shared memory
+      // can be released, whatever the consumers did.
+      mbar_wait_hw(&sm.bar_q, 0, wc);
+      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
+        mbar_wait_hw(&sm.bar_k_full[j & 1], (j >> 1) & 1, wc);
+        mbar_wait_hw(&sm.bar_v_full[j & 1], (j >> 1) & 1, wc);
+      }
+    }
+  } else if (warp == 1) {
+    // =============================== MMA issuer
+    if (lane == 0 && n_vis > 0) {
+      uint32_t tS[2] = {tmem, tmem + 128};
+      uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      bool ok = mbar_wait(&sm.bar_q, 0, wc) && mbar_wait(&sm.bar_k_full[0], 0, wc);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < n_tiles; ++t) {
+          issue_qk<D>(tS[t], sm.q[t], sm.k[0]);
+          tc_commit(&sm.bar_s_full[t]);
+        }
+      }
+      for (int j = 0; ok && j < n_vis; ++j) {
+        const int s = j & 1, s1 = (j + 1) & 1;
+        if (!mbar_wait(&sm.bar_v_full[s], (j >> 1) & 1, wc)) { ok = false; break; }
+        for (int t = 0; t < n_tiles; ++t) {
+          if (!mbar_wait(&sm.bar_p_ready[t], j & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv<D>(tO[t], tS[t], sm.v[s], j > 0);
+          if (j + 1 < n_vis) {
+            if (t == 0) {
+              if (!mbar_wait(&sm.bar_k_full[s1], ((j + 1) >> 1) & 1, wc)) { ok = false; break; }
+              tc_fence_after();
+            }
+            issue_qk<D>(tS[t], sm.q[t], sm.k[s1]);
+            tc_commit(&sm.bar_s_full[t]);
+          }
+        }
+        if (!ok) break;
+        tc_commit(&sm.bar_kv_empty[s]);
+      }
+      for (int t = 0; t < 2; ++t) tc_commit(&sm.bar_o_final[t]);
+      // MMAs already issued must finish before TMEM can be released.
+      mbar_wait_hw(&sm.bar_o_final[0], 0, wc);
+    }
+  } else if (warp >= 4) {
+    // =============================== softmax / epilogue
+    // tcgen05.ld/st are warp-collective: every branch around them below is
+    // warp-uniform (waits are combined with __all_sync, the O rescale is
+    // decided per warp and applied per row with a factor of 1 where unneeded).
+    const int t = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int q = qt * 128 + r;
+    const int h = h0 + t;
+    const bool active = t < n_tiles;
+    const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+    const uint32_t tS = tmem + uint32_t(t * 128) + lane_off;
+    const uint32_t tO = tmem + 256u + uint32_t(t * D) + lane_off;
+    const int e = row_bound(smp.I0, smp.I1, smp.L, q);
+    const float cs = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = active;
+    for (int j = 0; ok && j < n_vis; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_s_full[t], j & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      tmem_ld_wait();
+      if (j >= n_full) {
+        const int lim = e - j * 128;  // key j*128 + c is visible iff c <= lim
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c > lim) sr[c] = __float_as_uint(-INFINITY);
+      }
+      float mx = __uint_as_float(sr[0]);
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+      const float xmax = mx * cs;
+      if (j == 0) {
+        m = xmax;
+      } else {
+        const bool grow = xmax > m + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float f = grow ? ex2_approx(m - xmax) : 1.f;
+          l *= f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c * 32, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+            tmem_st32(tO + c * 32, ov);
+          }
+          if (grow) m = xmax;
+        }
+      }
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), cs, -m));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), cs, -m));
+        l += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sm.bar_p_ready[t]);
+    }
+    // ---- epilogue: O / l -> bf16 rows, LSE
+    if (active) {
+      bool have = n_vis > 0 && ok;
+      if (have) have = __all_sync(0xffffffffu, mbar_wait(&sm.bar_o_final[t], 0, wc));
+      if (have) tc_fence_after();
+      const bool store = q < p.S;
+      __nv_bfloat16* orow = p.o + int64_t(b) * p.o_sb + int64_t(q) * p.o_ss + int64_t(h / p.g) * p.o_shkv +
+                            int64_t(h % p.g) * p.o_shq;
+      const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        if (have) {
+          tmem_ld32(tO + c * 32, ov);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = 0u;
+        }
+        if (store) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      if (store)
+        p.lse[(int64_t(b) * p.Hq + h) * p.S + q] =
+            (have && l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+  __syncwarp();
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, int n_blocks, int D, cudaStream_t st) {
+  if (n_blocks == 0) return cudaSuccess;
+  if (D == 128) {
+    const size_t smem = sizeof(FwdSmem<128>) + 1024;
+    cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    attn_fwd_kernel<128><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, p);
+  } else {
+    const size_t smem = sizeof(FwdSmem<64>) + 1024;
+    cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    attn_fwd_kernel<64><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hia

@@ -1,0 +1,89 @@
+// kernels.h -- argument blocks and launchers of the device kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace hia {
+
+struct RotateArgs {
+  const void* src;  // bf16 [B,S,heads,D] with strides (elements)
+  int64_t src_sb, src_ss, src_shkv, src_shq;
+  int g;            // heads per stride_hkv group (1 for k)
+  const float* cos_t;
+  const float* sin_t;
+  __nv_bfloat16* dst;  // [B][H][S][D]
+  int B, S, H;
+};
+
+struct DqFinalArgs {
+  const float* acc;  // fp32 [B][H][S_pad][D]
+  int S_pad;
+  float scale;
+  const float* cos_t;
+  const float* sin_t;
+  void* dst;
+  int64_t dst_sb, dst_ss, dst_shkv, dst_shq;
+  int g;
+  int B, S, H;
+};
+
+struct FwdParams {
+  const SampleDev* samples;
+  const int32_t* tiles;  // [B][nQT][2]
+  const int32_t* work;   // [n_work][2]
+  int B, S, Hq, Hkv, g, nQT, n_hp;
+  __nv_bfloat16* o;
+  int64_t o_sb, o_ss, o_shkv, o_shq;
+  float* lse;
+  float scale_log2;  // softmax scale * log2(e)
+  int* status;
+  uint64_t timeout_ns;
+};
+
+struct BwdPreParams {
+  const __nv_bfloat16* o;
+  int64_t o_sb, o_ss, o_shkv, o_shq;
+  const __nv_bfloat16* dout;
+  int64_t d_sb, d_ss, d_shkv, d_shq;
+  const float* lse;     // [B][Hq][S]
+  float* lse2;          // [B][Hq][S_pad]: lse * log2(e); +inf beyond S
+  float* delta;         // [B][Hq][S_pad]: rowsum(dout * o); 0 beyond S
+  float* dq_acc;        // [B][Hq][S_pad][D] zeroed
+  int B, S, S_pad, Hq, g, D;
+};
+
+struct BwdParams {
+  const SampleDev* samples;
+  const int32_t* tiles;  // [B][bKT][2]
+  const int32_t* work;   // [n_work][2]
+  int B, S, S_pad, Hq, Hkv, g, bQT, bKT;
+  const float* lse2;
+  const float* delta;
+  float* dq_acc;
+  const float* cos_t;
+  const float* sin_t;
+  __nv_bfloat16* dk;
+  int64_t dk_sb, dk_ss, dk_sh;
+  __nv_bfloat16* dv;
+  int64_t dv_sb, dv_ss, dv_sh;
+  float scale;        // softmax scale
+  float scale_log2;   // scale * log2(e)
+  int* status;
+  uint64_t timeout_ns;
+};
+
+void launch_rope2d_tables(const SampleDev* samples, int B, int S, int D, double base, float* cos_out,
+                          float* sin_out, cudaStream_t st);
+void launch_rope_rotate(const RotateArgs& a, int D, cudaStream_t st);
+void launch_dq_finalize(const DqFinalArgs& a, int D, cudaStream_t st);
+cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, int n_blocks, int D, cudaStream_t st);
+cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st);
+cudaError_t launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const BwdParams& p, int n_blocks, int D, cudaStream_t st);
+cudaError_t launch_wait_probe(int* status, uint64_t timeout_ns, cudaStream_t st);
+
+}  // namespace hia
