@@ -1,0 +1,354 @@
+#!/usr/bin/env python
+"""Benchmark of the generalized-causal GQA attention with 2D RoPE (fwd + bwd).
+
+One step = one pass of the whole hot path over one synthetic 1024px batch:
+2D RoPE tables, forward (RoPE pre-pass + attention), recompute backward
+(RoPE pre-pass, row statistics, attention backward, dQ epilogue).  The metric
+is masked-FLOP throughput: forward 4*D*Hq*pairs + backward 10*D*Hq*pairs,
+where pairs counts only the visible (query, key) pairs of the generalized
+causal mask, so FLOPs spent on masked lanes of partial tiles are not credited.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU: one process per GPU (torchrun), each rank runs its own replica of
+the workload (the op has no cross-GPU exchange); value = all ranks' FLOPs /
+the slowest rank's time.  --impl reference times the fp64 CPU oracle on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "joint-attn fwd+bwd masked TFLOPS & % bf16 peak, 1024px (4096 img tok)"
+WORKLOAD = "1024px"
+PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_bwd_1024px.md")
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return PEAKS_FALLBACK, "fallback"
+
+
+def workload_desc(wl):
+    pre = [s[0] for s in wl.samples]
+    return (f"1024px fwd+bwd: B={wl.B}, prefix U[512,1536] drawn {pre} (seed 0), image 64x64=4096 tokens, "
+            f"suffix 2, right-padded to S={wl.S}; Hq={wl.Hq}, Hkv={wl.Hkv}, D={wl.D}, scale 1/sqrt(D), "
+            f"bf16 N(0,1) q/k/v/dout")
+
+
+def sample_rows(S, stride=64):
+    return list(range(0, S, stride))
+
+
+def oracle_sample_step(wl, q, k, v, do, rows, nthreads=0):
+    """One reference step: the fp64 oracle's forward and backward for batch row
+    0, kv head 0 (its g query heads), restricted to the given query rows.
+    Returns (seconds, credited masked FLOPs, threads used)."""
+    import numpy as np
+
+    import oracle
+    f64 = lambda t: t[:1].double().numpy()
+    qq, kk, vv, dd = f64(q), f64(k), f64(v), f64(do)
+    groups = np.zeros((1, wl.Hkv), dtype=bool)
+    groups[0, 0] = True
+    smp = wl.samples[:1]
+    t0 = time.perf_counter()
+    _, _, used = oracle.attn_fwd(smp, qq, kk, vv, wl.scale, wl.base, rows=rows, groups=groups,
+                                 nthreads=nthreads)
+    _, _, _, used2 = oracle.attn_bwd(smp, qq, kk, vv, dd, wl.scale, wl.base, rows=rows, groups=groups,
+                                     nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    P, h, w, s = smp[0]
+    I0, I1, L = P, P + h * w, P + h * w + s
+    pairs = sum(min(L - 1, I1 - 1 if I0 <= r < I1 else r) + 1 for r in rows)
+    g = wl.Hq // wl.Hkv
+    flops = 14.0 * wl.D * g * pairs
+    return dt, flops, min(max(used, used2), g)
+
+
+SAMPLE_DESC = ("batch row 0, kv head 0 (its {g} query heads), query rows 0, {stride}, ... ({n} rows): "
+               "fp64 oracle forward + backward restricted to those rows")
+
+
+def cached_traffic(kernel_src):
+    """dram bytes per launch from the committed ncu summary, or None if missing
+    or if the kernel source changed since the counters were taken."""
+    try:
+        txt = open(PROFILE_FILE).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", txt)
+    if not m or not h:
+        return None
+    cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    return float(m.group(1)) if h.group(1) == cur else None
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_id):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", dev_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_reference(args, rank):
+    """Reference arm: the fp64 CPU oracle on a bounded sample (rank 0 only)."""
+    if rank != 0:
+        return
+    import torch
+    from joint_text_image_b200 import synth
+    wl = synth.workload(WORKLOAD, seed=args.seed)
+    q, k, v, do = synth.tensors(wl, args.seed, grad=True)
+    rows = sample_rows(wl.S, args.ref_row_stride)
+    for _ in range(args.warmup):
+        oracle_sample_step(wl, q, k, v, do, rows)
+    tot, fl, used = 0.0, 0.0, 0
+    for _ in range(args.steps):
+        dt, f, used = oracle_sample_step(wl, q, k, v, do, rows)
+        tot += dt
+        fl += f
+    value = fl / tot / 1e12
+    sample = SAMPLE_DESC.format(g=wl.Hq // wl.Hkv, stride=args.ref_row_stride, n=len(rows))
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": workload_desc(wl), "seq_len": wl.S, "global_batch": wl.B},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": used, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--ref-row-stride", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import joint_text_image_b200 as jt
+    from joint_text_image_b200 import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = synth.workload(WORKLOAD, seed=args.seed)
+    q, k, v, do = synth.tensors(wl, args.seed + rank, grad=True)
+    seg = jt.hia_segments_build(wl.samples, wl.S)
+    info = seg.info()
+    pairs = info.visible_pairs
+    fwd_flops = 4.0 * wl.D * wl.Hq * pairs
+    bwd_flops = 10.0 * wl.D * wl.Hq * pairs
+    step_flops = fwd_flops + bwd_flops
+
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    cs = (torch.empty(wl.B, wl.S, wl.D, device=dev), torch.empty(wl.B, wl.S, wl.D, device=dev))
+    o = torch.empty_like(qd)
+    lse = torch.empty(wl.B, wl.Hq, wl.S, device=dev)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    wsf = torch.empty(jt.hia_attn_fwd_workspace_bytes(seg, wl.Hq, wl.Hkv, wl.D), dtype=torch.uint8, device=dev)
+    wsb = torch.empty(jt.hia_attn_bwd_workspace_bytes(seg, wl.Hq, wl.Hkv, wl.D), dtype=torch.uint8, device=dev)
+
+    def step(qi, ki, vi, doi):
+        c, s = jt.hia_rope2d_tables(seg, wl.D, wl.base, out=cs)
+        jt.hia_attn_fwd(seg, qi, ki, vi, c, s, wl.scale, o=o, lse=lse, workspace=wsf)
+        jt.hia_attn_bwd(seg, qi, ki, vi, c, s, o, lse, doi, wl.scale, dq=dq, dk=dk, dv=dv, workspace=wsb)
+
+    for _ in range(args.warmup):
+        step(qd, kd, vd, dod)
+    torch.cuda.synchronize()
+    if jt.hia_get_device_status() != 0:
+        raise RuntimeError("device wait timed out during warm-up")
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    dev_id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev_id)
+    time.sleep(0.3)
+    jt.hia_profile_begin()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(qd, kd, vd, dod)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    prof = jt.hia_profile_end()
+    barrier()
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if jt.hia_get_device_status() != 0:
+        raise RuntimeError("device wait timed out during the timed region")
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * step_flops / (ms * 1e-3) / 1e12
+    launches = sum(n for (n, _) in prof.values())
+
+    # per-kernel times measured live in the timed region (events on the launch stream)
+    kt = {name: {"launches": n, "avg_ms": tot / n, "share": 0.0} for name, (n, tot) in prof.items()}
+    tot_all = sum(tot for (_, tot) in prof.values())
+    for name, (n, tot) in prof.items():
+        kt[name]["share"] = tot / tot_all if tot_all else 0.0
+    pk, pk_kind = peaks()
+    peak_sus = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    peak_burst = float(pk["bf16_tflops"])
+    dom = max(("attn_fwd", "attn_bwd"), key=lambda n: kt.get(n, {"avg_ms": 0})["avg_ms"] * kt.get(n, {"launches": 0})["launches"])
+    dom_flops = bwd_flops if dom == "attn_bwd" else fwd_flops
+    achieved = dom_flops / (kt[dom]["avg_ms"] * 1e-3) / 1e12
+    src = os.path.join(ROOT, "joint_text_image_b200", "csrc", "attn_bwd.cu" if dom == "attn_bwd" else "attn_fwd.cu")
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
+                "frac": achieved / peak_sus, "traffic": cached_traffic(src) if dom == "attn_bwd" else None,
+                "peak_kind": f"bf16_tflops_sustained ({pk_kind}): the kernel runs inside a seconds-long loop",
+                "frac_of_burst_peak": achieved / peak_burst,
+                "algorithmic_flops_per_launch": dom_flops}
+    fwd_t = kt.get("attn_fwd", {}).get("avg_ms")
+    bwd_t = kt.get("attn_bwd", {}).get("avg_ms")
+
+    # end to end through the public API with host buffers (pinned), copies in the timed region
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
+        ho, hl = torch.empty(o.shape, dtype=o.dtype, pin_memory=True), torch.empty(lse.shape, pin_memory=True)
+        hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (dq, dk, dv))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
+        bq, bk, bv, bdo = (torch.empty_like(t) for t in (qd, kd, vd, dod))
+
+        def e2e_step():
+            for dst, src_ in ((bq, hq), (bk, hk), (bv, hv), (bdo, hdo)):
+                dst.copy_(src_, non_blocking=True)
+            step(bq, bk, bv, bdo)
+            for dst, src_ in ((ho, o), (hl, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
+                dst.copy_(src_, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * step_flops / (ems * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = sample_rows(wl.S, args.ref_row_stride)
+        dt, fl, used = oracle_sample_step(wl, q, k, v, do, rows)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOPS", "cores": used, "kind": "oracle",
+               "sample": SAMPLE_DESC.format(g=wl.Hq // wl.Hkv, stride=args.ref_row_stride, n=len(rows))
+                         + f", one step of {dt:.2f} s"}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; no dataset)",
+            "config": {"workload": workload_desc(wl), "global_batch": wl.B * world, "seq_len": wl.S,
+                       "parallelism": f"replicas x{world} (no cross-GPU exchange in this op)",
+                       "l2": f"inputs larger than L2: {(q.numel() + k.numel() + v.numel() + do.numel()) * 2 / 1e6:.0f} MB read per step",
+                       "visible_pairs": pairs, "fwd_flops": fwd_flops, "bwd_flops": bwd_flops},
+            "pct_of_bf16_peak": value / world / peak_burst * 100.0,
+            "fwd_tflops": fwd_flops / (fwd_t * 1e-3) / 1e12 if fwd_t else None,
+            "bwd_tflops": bwd_flops / (bwd_t * 1e-3) / 1e12 if bwd_t else None,
+            "kernels": kt,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -192,6 +192,24 @@ int hia_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 
 const char* hia_status_string(int status);
 
+/* Per-kernel device timing, for benchmarks.  Between hia_profile_begin() and
+ * hia_profile_end(), every kernel the library launches from any thread is
+ * bracketed by a pair of CUDA events recorded on its launch stream (event
+ * objects are created once and reused; recording adds no device work).
+ * hia_profile_end synchronizes those events and fills up to max_entries
+ * records, one per kernel name, with the launch count and the summed
+ * event-to-event time; *n_out receives the number of records.  Kernel names:
+ * "rope2d_tables", "rope_rotate", "attn_fwd", "bwd_pre", "attn_bwd",
+ * "dq_finalize".  Not a library-wide profiler: no other state changes. */
+typedef struct {
+    char name[32];
+    int32_t launches;
+    double total_ms;
+} hia_kernel_time;
+
+int hia_profile_begin(void);
+int hia_profile_end(hia_kernel_time* out, int max_entries, int* n_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -15,7 +15,8 @@ import os
 __all__ = [
     "HiaError", "Segments", "lib", "hia_segments_build", "hia_rope2d_tables", "hia_attn_fwd",
     "hia_attn_bwd", "hia_attn_fwd_workspace_bytes", "hia_attn_bwd_workspace_bytes",
-    "hia_get_device_status", "hia_debug_wait_timeout", "LIB_PATH", "EXPORTED_SYMBOLS",
+    "hia_get_device_status", "hia_debug_wait_timeout", "hia_profile_begin", "hia_profile_end",
+    "LIB_PATH", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libjointattn.so")
@@ -24,7 +25,8 @@ EXPORTED_SYMBOLS = (
     "hia_segments_build", "hia_segments_upload", "hia_segments_destroy", "hia_segments_info",
     "hia_segments_row_bound", "hia_segments_mask", "hia_segments_tile_classes", "hia_rope2d_tables",
     "hia_attn_fwd_workspace_bytes", "hia_attn_fwd", "hia_attn_bwd_workspace_bytes", "hia_attn_bwd",
-    "hia_get_device_status", "hia_debug_wait_timeout", "hia_status_string",
+    "hia_get_device_status", "hia_debug_wait_timeout", "hia_status_string", "hia_profile_begin",
+    "hia_profile_end",
 )
 
 
@@ -50,6 +52,10 @@ class SegmentsInfo(ctypes.Structure):
                 ("fwd_tiles_full", ctypes.c_int64), ("fwd_tiles_partial", ctypes.c_int64),
                 ("fwd_tiles_skipped", ctypes.c_int64), ("bwd_q_tiles", ctypes.c_int32),
                 ("bwd_kv_tiles", ctypes.c_int32)]
+
+
+class _KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_double)]
 
 
 _lib = None
@@ -81,6 +87,8 @@ def lib():
         L.hia_attn_bwd.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, T, P, T, T, T, T, P, Z, P]
         L.hia_get_device_status.argtypes = [P]
         L.hia_debug_wait_timeout.argtypes = [ctypes.c_uint64, P]
+        L.hia_profile_begin.argtypes = []
+        L.hia_profile_end.argtypes = [ctypes.POINTER(_KernelTime), I, ctypes.POINTER(I)]
         L.hia_status_string.argtypes = [I]
         L.hia_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -257,3 +265,16 @@ def hia_get_device_status():
 
 def hia_debug_wait_timeout(timeout_ns: int):
     _check(lib().hia_debug_wait_timeout(int(timeout_ns), _stream()), "hia_debug_wait_timeout")
+
+
+def hia_profile_begin():
+    """Start per-kernel CUDA-event timing of every library launch."""
+    _check(lib().hia_profile_begin(), "hia_profile_begin")
+
+
+def hia_profile_end():
+    """Stop timing; returns {kernel name: (launches, total_ms)}."""
+    arr = (_KernelTime * 16)()
+    n = ctypes.c_int(0)
+    _check(lib().hia_profile_end(arr, 16, ctypes.byref(n)), "hia_profile_end")
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(min(n.value, 16))}

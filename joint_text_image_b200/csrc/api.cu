@@ -68,10 +68,10 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
 }
 
 // [rows = S][D] per (b, head) slab of a [B*H][S][D] workspace tensor.
-bool make_ws_map(CUtensorMap* m, const void* base, int D, int S, int BH) {
+bool make_ws_map(CUtensorMap* m, const void* base, int D, int S, int BH, uint32_t rows = 128) {
   uint64_t dims[3] = {uint64_t(D), uint64_t(S), uint64_t(BH)};
   uint64_t st[2] = {uint64_t(D) * 2, uint64_t(S) * D * 2};
-  uint32_t box[3] = {64, 128, 1};
+  uint32_t box[3] = {64, rows, 1};
   return make_map(m, base, 3, dims, st, box);
 }
 
@@ -320,7 +320,108 @@ extern "C" int hia_attn_bwd(const hia_segments* g, int Hq, int Hkv, int D, hia_t
   int rc = check_common(g, Hq, Hkv, D, c, s);
   if (rc) return rc;
   if (g->B == 0 || g->S == 0) return HIA_OK;
-  (void)q; (void)k; (void)v; (void)scale; (void)o; (void)lse; (void)dout; (void)dq; (void)dk; (void)dv;
-  (void)ws; (void)ws_bytes; (void)stream;
-  return HIA_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return HIA_ERR_INVALID_ARG;
+  const int gq = Hq / Hkv;
+  if ((rc = check_tensor(q, true, g->B, g->S, gq)) || (rc = check_tensor(k, false, g->B, g->S, 1)) ||
+      (rc = check_tensor(v, false, g->B, g->S, 1)) || (rc = check_tensor(o, true, g->B, g->S, gq)) ||
+      (rc = check_tensor(dout, true, g->B, g->S, gq)) || (rc = check_tensor(dq, true, g->B, g->S, gq)) ||
+      (rc = check_tensor(dk, false, g->B, g->S, 1)) || (rc = check_tensor(dv, false, g->B, g->S, 1)))
+    return rc;
+  if (!q.ptr || !k.ptr || !v.ptr || !o.ptr || !lse || !dout.ptr || !dq.ptr || !dk.ptr || !dv.ptr || !ws)
+    return HIA_ERR_INVALID_ARG;
+  const BwdWs w = bwd_ws(g, Hq, Hkv, D);
+  if (ws_bytes < w.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return HIA_ERR_INVALID_ARG;
+  int* status = status_ptr();
+  if (!status) return HIA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* wb = static_cast<char*>(ws);
+  __nv_bfloat16* qr = reinterpret_cast<__nv_bfloat16*>(wb + w.q_off);
+  __nv_bfloat16* kr = reinterpret_cast<__nv_bfloat16*>(wb + w.k_off);
+  float* lse2 = reinterpret_cast<float*>(wb + w.lse_off);
+  float* delta = reinterpret_cast<float*>(wb + w.delta_off);
+  float* dq_acc = reinterpret_cast<float*>(wb + w.dq_off);
+  const int S_pad = S_pad64(g->S);
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_ws_map(&tq, qr, D, g->S, g->B * Hq, 64) || !make_ws_map(&tk, kr, D, g->S, g->B * Hkv, 128) ||
+      !make_kv_map(&tv, v, D, Hkv, g->S, g->B, 128) || !make_q_map(&tdo, dout, D, gq, Hkv, g->S, g->B, 64))
+    return HIA_ERR_CUDA;
+
+  rotate_into(q, Hq, gq, c, s, qr, g, D, st);
+  rotate_into(k, Hkv, 1, c, s, kr, g, D, st);
+  if (cudaMemsetAsync(dq_acc, 0, size_t(g->B) * Hq * S_pad * D * 4, st) != cudaSuccess) return HIA_ERR_CUDA;
+
+  hia::BwdPreParams pp{};
+  pp.o = static_cast<const __nv_bfloat16*>(o.ptr);
+  pp.o_sb = o.stride_b;
+  pp.o_ss = o.stride_s;
+  pp.o_shkv = o.stride_hkv;
+  pp.o_shq = o.stride_hq;
+  pp.dout = static_cast<const __nv_bfloat16*>(dout.ptr);
+  pp.d_sb = dout.stride_b;
+  pp.d_ss = dout.stride_s;
+  pp.d_shkv = dout.stride_hkv;
+  pp.d_shq = dout.stride_hq;
+  pp.lse = lse;
+  pp.lse2 = lse2;
+  pp.delta = delta;
+  pp.dq_acc = dq_acc;
+  pp.B = g->B;
+  pp.S = g->S;
+  pp.S_pad = S_pad;
+  pp.Hq = Hq;
+  pp.g = gq;
+  pp.D = D;
+  if ((rc = cuda_status(hia::launch_bwd_pre(pp, st)))) return rc;
+
+  hia::BwdParams p{};
+  p.samples = g->d_samples;
+  p.tiles = g->d_bwd_tiles;
+  p.work = g->d_bwd_work;
+  p.B = g->B;
+  p.S = g->S;
+  p.S_pad = S_pad;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.g = gq;
+  p.bQT = g->bQT;
+  p.bKT = g->bKT;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.dq_acc = dq_acc;
+  p.cos_t = c;
+  p.sin_t = s;
+  p.dk = static_cast<__nv_bfloat16*>(dk.ptr);
+  p.dk_sb = dk.stride_b;
+  p.dk_ss = dk.stride_s;
+  p.dk_sh = dk.stride_hkv;
+  p.dv = static_cast<__nv_bfloat16*>(dv.ptr);
+  p.dv_sb = dv.stride_b;
+  p.dv_ss = dv.stride_s;
+  p.dv_sh = dv.stride_hkv;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.status = status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  const int64_t n_blocks = int64_t(g->B) * g->bKT * Hkv;
+  if (n_blocks > (1ll << 31) - 1) return HIA_ERR_UNSUPPORTED;
+  if ((rc = cuda_status(hia::launch_attn_bwd(tq, tk, tv, tdo, p, int(n_blocks), D, st)))) return rc;
+
+  hia::DqFinalArgs fa{};
+  fa.acc = dq_acc;
+  fa.S_pad = S_pad;
+  fa.scale = scale;
+  fa.cos_t = c;
+  fa.sin_t = s;
+  fa.dst = dq.ptr;
+  fa.dst_sb = dq.stride_b;
+  fa.dst_ss = dq.stride_s;
+  fa.dst_shkv = dq.stride_hkv;
+  fa.dst_shq = dq.stride_hq;
+  fa.g = gq;
+  fa.B = g->B;
+  fa.S = g->S;
+  fa.H = Hq;
+  hia::launch_dq_finalize(fa, D, st);
+  return cuda_status(cudaGetLastError());
 }

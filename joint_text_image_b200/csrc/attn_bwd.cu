@@ -1,0 +1,466 @@
+// attn_bwd.cu -- recompute backward of the generalized-causal GQA attention.
+//
+// With P = softmax(scale * Qr Kr^T) over the visible pairs (the forward of
+// HunyuanImage3Attention under build_joint_attention_mask), dO the incoming
+// gradient and delta_q = dO_q . O_q:
+//   dV  = P^T dO,   dP = dO V^T,   dS = P o (dP - delta),
+//   dKr = scale dS^T Qr,   dQr = scale dS Kr,
+// summed over the g query heads of each kv head; dK, dQ = R^T dKr, R^T dQr.
+//
+// bwd_pre: delta and LSE * log2(e) per row, padded to a multiple of 64 rows.
+// attn_bwd: one CTA per (b, kv head, 128-key tile).  It keeps Kr and V in
+// shared memory and dK, dV in TMEM, and walks the g heads x the 64-row query
+// tiles that see its keys (a suffix of query tiles, since the row bound e(q)
+// is non-decreasing).  Per query tile, with keys on the MMA M side:
+//   S^T = Kr Qr^T, dP^T = V dO^T      (SS MMAs, M=128, N=64)
+//   P^T = exp2(S^T * scale*log2e - lse2), dS^T = P^T o (dP^T - delta)
+//   dV += P^T dO,  dK += dS^T Qr       (A = P^T / dS^T straight from TMEM)
+//   dQ^T = Kr^T dS^T                   (A = Kr read as MN-major, B = dS^T in
+//                                       shared memory) -> fp32 red.add
+// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 4-7 softmax (one key row
+// per thread, then the dK/dV epilogue with the inverse RoPE), 8-11 dQ
+// writers (one head-dim lane per thread, coalesced fp32 reductions).
+// TMEM: S^T[2] at 0/64, dP^T[2] at 128/192 (P^T, dS^T written over them as
+// packed bf16), dV at 256, dK at 256 + D; dQ^T of buffer i is written over
+// S^T[i] after the dV MMA that read P^T from there (MMAs run in issue order).
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace hia {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kStages = 3;
+constexpr int BK = kBwdBK;  // 128 keys
+constexpr int BQ = kBwdBQ;  // 64 query rows
+
+template <int D>
+struct BwdSmem {
+  alignas(1024) __nv_bfloat16 k[BK * D];
+  alignas(1024) __nv_bfloat16 v[BK * D];
+  alignas(1024) __nv_bfloat16 q[kStages][BQ * D];
+  alignas(1024) __nv_bfloat16 dout[kStages][BQ * D];
+  alignas(1024) __nv_bfloat16 ds[2][BK * BQ];  // dS^T rows = keys, 64 q per 128-byte row
+  alignas(16) float lse2[kStages][BQ];
+  alignas(16) float delta[kStages][BQ];
+  uint64_t bar_kv;
+  uint64_t bar_full[kStages];
+  uint64_t bar_empty[kStages];
+  uint64_t bar_s_full[2];
+  uint64_t bar_dp_full[2];
+  uint64_t bar_p_ready[2];
+  uint64_t bar_ds_ready[2];
+  uint64_t bar_dq_full[2];
+  uint64_t bar_dq_empty[2];
+  uint64_t bar_final;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// S^T / dP^T: A = 128-row tile (K-major, 64-wide D blocks 16 KB apart),
+// B = 64-row tile (K-major, D blocks 8 KB apart).
+template <int D>
+__device__ __forceinline__ void issue_kq(uint32_t d, const __nv_bfloat16* a, const __nv_bfloat16* b) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, BQ, 0, 0);
+  const uint32_t aa = smem_u32(a), ba = smem_u32(b);
+#pragma unroll
+  for (int kb = 0; kb < D / 16; ++kb) {
+    const uint32_t in = uint32_t(kb & 3) * 32u;
+    mma_ss(d, sdesc_sw128(aa + uint32_t(kb >> 2) * 16384u + in, 16, 1024),
+           sdesc_sw128(ba + uint32_t(kb >> 2) * 8192u + in, 16, 1024), idesc, kb > 0 ? 1u : 0u);
+  }
+}
+
+// dV += P^T dO or dK += dS^T Qr: A from TMEM (128 keys x 64 q, packed bf16),
+// B = 64-row tile read MN-major (N = D contiguous, D blocks 8 KB apart).
+template <int D>
+__device__ __forceinline__ void issue_acc(uint32_t d, uint32_t a_tmem, const __nv_bfloat16* b, bool acc) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+  const uint32_t ba = smem_u32(b);
+#pragma unroll
+  for (int kb = 0; kb < BQ / 16; ++kb)
+    mma_ts(d, a_tmem + uint32_t(kb) * 8u, sdesc_sw128(ba + uint32_t(kb) * 2048u, 8192, 1024), idesc,
+           (acc || kb > 0) ? 1u : 0u);
+}
+
+// dQ^T = Kr^T dS^T: M = 128 (head dims; for D = 64 the second 64-row block
+// reads the V tile and its result lanes are ignored), N = 64 q, K = 128 keys.
+// A = Kr tile read MN-major, B = dS^T tile read MN-major.
+template <int D>
+__device__ __forceinline__ void issue_dq(uint32_t d, const __nv_bfloat16* kt, const __nv_bfloat16* vt,
+                                         const __nv_bfloat16* ds) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, BQ, 1, 1);
+  const uint32_t ka = smem_u32(kt), da = smem_u32(ds);
+  const uint32_t lbo = (D == 128) ? 16384u : (smem_u32(vt) - ka);
+#pragma unroll
+  for (int kb = 0; kb < BK / 16; ++kb)
+    mma_ss(d, sdesc_sw128(ka + uint32_t(kb) * 2048u, lbo, 1024), sdesc_sw128(da + uint32_t(kb) * 2048u, 8192, 1024),
+           idesc, kb > 0 ? 1u : 0u);
+}
+
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  BwdSmem<D>& sm =
+      *reinterpret_cast<BwdSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  int bid = blockIdx.x;
+  const int hkv = bid % p.Hkv;
+  bid /= p.Hkv;
+  const int b = p.work[2 * bid], kt = p.work[2 * bid + 1];
+  const int qt_first = p.tiles[2 * (b * p.bKT + kt)];
+  const int qt_full = p.tiles[2 * (b * p.bKT + kt) + 1];
+  const int n_qt = p.bQT - qt_first;
+  const int n_it = n_qt * p.g;  // iteration i: head hkv*g + i / n_qt, query tile qt_first + i % n_qt
+  const SampleDev smp = p.samples[b];
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar_kv, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sm.bar_full[i], 1);
+      mbar_init(&sm.bar_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.bar_s_full[i], 1);
+      mbar_init(&sm.bar_dp_full[i], 1);
+      mbar_init(&sm.bar_p_ready[i], 128);
+      mbar_init(&sm.bar_ds_ready[i], 128);
+      mbar_init(&sm.bar_dq_full[i], 1);
+      mbar_init(&sm.bar_dq_empty[i], 128);
+    }
+    mbar_init(&sm.bar_final, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtx wc{&sm.abort_flag, p.status, p.timeout_ns};
+  const uint32_t tS[2] = {tmem, tmem + 64};
+  const uint32_t tdP[2] = {tmem + 128, tmem + 192};
+  const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D;
+
+  if (warp == 0) {
+    // =============================== TMA producer
+    if (lane == 0 && n_it > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      constexpr uint32_t kv_bytes = BK * D * 2, qd_bytes = BQ * D * 2;
+      mbar_arrive_expect_tx(&sm.bar_kv, 2 * kv_bytes);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(&sm.k[c * BK * 64], &tm_k, &sm.bar_kv, c * 64, kt * BK, b * p.Hkv + hkv);
+        tma_load_4d(&sm.v[c * BK * 64], &tm_v, &sm.bar_kv, c * 64, hkv, kt * BK, b);
+      }
+      int issued = 0;
+      for (int i = 0; i < n_it; ++i) {
+        const int s = i % kStages, n = i / kStages;
+        if (i >= kStages && !mbar_wait(&sm.bar_empty[s], (n - 1) & 1, wc)) break;
+        const int hi = i / n_qt, qt = qt_first + i % n_qt;
+        const int h = hkv * p.g + hi;
+        mbar_arrive_expect_tx(&sm.bar_full[s], 2 * qd_bytes + 2 * BQ * 4);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(&sm.q[s][c * BQ * 64], &tm_q, &sm.bar_full[s], c * 64, qt * BQ, b * p.Hq + h);
+          tma_load_5d(&sm.dout[s][c * BQ * 64], &tm_do, &sm.bar_full[s], c * 64, hi, hkv, qt * BQ, b);
+        }
+        const int64_t row = (int64_t(b) * p.Hq + h) * p.S_pad + int64_t(qt) * BQ;
+        bulk_load(sm.lse2[s], p.lse2 + row, BQ * 4, &sm.bar_full[s]);
+        bulk_load(sm.delta[s], p.delta + row, BQ * 4, &sm.bar_full[s]);
+        issued = i + 1;
+      }
+      mbar_wait_hw(&sm.bar_kv, 0, wc);
+      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+        mbar_wait_hw(&sm.bar_full[i % kStages], (i / kStages) & 1, wc);
+    }
+  } else if (warp == 1) {
+    // =============================== MMA issuer
+    if (lane == 0 && n_it > 0) {
+      bool ok = mbar_wait(&sm.bar_kv, 0, wc) && mbar_wait(&sm.bar_full[0], 0, wc);
+      if (ok) {
+        tc_fence_after();
+        issue_kq<D>(tS[0], sm.k, sm.q[0]);
+        tc_commit(&sm.bar_s_full[0]);
+        issue_kq<D>(tdP[0], sm.v, sm.dout[0]);
+        tc_commit(&sm.bar_dp_full[0]);
+      }
+      for (int i = 0; ok && i < n_it; ++i) {
+        const int bf = i & 1, s = i % kStages;
+        if (i + 1 < n_it) {
+          const int i1 = i + 1, b1 = i1 & 1, s1 = i1 % kStages;
+          ok = mbar_wait(&sm.bar_full[s1], (i1 / kStages) & 1, wc);
+          if (ok && i1 >= 2) ok = mbar_wait(&sm.bar_dq_empty[b1], ((i1 >> 1) - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          issue_kq<D>(tS[b1], sm.k, sm.q[s1]);
+          tc_commit(&sm.bar_s_full[b1]);
+          issue_kq<D>(tdP[b1], sm.v, sm.dout[s1]);
+          tc_commit(&sm.bar_dp_full[b1]);
+        }
+        if (!mbar_wait(&sm.bar_p_ready[bf], (i >> 1) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        issue_acc<D>(tdV, tS[bf], sm.dout[s], i > 0);
+        if (!mbar_wait(&sm.bar_ds_ready[bf], (i >> 1) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        issue_acc<D>(tdK, tdP[bf], sm.q[s], i > 0);
+        issue_dq<D>(tS[bf], sm.k, sm.v, sm.ds[bf]);
+        tc_commit(&sm.bar_dq_full[bf]);
+        tc_commit(&sm.bar_empty[s]);
+      }
+      tc_commit(&sm.bar_final);
+      mbar_wait_hw(&sm.bar_final, 0, wc);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // =============================== softmax: one key row per thread
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int key = kt * BK + r;
+    const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+    const float cs = p.scale_log2;
+    bool ok = true;
+    for (int i = 0; i < n_it; ++i) {
+      const int bf = i & 1, s = i % kStages;
+      const int qt = qt_first + i % n_qt;
+      const bool partial = qt < qt_full || (qt + 1) * BQ > p.S;
+      // the stage's lse2/delta were written by TMA: acquire them through its barrier
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_full[s], (i / kStages) & 1, wc) &&
+                                       mbar_wait(&sm.bar_s_full[bf], (i >> 1) & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(tS[bf] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS[bf] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld_wait();
+      float pv[64];
+      const float* l2 = sm.lse2[s];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) pv[c] = ex2_approx(fmaf(__uint_as_float(sr[c]), cs, -l2[c]));
+      if (partial) {
+        const int q0 = qt * BQ;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (key > row_bound(smp.I0, smp.I1, smp.L, q0 + c) || q0 + c >= p.S) pv[c] = 0.f;
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+      tmem_st32(tS[bf] + lane_off, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sm.bar_p_ready[bf]);
+
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_dp_full[bf], (i >> 1) & 1, wc));
+      if (!ok) break;
+      tc_fence_after();
+      tmem_ld32(tdP[bf] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tdP[bf] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld_wait();
+      const float* dl = sm.delta[s];
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        pk[c] = pack_bf16x2(pv[2 * c] * (__uint_as_float(sr[2 * c]) - dl[2 * c]),
+                            pv[2 * c + 1] * (__uint_as_float(sr[2 * c + 1]) - dl[2 * c + 1]));
+      tmem_st32(tdP[bf] + lane_off, pk);
+      // dS^T row -> shared memory, 128-byte swizzled rows of 64 query values
+      uint8_t* dsrow = reinterpret_cast<uint8_t*>(sm.ds[bf]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(dsrow + sw128_offset(uint32_t(r), uint32_t(c))) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sm.bar_ds_ready[bf]);
+    }
+    // ---- epilogue: dK = R^T (scale dKr), dV -> bf16
+    bool have = n_it > 0 && ok;
+    if (have) have = __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, wc));
+    if (have) tc_fence_after();
+    const bool store = key < p.S;
+    const int kc = store ? key : p.S - 1;
+    const float* cp = p.cos_t + (int64_t(b) * p.S + kc) * D;
+    const float* sp = p.sin_t + (int64_t(b) * p.S + kc) * D;
+    __nv_bfloat16* dkrow = p.dk + int64_t(b) * p.dk_sb + int64_t(key) * p.dk_ss + int64_t(hkv) * p.dk_sh;
+    __nv_bfloat16* dvrow = p.dv + int64_t(b) * p.dv_sb + int64_t(key) * p.dv_ss + int64_t(hkv) * p.dv_sh;
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      uint32_t lo[32], hi[32];
+      if (have) {
+        tmem_ld32(tdK + lane_off + c * 32, lo);
+        tmem_ld32(tdK + lane_off + D / 2 + c * 32, hi);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) lo[i] = hi[i] = 0u;
+      }
+      if (store) {
+        uint32_t olo[16], ohi[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float a[2], bb[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = c * 32 + 2 * i + e;
+            const float cj = __ldg(cp + j), sj = __ldg(sp + j);
+            const float l = __uint_as_float(lo[2 * i + e]) * p.scale, u = __uint_as_float(hi[2 * i + e]) * p.scale;
+            a[e] = fmaf(l, cj, u * sj);
+            bb[e] = fmaf(u, cj, -l * sj);
+          }
+          olo[i] = pack_bf16x2(a[0], a[1]);
+          ohi[i] = pack_bf16x2(bb[0], bb[1]);
+        }
+        uint4* d0 = reinterpret_cast<uint4*>(dkrow + c * 32);
+        uint4* d1 = reinterpret_cast<uint4*>(dkrow + D / 2 + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          d0[i] = make_uint4(olo[4 * i], olo[4 * i + 1], olo[4 * i + 2], olo[4 * i + 3]);
+          d1[i] = make_uint4(ohi[4 * i], ohi[4 * i + 1], ohi[4 * i + 2], ohi[4 * i + 3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t ov[32];
+      if (have) {
+        tmem_ld32(tdV + lane_off + c * 32, ov);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = 0u;
+      }
+      if (store) {
+        uint4* d0 = reinterpret_cast<uint4*>(dvrow + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          d0[i] = make_uint4(pack_bf16x2(__uint_as_float(ov[8 * i]), __uint_as_float(ov[8 * i + 1])),
+                             pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3])),
+                             pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5])),
+                             pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7])));
+      }
+    }
+  } else if (warp >= 8) {
+    // =============================== dQ writers: one head-dim lane per thread
+    const int quarter = warp & 3;
+    const int d = quarter * 32 + lane;
+    const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+    const bool live = quarter * 32 < D;  // warp-uniform
+    for (int i = 0; i < n_it; ++i) {
+      const int bf = i & 1;
+      const int hi = i / n_qt, qt = qt_first + i % n_qt;
+      const int h = hkv * p.g + hi;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dq_full[bf], (i >> 1) & 1, wc))) break;
+      tc_fence_after();
+      if (live) {
+        uint32_t a[32], c2[32];
+        tmem_ld32(tS[bf] + lane_off, a);
+        tmem_ld32(tS[bf] + lane_off + 32, c2);
+        tmem_ld_wait();
+        float* dst = p.dq_acc + ((int64_t(b) * p.Hq + h) * p.S_pad + int64_t(qt) * BQ) * D + d;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) red_add_f32(dst + int64_t(c) * D, __uint_as_float(a[c]));
+#pragma unroll
+        for (int c = 0; c < 32; ++c) red_add_f32(dst + int64_t(c + 32) * D, __uint_as_float(c2[c]));
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.bar_dq_empty[bf]);
+    }
+  }
+  __syncwarp();
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// delta = rowsum(dO o O) and lse2 = lse * log2(e) for every (b, h, q < S_pad);
+// rows q >= S get delta 0 and lse2 +inf (so they contribute nothing).
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreParams p) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= p.B * p.S_pad) return;
+  const int b = warp / p.S_pad, q = warp % p.S_pad;
+  const int per = p.D / 32;  // elements per lane: 4 (D=128) or 2 (D=64)
+  for (int h = 0; h < p.Hq; ++h) {
+    const int64_t orow = (int64_t(b) * p.Hq + h) * p.S_pad + q;
+    if (q >= p.S) {
+      if (lane == 0) {
+        p.delta[orow] = 0.f;
+        p.lse2[orow] = INFINITY;
+      }
+      continue;
+    }
+    const __nv_bfloat16* o = p.o + int64_t(b) * p.o_sb + int64_t(q) * p.o_ss + int64_t(h / p.g) * p.o_shkv +
+                             int64_t(h % p.g) * p.o_shq;
+    const __nv_bfloat16* d = p.dout + int64_t(b) * p.d_sb + int64_t(q) * p.d_ss + int64_t(h / p.g) * p.d_shkv +
+                             int64_t(h % p.g) * p.d_shq;
+    float acc = 0.f;
+    if (per == 4) {
+      const uint2 ov = *reinterpret_cast<const uint2*>(o + lane * 4);
+      const uint2 dv = *reinterpret_cast<const uint2*>(d + lane * 4);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+      const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float2 a = __bfloat1622float2(o2[i]), c = __bfloat1622float2(d2[i]);
+        acc = fmaf(a.x, c.x, acc);
+        acc = fmaf(a.y, c.y, acc);
+      }
+    } else {
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + lane * 2));
+      const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(d + lane * 2));
+      acc = fmaf(a.x, c.x, a.y * c.y);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      p.delta[orow] = acc;
+      p.lse2[orow] = p.lse[(int64_t(b) * p.Hq + h) * p.S + q] * 1.4426950408889634f;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st) {
+  const int64_t warps = int64_t(p.B) * p.S_pad;
+  if (warps == 0) return cudaSuccess;
+  prof_begin(kBwdPre, st);
+  bwd_pre_kernel<<<int((warps + 7) / 8), 256, 0, st>>>(p);
+  prof_end(kBwdPre, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const BwdParams& p, int n_blocks, int D, cudaStream_t st) {
+  if (n_blocks == 0) return cudaSuccess;
+  prof_begin(kAttnBwd, st);
+  if (D == 128) {
+    const size_t smem = sizeof(BwdSmem<128>) + 1024;
+    cudaFuncSetAttribute(attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    attn_bwd_kernel<128><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, tdo, p);
+  } else {
+    const size_t smem = sizeof(BwdSmem<64>) + 1024;
+    cudaFuncSetAttribute(attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    attn_bwd_kernel<64><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, tdo, p);
+  }
+  prof_end(kAttnBwd, st);
+  return cudaGetLastError();
+}
+
+}  // namespace hia

@@ -304,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int n_blocks, int D, cudaStream_t st) {
   if (n_blocks == 0) return cudaSuccess;
+  prof_begin(kAttnFwd, st);
   if (D == 128) {
     const size_t smem = sizeof(FwdSmem<128>) + 1024;
     cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
@@ -313,6 +314,7 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
     cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     attn_fwd_kernel<64><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, p);
   }
+  prof_end(kAttnFwd, st);
   return cudaGetLastError();
 }
 

@@ -75,6 +75,11 @@ struct BwdParams {
   uint64_t timeout_ns;
 };
 
+// Profiling brackets around one kernel launch (no-ops unless profiling is on).
+enum KernelId { kRopeTables = 0, kRopeRotate, kAttnFwd, kBwdPre, kAttnBwd, kDqFinalize, kNumKernels };
+void prof_begin(KernelId id, cudaStream_t st);
+void prof_end(KernelId id, cudaStream_t st);
+
 void launch_rope2d_tables(const SampleDev* samples, int B, int S, int D, double base, float* cos_out,
                           float* sin_out, cudaStream_t st);
 void launch_rope_rotate(const RotateArgs& a, int D, cudaStream_t st);

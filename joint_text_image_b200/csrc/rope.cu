@@ -149,23 +149,29 @@ void launch_rope2d_tables(const SampleDev* samples, int B, int S, int D, double 
   const int threads = 256;
   int64_t blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 64) blocks = 148 * 64;
+  prof_begin(kRopeTables, st);
   rope2d_tables_kernel<<<int(blocks), threads, 0, st>>>(samples, B, S, D, base, cos_out, sin_out);
+  prof_end(kRopeTables, st);
 }
 
 void launch_rope_rotate(const RotateArgs& a, int D, cudaStream_t st) {
   const int64_t warps = int64_t(a.B) * a.S;
   if (warps == 0) return;
   const int blocks = int((warps + 7) / 8);
+  prof_begin(kRopeRotate, st);
   if (D == 128) rope_rotate_kernel<128><<<blocks, 256, 0, st>>>(a);
   else rope_rotate_kernel<64><<<blocks, 256, 0, st>>>(a);
+  prof_end(kRopeRotate, st);
 }
 
 void launch_dq_finalize(const DqFinalArgs& a, int D, cudaStream_t st) {
   const int64_t warps = int64_t(a.B) * a.S;
   if (warps == 0) return;
   const int blocks = int((warps + 7) / 8);
+  prof_begin(kDqFinalize, st);
   if (D == 128) dq_finalize_kernel<128><<<blocks, 256, 0, st>>>(a);
   else dq_finalize_kernel<64><<<blocks, 256, 0, st>>>(a);
+  prof_end(kDqFinalize, st);
 }
 
 }  // namespace hia

@@ -45,7 +45,7 @@ def _load():
         lib.oracle_rope_tables.argtypes = [I, I, I, P, P, P, P, D, P, P]
         lib.oracle_rope_apply.argtypes = [I, I, I, I, P, P, P, P, D, I, P, P]
         lib.oracle_attn_fwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, D, D, I, P, I, P, P, P, I]
-        lib.oracle_attn_bwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, D, D, I, P, P, P, P, I]
+        lib.oracle_attn_bwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, D, D, I, P, I, P, P, P, P, I]
         _lib = lib
     return _lib
 
@@ -130,8 +130,10 @@ def attn_fwd(samples, q, k, v, scale=None, base=10000.0, rotate=True, rows=None,
 
 
 def attn_bwd(samples, q, k, v, dout, scale=None, base=10000.0, rotate=True, groups=None,
-             nthreads=0):
-    """Backward: returns (dq [B,S,Hq,D], dk, dv [B,S,Hkv,D], threads_used)."""
+             nthreads=0, rows=None):
+    """Backward: returns (dq [B,S,Hq,D], dk, dv [B,S,Hkv,D], threads_used).
+
+    rows: optional query-row subset (dq of those rows; dk, dv summed over them)."""
     g = _geom(samples)
     q = np.ascontiguousarray(q, dtype=np.float64)
     k = np.ascontiguousarray(k, dtype=np.float64)
@@ -142,11 +144,13 @@ def attn_bwd(samples, q, k, v, dout, scale=None, base=10000.0, rotate=True, grou
     if scale is None:
         scale = 1.0 / np.sqrt(D)
     gs = None if groups is None else np.ascontiguousarray(groups, dtype=np.uint8).reshape(-1)
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
     dq = np.zeros((B, S, Hq, D))
     dk = np.zeros((B, S, Hkv, D))
     dv = np.zeros((B, S, Hkv, D))
     used = _load().oracle_attn_bwd(B, S, Hq, Hkv, D, *map(_p, g), _p(q), _p(k), _p(v), _p(dout),
-                                   float(scale), float(base), int(rotate), _p(gs), _p(dq),
+                                   float(scale), float(base), int(rotate), _p(r),
+                                   0 if r is None else len(r), _p(gs), _p(dq),
                                    _p(dk), _p(dv), int(nthreads))
     if used < 0:
         raise ValueError("bad arguments")

@@ -287,7 +287,9 @@ static void bwd_task(job_t* J, int b, int h) {
     gather_head(J, J->q, J->Hq, b, h, J->rotate_inputs, qr);
     gather_head(J, J->k, J->Hkv, b, h / g, J->rotate_inputs, kr);
     gather_head(J, J->v, J->Hkv, b, h / g, 0, vv);
-    for (int64_t q = 0; q < S; ++q) {
+    int nr = J->rows ? J->n_rows : S;
+    for (int ri = 0; ri < nr; ++ri) {
+        int64_t q = J->rows ? J->rows[ri] : ri;
         const double* dorow = J->dout + (((int64_t)b * S + q) * J->Hq + h) * D;
         double* dqout = J->dq + (((int64_t)b * S + q) * J->Hq + h) * D;
         double m = -INFINITY;
@@ -401,12 +403,14 @@ int oracle_attn_fwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
 }
 
 /* Backward.  dq [B,S,Hq,D]; dk, dv [B,S,Hkv,D].  group_sel as above (dq of
- * unselected groups and their dk/dv are left untouched). */
+ * unselected groups and their dk/dv are left untouched).  rows/n_rows
+ * restrict the query rows: dq is written for those rows only and dk, dv hold
+ * the contributions of those rows only (a partial sum over queries). */
 int oracle_attn_bwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
                     const int32_t* img_h, const int32_t* img_w, const int32_t* suffix,
                     const double* q, const double* k, const double* v, const double* dout,
-                    double scale, double base, int rotate_inputs, const uint8_t* group_sel,
-                    double* dq, double* dk, double* dv, int nthreads) {
+                    double scale, double base, int rotate_inputs, const int32_t* rows, int n_rows,
+                    const uint8_t* group_sel, double* dq, double* dk, double* dv, int nthreads) {
     if (check_geom(B, S, Hq, Hkv, D, prefix, img_h, img_w, suffix)) return -1;
     size_t n = (size_t)B * S * Hq * D;
     job_t J;
@@ -414,7 +418,8 @@ int oracle_attn_bwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
     J.B = B; J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.D = D;
     J.prefix = prefix; J.img_h = img_h; J.img_w = img_w; J.suffix = suffix;
     J.q = q; J.k = k; J.v = v; J.dout = dout; J.scale = scale; J.base = base;
-    J.rotate_inputs = rotate_inputs; J.group_sel = group_sel; J.dq = dq;
+    J.rotate_inputs = rotate_inputs; J.rows = rows; J.n_rows = n_rows;
+    J.group_sel = group_sel; J.dq = dq;
     J.dk_h = calloc(n ? n : 1, sizeof(double));
     J.dv_h = calloc(n ? n : 1, sizeof(double));
     int used = run_job(&J, 1, nthreads);

@@ -77,3 +77,43 @@ def check_fwd(oracle_mod, wl, q, k, v, o, lse, rows=None, groups=None):
     print(f"[parity] {wl.name}: O max {e.max():.3e} mean {e.mean():.3e}; LSE max {le.max():.3e} "
           f"mean {le.mean():.3e}")
     return e.max(), e.mean(), le.max()
+
+
+def run_fwd_bwd(wl, seed=0):
+    q, k, v, do = synth.tensors(wl, seed, grad=True)
+    seg = jt.hia_segments_build(wl.samples, wl.S)
+    c, s = gpu_tables(seg, wl.D, wl.base)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = jt.hia_attn_fwd(seg, qd, kd, vd, c, s, wl.scale)
+    dq, dk, dv = jt.hia_attn_bwd(seg, qd, kd, vd, c, s, o, lse, dod, wl.scale)
+    torch.cuda.synchronize()
+    assert jt.hia_get_device_status() == 0
+    f = lambda t: t.float().cpu().numpy()
+    return (q, k, v, do), (f(dq), f(dk), f(dv))
+
+
+def check_bwd(oracle_mod, wl, inputs, grads, groups=None):
+    q, k, v, do = inputs
+    f64 = lambda t: t.double().numpy()
+    ref = oracle_mod.attn_bwd(wl.samples, f64(q), f64(k), f64(v), f64(do), wl.scale, wl.base,
+                              groups=groups)[:3]
+    g = wl.Hq // wl.Hkv
+    gsel = np.ones((wl.B, wl.Hkv), dtype=bool) if groups is None else np.asarray(groups, dtype=bool)
+    out = {}
+    for name, got, r in zip(("dq", "dk", "dv"), grads, ref):
+        per = g if name == "dq" else 1
+        a, bref = [], []
+        for b in range(wl.B):
+            for hk in range(wl.Hkv):
+                if gsel[b, hk]:
+                    a.append(got[b, :, hk * per:(hk + 1) * per])
+                    bref.append(r[b, :, hk * per:(hk + 1) * per])
+        a = np.concatenate([x.ravel() for x in a])
+        bref = np.concatenate([x.ravel() for x in bref])
+        assert np.all(np.isfinite(a)), f"{name} non-finite"
+        nr = np.linalg.norm(bref)
+        rel = np.linalg.norm(a - bref) / nr if nr > 0 else np.linalg.norm(a)
+        out[name] = rel
+        assert rel <= GRAD_REL, f"{name} relative Frobenius {rel:.3e}"
+    print(f"[parity-bwd] {wl.name}: " + " ".join(f"{k} {v:.3e}" for k, v in out.items()))
+    return out

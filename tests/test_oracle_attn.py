@@ -131,3 +131,17 @@ def test_bwd_finite_differences_through_rope(oracle_mod, D):
             fd[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
         err = np.linalg.norm(fd - g) / np.linalg.norm(g)
         assert err < 1e-6, (name, err)
+
+
+def test_bwd_row_subsets_are_partial_sums(oracle_mod):
+    """dQ of a row depends on that row only; dK, dV are sums over query rows,
+    so disjoint row subsets add up to the full gradient."""
+    rng = np.random.default_rng(9)
+    S, Hq, Hkv, D = 15, 4, 2, 16
+    q, k, v, do = _inputs(rng, S, Hq, Hkv, D, len(SAMPLES))
+    dq, dk, dv, _ = oracle_mod.attn_bwd(SAMPLES, q, k, v, do)
+    ra, rb = list(range(0, S, 2)), list(range(1, S, 2))
+    dqa, dka, dva, _ = oracle_mod.attn_bwd(SAMPLES, q, k, v, do, rows=ra)
+    dqb, dkb, dvb, _ = oracle_mod.attn_bwd(SAMPLES, q, k, v, do, rows=rb)
+    assert np.array_equal(dqa[:, ra], dq[:, ra]) and np.all(dqa[:, rb] == 0)
+    assert np.allclose(dka + dkb, dk, atol=1e-13) and np.allclose(dva + dvb, dv, atol=1e-13)
