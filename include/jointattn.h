@@ -38,7 +38,8 @@ typedef enum {
     HIA_ERR_UNSUPPORTED = 2,    /* D not in {64,128}, Hq % Hkv != 0, misaligned pointer/stride */
     HIA_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed */
     HIA_ERR_DEVICE_TIMEOUT = 4, /* a kernel's bounded wait expired (see hia_get_device_status) */
-    HIA_ERR_NOT_ON_DEVICE = 5   /* hia_segments used on the device before hia_segments_upload */
+    HIA_ERR_NOT_ON_DEVICE = 5,  /* hia_segments used on the device before hia_segments_upload */
+    HIA_ERR_SCRATCH_LIMIT = 6   /* problem larger than hia_attn_fwd_noalloc's fixed scratch */
 } hia_status;
 
 /* One sample of the batch.  Layout (HunyuanImage-3.0 coverage page, Cache
@@ -164,6 +165,34 @@ int hia_attn_fwd(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, 
                  hia_tensor v, const float* cos_t, const float* sin_t, float scale,
                  hia_tensor o, float* lse, void* workspace, size_t workspace_bytes,
                  void* stream);
+
+/* hia_attn_fwd for callers that cannot allocate device memory.  (No
+ * counterpart on the pages: this is a property of the library, not of the
+ * method.)  Some callers may not call cudaMalloc at all: a plug-in inside a
+ * host runtime that owns all device memory and passes it only its inputs and
+ * outputs, or a step that must not call cudaMalloc/cudaFree midway because
+ * they synchronize the device.  This entry point takes the same inputs and
+ * outputs as hia_attn_fwd but no workspace: the rotated q and k go into a
+ * fixed 64 MiB array compiled into the library (a __device__ variable), which
+ * every GPU that loads the library holds until the process exits.  It calls
+ * no cudaMalloc, cudaFree or other allocating routine.
+ *   - Limit: hia_attn_fwd_workspace_bytes(seg, Hq, Hkv, D) must not exceed
+ *     64 MiB = 67,108,864 bytes (B*S*(Hq+Hkv)*D*2 bytes
+ *     plus 256-byte alignment; e.g. one 1024px sample, S = 5122, Hq = 32, Hkv = 8,
+ *     D = 128 needs 52.5 MB).  Larger problems return HIA_ERR_SCRATCH_LIMIT
+ *     before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current), which also loads the
+ *     library module holding it; make that first call before any stream
+ *     capture on the device.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (nothing in it needs to start at zero: every element that is read is
+ *     first rewritten by the same call).  Calls whose GPU work overlaps, e.g.
+ *     on two streams, race on it: issue them on one stream or order them.
+ * Errors: those of hia_attn_fwd, plus HIA_ERR_SCRATCH_LIMIT. */
+int hia_attn_fwd_noalloc(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                         hia_tensor v, const float* cos_t, const float* sin_t, float scale,
+                         hia_tensor o, float* lse, void* stream);
 
 /* Bytes of device workspace hia_attn_bwd needs. */
 size_t hia_attn_bwd_workspace_bytes(const hia_segments* seg, int Hq, int Hkv, int D);

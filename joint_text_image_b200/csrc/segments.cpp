@@ -188,6 +188,7 @@ extern "C" const char* hia_status_string(int s) {
     case HIA_ERR_CUDA: return "CUDA error";
     case HIA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case HIA_ERR_NOT_ON_DEVICE: return "segments not uploaded to the device";
+    case HIA_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed 64 MiB scratch of hia_attn_fwd_noalloc";
     default: return "unknown status";
   }
 }
