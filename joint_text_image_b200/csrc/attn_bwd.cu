@@ -16,10 +16,14 @@
 //   P^T = exp2(S^T * scale*log2e - lse2), dS^T = P^T o (dP^T - delta)
 //   dV += P^T dO,  dK += dS^T Qr       (A = P^T / dS^T straight from TMEM)
 //   dQ^T = Kr^T dS^T                   (A = Kr read as MN-major, B = dS^T in
-//                                       shared memory) -> fp32 red.add
-// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 4-7 softmax (one key row
-// per thread, then the dK/dV epilogue with the inverse RoPE), 8-11 dQ
-// writers (one head-dim lane per thread, coalesced fp32 reductions).
+//                                       shared memory)
+// and dQ^T goes TMEM -> registers -> shared memory -> one bulk fp32
+// reduce-add into the dq accumulator (the reduction runs in L2).
+// Warps (512 threads): 0 TMA producer, 1 TMEM owner + MMA issuer, 4-7 and
+// 8-11 two softmax warpgroups that take alternate query tiles (one key row
+// per thread; then the dK and dV epilogues), 12-15 dQ writers (one head-dim
+// lane per thread).  setmaxnreg moves registers from the producer/MMA and dQ
+// warpgroups to the softmax warpgroups: 128*56 + 256*176 + 128*104 = 512*128.
 // TMEM: S^T[2] at 0/64, dP^T[2] at 128/192 (P^T, dS^T written over them as
 // packed bf16), dV at 256, dK at 256 + D; dQ^T of buffer i is written over
 // S^T[i] after the dV MMA that read P^T from there (MMAs run in issue order).
@@ -32,7 +36,8 @@
 namespace hia {
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int kLaunchRegs = 128;  // the setmaxnreg split below assumes 512 x 128 at launch
 constexpr int kStages = 3;
 constexpr int BK = kBwdBK;  // 128 keys
 constexpr int BQ = kBwdBQ;  // 64 query rows
@@ -44,6 +49,7 @@ struct BwdSmem {
   alignas(1024) __nv_bfloat16 q[kStages][BQ * D];
   alignas(1024) __nv_bfloat16 dout[kStages][BQ * D];
   alignas(1024) __nv_bfloat16 ds[2][BK * BQ];  // dS^T rows = keys, 64 q per 128-byte row
+  alignas(1024) float dq[2][(BQ / 2) * D];     // half query tile of dQ, fp32 [32 q][D]
   alignas(16) float lse2[kStages][BQ];
   alignas(16) float delta[kStages][BQ];
   uint64_t bar_kv;
@@ -156,7 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tdP[2] = {tmem + 128, tmem + 192};
   const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D;
 
-  if (warp == 0) {
+  if (warp < 4) {
+   regs_dec<56>();
+   if (warp == 0) {
     // =============================== TMA producer
     if (lane == 0 && n_it > 0) {
       tma_prefetch_desc(&tm_q);
@@ -224,16 +232,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(&sm.bar_final);
       mbar_wait_hw(&sm.bar_final, 0, wc);
     }
-  } else if (warp >= 4 && warp < 8) {
+   }
+  } else if (warp < 12) {
+    regs_inc<176>();
     // =============================== softmax: one key row per thread
+    const int bf = (warp - 4) >> 2;  // this warpgroup's TMEM / dS buffer and iteration parity
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int key = kt * BK + r;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const float cs = p.scale_log2;
     bool ok = true;
-    for (int i = 0; i < n_it; ++i) {
-      const int bf = i & 1, s = i % kStages;
+    for (int i = bf; i < n_it; i += 2) {
+      const int s = i % kStages;
       const int qt = qt_first + i % n_qt;
       const bool partial = qt < qt_full || (qt + 1) * BQ > p.S;
       // the stage's lse2/delta were written by TMA: acquire them through its barrier
@@ -246,9 +257,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tS[bf] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
       float pv[64];
-      const float* l2 = sm.lse2[s];
+      const float4* l2 = reinterpret_cast<const float4*>(sm.lse2[s]);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) pv[c] = ex2_approx(fmaf(__uint_as_float(sr[c]), cs, -l2[c]));
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l = l2[c4];
+        pv[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 0]), cs, -l.x));
+        pv[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), cs, -l.y));
+        pv[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), cs, -l.z));
+        pv[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), cs, -l.w));
+      }
       if (partial) {
         const int q0 = qt * BQ;
 #pragma unroll
@@ -269,11 +286,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tdP[bf] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(tdP[bf] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
-      const float* dl = sm.delta[s];
+      const float4* dl = reinterpret_cast<const float4*>(sm.delta[s]);
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
-        pk[c] = pack_bf16x2(pv[2 * c] * (__uint_as_float(sr[2 * c]) - dl[2 * c]),
-                            pv[2 * c + 1] * (__uint_as_float(sr[2 * c + 1]) - dl[2 * c + 1]));
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 d = dl[c4];
+        pk[2 * c4] = pack_bf16x2(pv[4 * c4 + 0] * (__uint_as_float(sr[4 * c4 + 0]) - d.x),
+                                 pv[4 * c4 + 1] * (__uint_as_float(sr[4 * c4 + 1]) - d.y));
+        pk[2 * c4 + 1] = pack_bf16x2(pv[4 * c4 + 2] * (__uint_as_float(sr[4 * c4 + 2]) - d.z),
+                                     pv[4 * c4 + 3] * (__uint_as_float(sr[4 * c4 + 3]) - d.w));
+      }
       tmem_st32(tdP[bf] + lane_off, pk);
       // dS^T row -> shared memory, 128-byte swizzled rows of 64 query values
       uint8_t* dsrow = reinterpret_cast<uint8_t*>(sm.ds[bf]);
@@ -286,98 +307,117 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&sm.bar_ds_ready[bf]);
     }
-    // ---- epilogue: dK = R^T (scale dKr), dV -> bf16
+    // ---- epilogue: warpgroup 0 writes dK = R^T (scale dKr), warpgroup 1 dV
     bool have = n_it > 0 && ok;
     if (have) have = __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, wc));
     if (have) tc_fence_after();
     const bool store = key < p.S;
-    const int kc = store ? key : p.S - 1;
-    const float* cp = p.cos_t + (int64_t(b) * p.S + kc) * D;
-    const float* sp = p.sin_t + (int64_t(b) * p.S + kc) * D;
-    __nv_bfloat16* dkrow = p.dk + int64_t(b) * p.dk_sb + int64_t(key) * p.dk_ss + int64_t(hkv) * p.dk_sh;
-    __nv_bfloat16* dvrow = p.dv + int64_t(b) * p.dv_sb + int64_t(key) * p.dv_ss + int64_t(hkv) * p.dv_sh;
+    if (bf == 0) {
+      const int kc = store ? key : p.S - 1;
+      const float* cp = p.cos_t + (int64_t(b) * p.S + kc) * D;
+      const float* sp = p.sin_t + (int64_t(b) * p.S + kc) * D;
+      __nv_bfloat16* dkrow = p.dk + int64_t(b) * p.dk_sb + int64_t(key) * p.dk_ss + int64_t(hkv) * p.dk_sh;
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t lo[32], hi[32];
+        if (have) {
+          tmem_ld32(tdK + lane_off + c * 32, lo);
+          tmem_ld32(tdK + lane_off + D / 2 + c * 32, hi);
+          tmem_ld_wait();
+        } else {
 #pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      uint32_t lo[32], hi[32];
-      if (have) {
-        tmem_ld32(tdK + lane_off + c * 32, lo);
-        tmem_ld32(tdK + lane_off + D / 2 + c * 32, hi);
-        tmem_ld_wait();
-      } else {
+          for (int i = 0; i < 32; ++i) lo[i] = hi[i] = 0u;
+        }
+        if (store) {
+          uint32_t olo[16], ohi[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) lo[i] = hi[i] = 0u;
-      }
-      if (store) {
-        uint32_t olo[16], ohi[16];
+          for (int i = 0; i < 16; ++i) {
+            float a[2], bb[2];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float a[2], bb[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int j = c * 32 + 2 * i + e;
-            const float cj = __ldg(cp + j), sj = __ldg(sp + j);
-            const float l = __uint_as_float(lo[2 * i + e]) * p.scale, u = __uint_as_float(hi[2 * i + e]) * p.scale;
-            a[e] = fmaf(l, cj, u * sj);
-            bb[e] = fmaf(u, cj, -l * sj);
+            for (int e = 0; e < 2; ++e) {
+              const int j = c * 32 + 2 * i + e;
+              const float cj = __ldg(cp + j), sj = __ldg(sp + j);
+              const float l = __uint_as_float(lo[2 * i + e]) * p.scale, u = __uint_as_float(hi[2 * i + e]) * p.scale;
+              a[e] = fmaf(l, cj, u * sj);
+              bb[e] = fmaf(u, cj, -l * sj);
+            }
+            olo[i] = pack_bf16x2(a[0], a[1]);
+            ohi[i] = pack_bf16x2(bb[0], bb[1]);
           }
-          olo[i] = pack_bf16x2(a[0], a[1]);
-          ohi[i] = pack_bf16x2(bb[0], bb[1]);
-        }
-        uint4* d0 = reinterpret_cast<uint4*>(dkrow + c * 32);
-        uint4* d1 = reinterpret_cast<uint4*>(dkrow + D / 2 + c * 32);
+          uint4* d0 = reinterpret_cast<uint4*>(dkrow + c * 32);
+          uint4* d1 = reinterpret_cast<uint4*>(dkrow + D / 2 + c * 32);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          d0[i] = make_uint4(olo[4 * i], olo[4 * i + 1], olo[4 * i + 2], olo[4 * i + 3]);
-          d1[i] = make_uint4(ohi[4 * i], ohi[4 * i + 1], ohi[4 * i + 2], ohi[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) {
+            d0[i] = make_uint4(olo[4 * i], olo[4 * i + 1], olo[4 * i + 2], olo[4 * i + 3]);
+            d1[i] = make_uint4(ohi[4 * i], ohi[4 * i + 1], ohi[4 * i + 2], ohi[4 * i + 3]);
+          }
+        }
+      }
+    } else {
+      __nv_bfloat16* dvrow = p.dv + int64_t(b) * p.dv_sb + int64_t(key) * p.dv_ss + int64_t(hkv) * p.dv_sh;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        if (have) {
+          tmem_ld32(tdV + lane_off + c * 32, ov);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = 0u;
+        }
+        if (store) {
+          uint4* d0 = reinterpret_cast<uint4*>(dvrow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            d0[i] = make_uint4(pack_bf16x2(__uint_as_float(ov[8 * i]), __uint_as_float(ov[8 * i + 1])),
+                               pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3])),
+                               pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5])),
+                               pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7])));
         }
       }
     }
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t ov[32];
-      if (have) {
-        tmem_ld32(tdV + lane_off + c * 32, ov);
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] = 0u;
-      }
-      if (store) {
-        uint4* d0 = reinterpret_cast<uint4*>(dvrow + c * 32);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          d0[i] = make_uint4(pack_bf16x2(__uint_as_float(ov[8 * i]), __uint_as_float(ov[8 * i + 1])),
-                             pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3])),
-                             pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5])),
-                             pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7])));
-      }
-    }
-  } else if (warp >= 8) {
+  } else {
     // =============================== dQ writers: one head-dim lane per thread
+    regs_dec<104>();
     const int quarter = warp & 3;
     const int d = quarter * 32 + lane;
+    const bool leader = warp == 12 && lane == 0;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    const bool live = quarter * 32 < D;  // warp-uniform
+    const bool live = quarter * 32 < D;  // warp-uniform (D = 64 uses lanes 0-63 only)
     for (int i = 0; i < n_it; ++i) {
       const int bf = i & 1;
       const int hi = i / n_qt, qt = qt_first + i % n_qt;
       const int h = hkv * p.g + hi;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dq_full[bf], (i >> 1) & 1, wc))) break;
       tc_fence_after();
+      uint32_t a[64];
       if (live) {
-        uint32_t a[32], c2[32];
-        tmem_ld32(tS[bf] + lane_off, a);
-        tmem_ld32(tS[bf] + lane_off + 32, c2);
+        tmem_ld32(tS[bf] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+        tmem_ld32(tS[bf] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
         tmem_ld_wait();
-        float* dst = p.dq_acc + ((int64_t(b) * p.Hq + h) * p.S_pad + int64_t(qt) * BQ) * D + d;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) red_add_f32(dst + int64_t(c) * D, __uint_as_float(a[c]));
-#pragma unroll
-        for (int c = 0; c < 32; ++c) red_add_f32(dst + int64_t(c + 32) * D, __uint_as_float(c2[c]));
       }
       tc_fence_before();
       mbar_arrive(&sm.bar_dq_empty[bf]);
+      float* dst = p.dq_acc + ((int64_t(b) * p.Hq + h) * p.S_pad + int64_t(qt) * BQ) * D;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        // buffer hh was last handed to the bulk engine two groups ago
+        if (leader) bulk_wait_group_read<1>();
+        named_bar_sync(1, 128);
+        if (live) {
+          float* t = sm.dq[hh];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) t[c * D + d] = __uint_as_float(a[hh * 32 + c]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (leader) {
+          bulk_reduce_add_f32(dst + hh * (BQ / 2) * D, sm.dq[hh], (BQ / 2) * D * 4);
+          bulk_commit_group();
+        }
+      }
     }
+    if (leader) bulk_wait_group<0>();
   }
   __syncwarp();
 
@@ -449,8 +489,13 @@ cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st) {
 cudaError_t launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const BwdParams& p, int n_blocks, int D, cudaStream_t st) {
   if (n_blocks == 0) return cudaSuccess;
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, D == 128 ? attn_bwd_kernel<128> : attn_bwd_kernel<64>) != cudaSuccess ||
+      fa.numRegs != kLaunchRegs)
+    return cudaErrorInvalidConfiguration;
   prof_begin(kAttnBwd, st);
   if (D == 128) {
+    static_assert(sizeof(BwdSmem<128>) + 1024 <= 232448, "shared memory budget");
     const size_t smem = sizeof(BwdSmem<128>) + 1024;
     cudaFuncSetAttribute(attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     attn_bwd_kernel<128><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, tdo, p);

@@ -32,6 +32,10 @@ namespace hia {
 namespace {
 
 constexpr int kThreads = 384;
+// Register split (setmaxnreg): launch budget 384 x 168; warpgroup 0 (TMA, MMA)
+// drops to 56, the two softmax warpgroups rise to 224:
+// 128*56 + 256*224 = 384*168.  The launcher checks the compiled count first.
+constexpr int kLaunchRegs = 168;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 
 template <int D>
@@ -119,7 +123,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const WaitCtx wc{&sm.abort_flag, p.status, p.timeout_ns};
 
-  if (warp == 0) {
+  if (warp < 4) {
+   regs_dec<56>();
+   if (warp == 0) {
     // =============================== TMA producer
     if (lane == 0 && n_vis > 0) {
       tma_prefetch_desc(&tm_q);
@@ -186,7 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // MMAs already issued must finish before TMEM can be released.
       mbar_wait_hw(&sm.bar_o_final[0], 0, wc);
     }
-  } else if (warp >= 4) {
+   }
+  } else {
+    regs_inc<224>();
     // =============================== softmax / epilogue
     // tcgen05.ld/st are warp-collective: every branch around them below is
     // warp-uniform (waits are combined with __all_sync, the O rescale is
@@ -218,10 +226,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (c > lim) sr[c] = __float_as_uint(-INFINITY);
       }
-      float mx = __uint_as_float(sr[0]);
+      // row max with 8 independent partial maxima (short dependency chains)
+      float mp[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
-      const float xmax = mx * cs;
+      for (int c = 0; c < 8; ++c) mp[c] = __uint_as_float(sr[c]);
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
+      const float xmax = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * cs;
       if (j == 0) {
         m = xmax;
       } else {
@@ -242,13 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       uint32_t pk[64];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), cs, -m));
         const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), cs, -m));
-        l += p0 + p1;
+        ls[c & 3] += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
       }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_st_wait();
@@ -304,6 +318,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int n_blocks, int D, cudaStream_t st) {
   if (n_blocks == 0) return cudaSuccess;
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, D == 128 ? attn_fwd_kernel<128> : attn_fwd_kernel<64>) != cudaSuccess ||
+      fa.numRegs != kLaunchRegs)
+    return cudaErrorInvalidConfiguration;  // the setmaxnreg split assumes kLaunchRegs
   prof_begin(kAttnFwd, st);
   if (D == 128) {
     const size_t smem = sizeof(FwdSmem<128>) + 1024;
