@@ -23,7 +23,7 @@
 // 8-11 two softmax warpgroups that take alternate query tiles (one key row
 // per thread; then the dK and dV epilogues), 12-15 dQ writers (one head-dim
 // lane per thread).  setmaxnreg moves registers from the producer/MMA and dQ
-// warpgroups to the softmax warpgroups: 128*56 + 256*176 + 128*104 = 512*128.
+// warpgroups to the softmax warpgroups: 128*80 + 256*168 + 128*96 = 65536 = 512*128.
 // TMEM: S^T[2] at 0/64, dP^T[2] at 128/192 (P^T, dS^T written over them as
 // packed bf16), dV at 256, dK at 256 + D; dQ^T of buffer i is written over
 // S^T[i] after the dV MMA that read P^T from there (MMAs run in issue order).
@@ -66,45 +66,31 @@ struct BwdSmem {
   int abort_flag;
 };
 
-// S^T / dP^T: A = 128-row tile (K-major, 64-wide D blocks 16 KB apart),
-// B = 64-row tile (K-major, D blocks 8 KB apart).
+// S^T = Kr Qr^T and dP^T = V dO^T: A = 128-row tile (K-major, 64-wide D
+// blocks 16 KB apart), B = 64-row tile (K-major, D blocks 8 KB apart); N = 64.
 template <int D>
-__device__ __forceinline__ void issue_kq(uint32_t d, const __nv_bfloat16* a, const __nv_bfloat16* b) {
+__device__ __forceinline__ void issue_kq(uint32_t d, uint64_t adesc, uint64_t bdesc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, BQ, 0, 0);
-  const uint32_t aa = smem_u32(a), ba = smem_u32(b);
-#pragma unroll
-  for (int kb = 0; kb < D / 16; ++kb) {
-    const uint32_t in = uint32_t(kb & 3) * 32u;
-    mma_ss(d, sdesc_sw128(aa + uint32_t(kb >> 2) * 16384u + in, 16, 1024),
-           sdesc_sw128(ba + uint32_t(kb >> 2) * 8192u + in, 16, 1024), idesc, kb > 0 ? 1u : 0u);
-  }
+  constexpr KMajorSteps<D / 16> sa(16384), sb(8192);
+  mma_chain_ss<D / 16>(d, adesc, sa.v, bdesc, sb.v, idesc, 0u);
 }
 
 // dV += P^T dO or dK += dS^T Qr: A from TMEM (128 keys x 64 q, packed bf16),
 // B = 64-row tile read MN-major (N = D contiguous, D blocks 8 KB apart).
 template <int D>
-__device__ __forceinline__ void issue_acc(uint32_t d, uint32_t a_tmem, const __nv_bfloat16* b, bool acc) {
+__device__ __forceinline__ void issue_acc(uint32_t d, uint32_t a_tmem, uint64_t bdesc, bool acc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
-  const uint32_t ba = smem_u32(b);
-#pragma unroll
-  for (int kb = 0; kb < BQ / 16; ++kb)
-    mma_ts(d, a_tmem + uint32_t(kb) * 8u, sdesc_sw128(ba + uint32_t(kb) * 2048u, 8192, 1024), idesc,
-           (acc || kb > 0) ? 1u : 0u);
+  constexpr MNMajorSteps<BQ / 16> st;
+  mma_chain_ts<BQ / 16>(d, a_tmem, 8u, bdesc, st.v, idesc, acc ? 1u : 0u);
 }
 
 // dQ^T = Kr^T dS^T: M = 128 (head dims; for D = 64 the second 64-row block
 // reads the V tile and its result lanes are ignored), N = 64 q, K = 128 keys.
 // A = Kr tile read MN-major, B = dS^T tile read MN-major.
-template <int D>
-__device__ __forceinline__ void issue_dq(uint32_t d, const __nv_bfloat16* kt, const __nv_bfloat16* vt,
-                                         const __nv_bfloat16* ds) {
+__device__ __forceinline__ void issue_dq(uint32_t d, uint64_t kt_mn_desc, uint64_t ds_desc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, BQ, 1, 1);
-  const uint32_t ka = smem_u32(kt), da = smem_u32(ds);
-  const uint32_t lbo = (D == 128) ? 16384u : (smem_u32(vt) - ka);
-#pragma unroll
-  for (int kb = 0; kb < BK / 16; ++kb)
-    mma_ss(d, sdesc_sw128(ka + uint32_t(kb) * 2048u, lbo, 1024), sdesc_sw128(da + uint32_t(kb) * 2048u, 8192, 1024),
-           idesc, kb > 0 ? 1u : 0u);
+  constexpr MNMajorSteps<BK / 16> st;
+  mma_chain_ss<BK / 16>(d, kt_mn_desc, st.v, ds_desc, st.v, idesc, 0u);
 }
 
 __device__ __forceinline__ void red_add_f32(float* p, float v) {
@@ -163,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D;
 
   if (warp < 4) {
-   regs_dec<56>();
+   regs_dec<80>();
    if (warp == 0) {
     // =============================== TMA producer
     if (lane == 0 && n_it > 0) {
@@ -198,12 +184,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // =============================== MMA issuer
     if (lane == 0 && n_it > 0) {
+      // descriptor bases; the stages of q / dout and the two dS buffers are adjacent
+      const uint64_t k_km = sdesc_sw128(smem_u32(sm.k), 16, 1024);
+      const uint64_t k_mn = sdesc_sw128(smem_u32(sm.k), D == 128 ? 16384u : smem_u32(sm.v) - smem_u32(sm.k), 1024);
+      const uint64_t v_km = sdesc_sw128(smem_u32(sm.v), 16, 1024);
+      const uint64_t q_km = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
+      const uint64_t q_mn = sdesc_sw128(smem_u32(sm.q[0]), 8192, 1024);
+      const uint64_t o_km = sdesc_sw128(smem_u32(sm.dout[0]), 16, 1024);
+      const uint64_t o_mn = sdesc_sw128(smem_u32(sm.dout[0]), 8192, 1024);
+      const uint64_t ds_mn = sdesc_sw128(smem_u32(sm.ds[0]), 8192, 1024);
+      constexpr uint32_t kQStep = (BQ * D * 2u) >> 4, kDsStep = (BK * BQ * 2u) >> 4;
       bool ok = mbar_wait(&sm.bar_kv, 0, wc) && mbar_wait(&sm.bar_full[0], 0, wc);
       if (ok) {
         tc_fence_after();
-        issue_kq<D>(tS[0], sm.k, sm.q[0]);
+        issue_kq<D>(tS[0], k_km, q_km);
         tc_commit(&sm.bar_s_full[0]);
-        issue_kq<D>(tdP[0], sm.v, sm.dout[0]);
+        issue_kq<D>(tdP[0], v_km, o_km);
         tc_commit(&sm.bar_dp_full[0]);
       }
       for (int i = 0; ok && i < n_it; ++i) {
@@ -214,18 +210,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok && i1 >= 2) ok = mbar_wait(&sm.bar_dq_empty[b1], ((i1 >> 1) - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after();
-          issue_kq<D>(tS[b1], sm.k, sm.q[s1]);
+          issue_kq<D>(tS[b1], k_km, q_km + uint32_t(s1) * kQStep);
           tc_commit(&sm.bar_s_full[b1]);
-          issue_kq<D>(tdP[b1], sm.v, sm.dout[s1]);
+          issue_kq<D>(tdP[b1], v_km, o_km + uint32_t(s1) * kQStep);
           tc_commit(&sm.bar_dp_full[b1]);
         }
         if (!mbar_wait(&sm.bar_p_ready[bf], (i >> 1) & 1, wc)) { ok = false; break; }
         tc_fence_after();
-        issue_acc<D>(tdV, tS[bf], sm.dout[s], i > 0);
+        issue_acc<D>(tdV, tS[bf], o_mn + uint32_t(s) * kQStep, i > 0);
         if (!mbar_wait(&sm.bar_ds_ready[bf], (i >> 1) & 1, wc)) { ok = false; break; }
         tc_fence_after();
-        issue_acc<D>(tdK, tdP[bf], sm.q[s], i > 0);
-        issue_dq<D>(tS[bf], sm.k, sm.v, sm.ds[bf]);
+        issue_acc<D>(tdK, tdP[bf], q_mn + uint32_t(s) * kQStep, i > 0);
+        issue_dq(tS[bf], k_mn, ds_mn + uint32_t(bf) * kDsStep);
         tc_commit(&sm.bar_dq_full[bf]);
         tc_commit(&sm.bar_empty[s]);
       }
@@ -234,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
    }
   } else if (warp < 12) {
-    regs_inc<176>();
+    regs_inc<168>();
     // =============================== softmax: one key row per thread
     const int bf = (warp - 4) >> 2;  // this warpgroup's TMEM / dS buffer and iteration parity
     const int quarter = warp & 3;
@@ -378,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // =============================== dQ writers: one head-dim lane per thread
-    regs_dec<104>();
+    regs_dec<96>();
     const int quarter = warp & 3;
     const int d = quarter * 32 + lane;
     const bool leader = warp == 12 && lane == 0;

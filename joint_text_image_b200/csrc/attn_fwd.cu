@@ -33,8 +33,8 @@ namespace {
 
 constexpr int kThreads = 384;
 // Register split (setmaxnreg): launch budget 384 x 168; warpgroup 0 (TMA, MMA)
-// drops to 56, the two softmax warpgroups rise to 224:
-// 128*56 + 256*224 = 384*168.  The launcher checks the compiled count first.
+// drops to 88, the two softmax warpgroups rise to 208:
+// 128*88 + 256*208 = 64512 = 384*168.  The launcher checks the compiled count first.
 constexpr int kLaunchRegs = 168;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 
@@ -55,27 +55,22 @@ struct FwdSmem {
   int abort_flag;
 };
 
+// S_t = Q_t K^T: M = 128 query rows, N = 128 keys, K = D.  Both operands
+// K-major, 64-wide D blocks 16 KB apart.
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t tS, const __nv_bfloat16* q, const __nv_bfloat16* k) {
+__device__ __forceinline__ void issue_qk(uint32_t tS, uint64_t qdesc, uint64_t kdesc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
-  const uint32_t qa = smem_u32(q), ka = smem_u32(k);
-#pragma unroll
-  for (int kb = 0; kb < D / 16; ++kb) {
-    const uint32_t off = uint32_t(kb >> 2) * 16384u + uint32_t(kb & 3) * 32u;
-    mma_ss(tS, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc, kb > 0 ? 1u : 0u);
-  }
+  constexpr KMajorSteps<D / 16> st(16384);
+  mma_chain_ss<D / 16>(tS, qdesc, st.v, kdesc, st.v, idesc, 0u);
 }
 
+// O_t (+)= P_t V: A = P_t from TMEM (packed bf16, 8 columns per 16 keys),
+// B = V tile [128 keys][D] read MN-major (D blocks 16 KB apart, 2 KB per 16 keys).
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, const __nv_bfloat16* v, bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint64_t vdesc, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
-  const uint32_t va = smem_u32(v);
-#pragma unroll
-  for (int kb = 0; kb < 8; ++kb) {
-    // V tile: [128 keys][D], 64-wide D blocks 16 KB apart; 16 keys = 2 KB.
-    const uint64_t bd = sdesc_sw128(va + uint32_t(kb) * 2048u, 16384, 1024);
-    mma_ts(tO, tP + uint32_t(kb) * 8u, bd, idesc, (accumulate || kb > 0) ? 1u : 0u);
-  }
+  constexpr MNMajorSteps<8> st;
+  mma_chain_ts<8>(tO, tP, 8u, vdesc, st.v, idesc, accumulate ? 1u : 0u);
 }
 
 template <int D>
@@ -124,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wc{&sm.abort_flag, p.status, p.timeout_ns};
 
   if (warp < 4) {
-   regs_dec<56>();
+   regs_dec<88>();
    if (warp == 0) {
     // =============================== TMA producer
     if (lane == 0 && n_vis > 0) {
@@ -161,11 +156,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n_vis > 0) {
       uint32_t tS[2] = {tmem, tmem + 128};
       uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      // descriptor bases (start address of each buffer); stages are adjacent
+      const uint64_t qd[2] = {sdesc_sw128(smem_u32(sm.q[0]), 16, 1024), sdesc_sw128(smem_u32(sm.q[1]), 16, 1024)};
+      const uint64_t kd0 = sdesc_sw128(smem_u32(sm.k[0]), 16, 1024);
+      const uint64_t vd0 = sdesc_sw128(smem_u32(sm.v[0]), 16384, 1024);
+      constexpr uint32_t kStageStep = (128u * D * 2u) >> 4;  // one K or V stage, 16-byte units
       bool ok = mbar_wait(&sm.bar_q, 0, wc) && mbar_wait(&sm.bar_k_full[0], 0, wc);
       if (ok) {
         tc_fence_after();
         for (int t = 0; t < n_tiles; ++t) {
-          issue_qk<D>(tS[t], sm.q[t], sm.k[0]);
+          issue_qk<D>(tS[t], qd[t], kd0);
           tc_commit(&sm.bar_s_full[t]);
         }
       }
@@ -175,13 +175,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < n_tiles; ++t) {
           if (!mbar_wait(&sm.bar_p_ready[t], j & 1, wc)) { ok = false; break; }
           tc_fence_after();
-          issue_pv<D>(tO[t], tS[t], sm.v[s], j > 0);
+          issue_pv<D>(tO[t], tS[t], vd0 + uint32_t(s) * kStageStep, j > 0);
           if (j + 1 < n_vis) {
             if (t == 0) {
               if (!mbar_wait(&sm.bar_k_full[s1], ((j + 1) >> 1) & 1, wc)) { ok = false; break; }
               tc_fence_after();
             }
-            issue_qk<D>(tS[t], sm.q[t], sm.k[s1]);
+            issue_qk<D>(tS[t], qd[t], kd0 + uint32_t(s1) * kStageStep);
             tc_commit(&sm.bar_s_full[t]);
           }
         }
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
    }
   } else {
-    regs_inc<224>();
+    regs_inc<208>();
     // =============================== softmax / epilogue
     // tcgen05.ld/st are warp-collective: every branch around them below is
     // warp-uniform (waits are combined with __all_sync, the O rescale is

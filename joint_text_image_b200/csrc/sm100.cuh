@@ -239,6 +239,54 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
          (uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
+// Issue a chain of kind::f16 MMAs whose descriptors are `base + offset`
+// (offsets in 16-byte units, compile-time constants).  All descriptors are
+// formed before the first MMA so the single issuing thread never waits on
+// address arithmetic between MMAs (that dependency chain, not the tensor
+// core, bounded the issue rate to ~100 clocks per MMA).
+template <int NK>
+__device__ __forceinline__ void mma_chain_ss(uint32_t d, uint64_t abase, const uint32_t (&aoff)[NK], uint64_t bbase,
+                                             const uint32_t (&boff)[NK], uint32_t idesc, uint32_t acc_first) {
+  uint64_t a[NK], b[NK];
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    a[i] = abase + aoff[i];
+    b[i] = bbase + boff[i];
+  }
+#pragma unroll
+  for (int i = 0; i < NK; ++i) mma_ss(d, a[i], b[i], idesc, i == 0 ? acc_first : 1u);
+}
+template <int NK>
+__device__ __forceinline__ void mma_chain_ts(uint32_t d, uint32_t a_tmem, uint32_t a_step, uint64_t bbase,
+                                             const uint32_t (&boff)[NK], uint32_t idesc, uint32_t acc_first) {
+  uint64_t b[NK];
+  uint32_t a[NK];
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    b[i] = bbase + boff[i];
+    a[i] = a_tmem + uint32_t(i) * a_step;
+  }
+#pragma unroll
+  for (int i = 0; i < NK; ++i) mma_ts(d, a[i], b[i], idesc, i == 0 ? acc_first : 1u);
+}
+// Offsets (16-byte units) of the K-steps of a K-major SW128 operand whose
+// 64-wide K blocks are `block_bytes` apart: 32 bytes per 16-element step.
+template <int NK>
+struct KMajorSteps {
+  uint32_t v[NK];
+  __host__ __device__ constexpr KMajorSteps(uint32_t block_bytes) : v{} {
+    for (int i = 0; i < NK; ++i) v[i] = (uint32_t(i >> 2) * block_bytes + uint32_t(i & 3) * 32u) >> 4;
+  }
+};
+// Offsets of the K-steps of an MN-major SW128 operand: 16 K rows (2 KB) per step.
+template <int NK>
+struct MNMajorSteps {
+  uint32_t v[NK];
+  __host__ __device__ constexpr MNMajorSteps() : v{} {
+    for (int i = 0; i < NK; ++i) v[i] = uint32_t(i) * (2048u >> 4);
+  }
+};
+
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
