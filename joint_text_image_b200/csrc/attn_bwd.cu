@@ -24,7 +24,8 @@
 // per thread; then the dK and dV epilogues), 12-15 dQ writers (one head-dim
 // lane per thread).  setmaxnreg moves registers from the producer/MMA and dQ
 // warpgroups to the softmax warpgroups: 128*80 + 256*168 + 128*96 = 65536 = 512*128.
-// TMEM: S^T[2] at 0/64, dP^T[2] at 128/192 (P^T, dS^T written over them as
+// P^T and dS^T become visible to the MMA thread together (one barrier per
+// tile).  TMEM: S^T[2] at 0/64, dP^T[2] at 128/192 (P^T, dS^T written over them as
 // packed bf16), dV at 256, dK at 256 + D; dQ^T of buffer i is written over
 // S^T[i] after the dV MMA that read P^T from there (MMAs run in issue order).
 #include <cuda.h>
@@ -57,7 +58,6 @@ struct BwdSmem {
   uint64_t bar_empty[kStages];
   uint64_t bar_s_full[2];
   uint64_t bar_dp_full[2];
-  uint64_t bar_p_ready[2];
   uint64_t bar_ds_ready[2];
   uint64_t bar_dq_full[2];
   uint64_t bar_dq_empty[2];
@@ -126,7 +126,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.bar_s_full[i], 1);
       mbar_init(&sm.bar_dp_full[i], 1);
-      mbar_init(&sm.bar_p_ready[i], 128);
       mbar_init(&sm.bar_ds_ready[i], 128);
       mbar_init(&sm.bar_dq_full[i], 1);
       mbar_init(&sm.bar_dq_empty[i], 128);
@@ -204,22 +203,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int i = 0; ok && i < n_it; ++i) {
         const int bf = i & 1, s = i % kStages;
+        // Every wait/fence in this thread lets the short MMA queue drain, so the
+        // loop has two synchronisation points per query tile: (1) the next
+        // tile's operands are loaded and its TMEM buffer was read out by the dQ
+        // writers, (2) this tile's dS^T (hence also P^T) is ready.
         if (i + 1 < n_it) {
           const int i1 = i + 1, b1 = i1 & 1, s1 = i1 % kStages;
           ok = mbar_wait(&sm.bar_full[s1], (i1 / kStages) & 1, wc);
           if (ok && i1 >= 2) ok = mbar_wait(&sm.bar_dq_empty[b1], ((i1 >> 1) - 1) & 1, wc);
           if (!ok) break;
-          tc_fence_after();
+          if (i1 >= 2) tc_fence_after();  // TMEM reuse after the dQ writers' loads
           issue_kq<D>(tS[b1], k_km, q_km + uint32_t(s1) * kQStep);
           tc_commit(&sm.bar_s_full[b1]);
           issue_kq<D>(tdP[b1], v_km, o_km + uint32_t(s1) * kQStep);
           tc_commit(&sm.bar_dp_full[b1]);
         }
-        if (!mbar_wait(&sm.bar_p_ready[bf], (i >> 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        issue_acc<D>(tdV, tS[bf], o_mn + uint32_t(s) * kQStep, i > 0);
         if (!mbar_wait(&sm.bar_ds_ready[bf], (i >> 1) & 1, wc)) { ok = false; break; }
         tc_fence_after();
+        issue_acc<D>(tdV, tS[bf], o_mn + uint32_t(s) * kQStep, i > 0);
         issue_acc<D>(tdK, tdP[bf], q_mn + uint32_t(s) * kQStep, i > 0);
         issue_dq(tS[bf], k_mn, ds_mn + uint32_t(bf) * kDsStep);
         tc_commit(&sm.bar_dq_full[bf]);
@@ -272,9 +273,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
       tmem_st32(tS[bf] + lane_off, pk);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&sm.bar_p_ready[bf]);
 
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_dp_full[bf], (i >> 1) & 1, wc));
       if (!ok) break;

@@ -12,7 +12,8 @@
 // registers, fully masked and padded tiles are never loaded.
 //
 // Warp roles (384 threads):
-//   warp 0      TMA producer: Q tiles once, then K/V tiles into a 2-stage ring
+//   warp 0      TMA producer: Q tiles once, then K tiles (3-stage ring) and V
+//               tiles (2-stage ring)
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer
 //   warps 4-7   softmax / correction / epilogue of tile 0 (one row per thread)
 //   warps 8-11  the same for tile 1
@@ -38,16 +39,20 @@ constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 
+constexpr int kKStages = 3;  // K(j+1) is awaited together with V(j), so K runs one stage deeper
+constexpr int kVStages = 2;
+
 template <int D>
 struct FwdSmem {
   static constexpr int kTileElems = 128 * D;
   alignas(1024) __nv_bfloat16 q[2][kTileElems];
-  alignas(1024) __nv_bfloat16 k[2][kTileElems];
-  alignas(1024) __nv_bfloat16 v[2][kTileElems];
+  alignas(1024) __nv_bfloat16 k[kKStages][kTileElems];
+  alignas(1024) __nv_bfloat16 v[kVStages][kTileElems];
   uint64_t bar_q;
-  uint64_t bar_k_full[2];
-  uint64_t bar_v_full[2];
-  uint64_t bar_kv_empty[2];
+  uint64_t bar_k_full[kKStages];
+  uint64_t bar_k_empty[kKStages];
+  uint64_t bar_v_full[kVStages];
+  uint64_t bar_v_empty[kVStages];
   uint64_t bar_s_full[2];
   uint64_t bar_p_ready[2];
   uint64_t bar_o_final[2];
@@ -97,10 +102,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(&sm.bar_k_full[i], 1);
+      mbar_init(&sm.bar_k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(&sm.bar_v_full[i], 1);
-      mbar_init(&sm.bar_kv_empty[i], 1);
+      mbar_init(&sm.bar_v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.bar_s_full[i], 1);
       mbar_init(&sm.bar_p_ready[i], 128);
       mbar_init(&sm.bar_o_final[i], 1);
@@ -131,25 +141,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < n_tiles; ++t)
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(&sm.q[t][c * 128 * 64], &tm_q, &sm.bar_q, c * 64, qt * 128, b * p.Hq + h0 + t);
-      int issued = 0;
+      int kiss = 0, viss = 0;
       for (int j = 0; j < n_vis; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !mbar_wait(&sm.bar_kv_empty[s], ((j >> 1) - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(&sm.bar_k_full[s], tile_bytes);
+        const int ks = j % kKStages, vs = j % kVStages;
+        if (j >= kKStages && !mbar_wait(&sm.bar_k_empty[ks], ((j / kKStages) - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&sm.bar_k_full[ks], tile_bytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(&sm.k[s][c * 128 * 64], &tm_k, &sm.bar_k_full[s], c * 64, j * 128, b * p.Hkv + hkv);
-        mbar_arrive_expect_tx(&sm.bar_v_full[s], tile_bytes);
+          tma_load_3d(&sm.k[ks][c * 128 * 64], &tm_k, &sm.bar_k_full[ks], c * 64, j * 128, b * p.Hkv + hkv);
+        kiss = j + 1;
+        if (j >= kVStages && !mbar_wait(&sm.bar_v_empty[vs], ((j / kVStages) - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&sm.bar_v_full[vs], tile_bytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(&sm.v[s][c * 128 * 64], &tm_v, &sm.bar_v_full[s], c * 64, hkv, j * 128, b);
-        issued = j + 1;
+          tma_load_4d(&sm.v[vs][c * 128 * 64], &tm_v, &sm.bar_v_full[vs], c * 64, hkv, j * 128, b);
+        viss = j + 1;
       }
       // Drain: the copies this CTA issued must land before its shared memory
       // can be released, whatever the consumers did.
       mbar_wait_hw(&sm.bar_q, 0, wc);
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
-        mbar_wait_hw(&sm.bar_k_full[j & 1], (j >> 1) & 1, wc);
-        mbar_wait_hw(&sm.bar_v_full[j & 1], (j >> 1) & 1, wc);
-      }
+      for (int j = (kiss > kKStages ? kiss - kKStages : 0); j < kiss; ++j)
+        mbar_wait_hw(&sm.bar_k_full[j % kKStages], (j / kKStages) & 1, wc);
+      for (int j = (viss > kVStages ? viss - kVStages : 0); j < viss; ++j)
+        mbar_wait_hw(&sm.bar_v_full[j % kVStages], (j / kVStages) & 1, wc);
     }
   } else if (warp == 1) {
     // =============================== MMA issuer
@@ -163,30 +175,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kStageStep = (128u * D * 2u) >> 4;  // one K or V stage, 16-byte units
       bool ok = mbar_wait(&sm.bar_q, 0, wc) && mbar_wait(&sm.bar_k_full[0], 0, wc);
       if (ok) {
-        tc_fence_after();
         for (int t = 0; t < n_tiles; ++t) {
           issue_qk<D>(tS[t], qd[t], kd0);
           tc_commit(&sm.bar_s_full[t]);
         }
+        tc_commit(&sm.bar_k_empty[0]);
       }
+      // Every wait/fence in this thread lets the short MMA queue drain, so each
+      // kv step has two synchronisation points, one per query tile: (1) V(j),
+      // K(j+1) loaded and P0(j) written; (2) P1(j) written.
       for (int j = 0; ok && j < n_vis; ++j) {
-        const int s = j & 1, s1 = (j + 1) & 1;
-        if (!mbar_wait(&sm.bar_v_full[s], (j >> 1) & 1, wc)) { ok = false; break; }
+        const int vs = j % kVStages, ks1 = (j + 1) % kKStages;
+        const bool more = j + 1 < n_vis;
         for (int t = 0; t < n_tiles; ++t) {
+          if (t == 0) {
+            ok = mbar_wait(&sm.bar_v_full[vs], (j / kVStages) & 1, wc) &&
+                 (!more || mbar_wait(&sm.bar_k_full[ks1], ((j + 1) / kKStages) & 1, wc));
+            if (!ok) break;
+          }
           if (!mbar_wait(&sm.bar_p_ready[t], j & 1, wc)) { ok = false; break; }
           tc_fence_after();
-          issue_pv<D>(tO[t], tS[t], vd0 + uint32_t(s) * kStageStep, j > 0);
-          if (j + 1 < n_vis) {
-            if (t == 0) {
-              if (!mbar_wait(&sm.bar_k_full[s1], ((j + 1) >> 1) & 1, wc)) { ok = false; break; }
-              tc_fence_after();
-            }
-            issue_qk<D>(tS[t], qd[t], kd0 + uint32_t(s1) * kStageStep);
+          issue_pv<D>(tO[t], tS[t], vd0 + uint32_t(vs) * kStageStep, j > 0);
+          if (more) {
+            issue_qk<D>(tS[t], qd[t], kd0 + uint32_t(ks1) * kStageStep);
             tc_commit(&sm.bar_s_full[t]);
           }
         }
         if (!ok) break;
-        tc_commit(&sm.bar_kv_empty[s]);
+        tc_commit(&sm.bar_v_empty[vs]);
+        if (more) tc_commit(&sm.bar_k_empty[ks1]);
       }
       for (int t = 0; t < 2; ++t) tc_commit(&sm.bar_o_final[t]);
       // MMAs already issued must finish before TMEM can be released.
@@ -324,6 +341,7 @@ cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const 
     return cudaErrorInvalidConfiguration;  // the setmaxnreg split assumes kLaunchRegs
   prof_begin(kAttnFwd, st);
   if (D == 128) {
+    static_assert(sizeof(FwdSmem<128>) + 1024 <= 232448, "shared memory budget");
     const size_t smem = sizeof(FwdSmem<128>) + 1024;
     cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     attn_fwd_kernel<128><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, p);
