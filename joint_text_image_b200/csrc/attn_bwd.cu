@@ -27,7 +27,8 @@
 // P^T and dS^T become visible to the MMA thread together (one barrier per
 // tile).  TMEM: S^T[2] at 0/64, dP^T[2] at 128/192 (P^T, dS^T written over them as
 // packed bf16), dV at 256, dK at 256 + D; dQ^T of buffer i is written over
-// S^T[i] after the dV MMA that read P^T from there (MMAs run in issue order).
+// dP^T[i] after the dK MMA that read dS^T from there (MMAs run in issue
+// order), so the next S^T never waits for the dQ writers.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -209,12 +210,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // writers, (2) this tile's dS^T (hence also P^T) is ready.
         if (i + 1 < n_it) {
           const int i1 = i + 1, b1 = i1 & 1, s1 = i1 % kStages;
-          ok = mbar_wait(&sm.bar_full[s1], (i1 / kStages) & 1, wc);
-          if (ok && i1 >= 2) ok = mbar_wait(&sm.bar_dq_empty[b1], ((i1 >> 1) - 1) & 1, wc);
-          if (!ok) break;
-          if (i1 >= 2) tc_fence_after();  // TMEM reuse after the dQ writers' loads
+          // S^T(i+1) reuses the buffer whose P^T(i-1) the dV MMA already read;
+          // dP^T(i+1) reuses the buffer the dQ writers read dQ^T(i-1) from.
+          if (!mbar_wait(&sm.bar_full[s1], (i1 / kStages) & 1, wc)) { ok = false; break; }
           issue_kq<D>(tS[b1], k_km, q_km + uint32_t(s1) * kQStep);
           tc_commit(&sm.bar_s_full[b1]);
+          if (i1 >= 2) {
+            if (!mbar_wait(&sm.bar_dq_empty[b1], ((i1 >> 1) - 1) & 1, wc)) { ok = false; break; }
+            tc_fence_after();  // TMEM reuse after the dQ writers' loads
+          }
           issue_kq<D>(tdP[b1], v_km, o_km + uint32_t(s1) * kQStep);
           tc_commit(&sm.bar_dp_full[b1]);
         }
@@ -222,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_acc<D>(tdV, tS[bf], o_mn + uint32_t(s) * kQStep, i > 0);
         issue_acc<D>(tdK, tdP[bf], q_mn + uint32_t(s) * kQStep, i > 0);
-        issue_dq(tS[bf], k_mn, ds_mn + uint32_t(bf) * kDsStep);
+        issue_dq(tdP[bf], k_mn, ds_mn + uint32_t(bf) * kDsStep);  // over dS^T, after the dK MMA read it
         tc_commit(&sm.bar_dq_full[bf]);
         tc_commit(&sm.bar_empty[s]);
       }
@@ -386,8 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t a[64];
       if (live) {
-        tmem_ld32(tS[bf] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-        tmem_ld32(tS[bf] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+        tmem_ld32(tdP[bf] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+        tmem_ld32(tdP[bf] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
         tmem_ld_wait();
       }
       tc_fence_before();
