@@ -31,7 +31,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "joint-attn fwd+bwd masked TFLOPS & % bf16 peak, 1024px (4096 img tok)"
 WORKLOAD = "1024px"
-PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_bwd_1024px.md")
+# committed ncu summaries holding dram traffic per launch at the 1024px workload
+PROFILE_FILES = {k: os.path.join(ROOT, "profiles", f"{k}_1024px.md") for k in ("attn_fwd", "attn_bwd")}
+# the files a kernel's machine code depends on (its translation unit and headers)
+KERNEL_SOURCES = {k: [f"{k}.cu", "sm100.cuh", "kernels.h", "internal.h"] for k in ("attn_fwd", "attn_bwd")}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -44,6 +47,9 @@ def peaks():
 
 
 def workload_desc(wl):
+    if wl.name != "1024px":
+        return (f"{wl.name} fwd+bwd: samples (prefix, h, w, suffix) {wl.samples}, S={wl.S}; Hq={wl.Hq}, "
+                f"Hkv={wl.Hkv}, D={wl.D}, bf16 N(0,1) q/k/v/dout")
     pre = [s[0] for s in wl.samples]
     return (f"1024px fwd+bwd: B={wl.B}, prefix U[512,1536] drawn {pre} (seed 0), image 64x64=4096 tokens, "
             f"suffix 2, right-padded to S={wl.S}; Hq={wl.Hq}, Hkv={wl.Hkv}, D={wl.D}, scale 1/sqrt(D), "
@@ -84,19 +90,27 @@ SAMPLE_DESC = ("batch row 0, kv head 0 (its {g} query heads), query rows 0, {str
                "fp64 oracle forward + backward restricted to those rows")
 
 
-def cached_traffic(kernel_src):
+def kernel_source_sha256(kernel):
+    """sha256 over the sources the kernel is compiled from, in a fixed order."""
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "joint_text_image_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def cached_traffic(kernel):
     """dram bytes per launch from the committed ncu summary, or None if missing
-    or if the kernel source changed since the counters were taken."""
+    or if the kernel's sources changed since the counters were taken."""
     try:
-        txt = open(PROFILE_FILE).read()
-    except OSError:
+        txt = open(PROFILE_FILES[kernel]).read()
+    except (OSError, KeyError):
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", txt)
     if not m or not h:
         return None
-    cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
-    return float(m.group(1)) if h.group(1) == cur else None
+    return float(m.group(1)) if h.group(1) == kernel_source_sha256(kernel) else None
 
 
 class ClockSampler:
@@ -180,7 +194,14 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--ref-row-stride", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=["tiny", "256px", "1024px", "mixed", "1024px_bwd"],
+                    help="synthetic workload (the metric is quoted on 1024px; the others are for profiling)")
+    ap.add_argument("--source-hash", choices=sorted(KERNEL_SOURCES),
+                    help="print the kernel_source_sha256 an ncu summary of this kernel records, and exit")
     args = ap.parse_args()
+    if args.source_hash:
+        print(kernel_source_sha256(args.source_hash))
+        return
     args.warmup = max(args.warmup, 3)
 
     rank = int(os.environ.get("RANK", "0"))
@@ -206,7 +227,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    wl = synth.workload(WORKLOAD, seed=args.seed)
+    wl = synth.workload(args.workload, seed=args.seed)
     q, k, v, do = synth.tensors(wl, args.seed + rank, grad=True)
     seg = jt.hia_segments_build(wl.samples, wl.S)
     info = seg.info()
@@ -272,9 +293,8 @@ def main():
     dom = max(("attn_fwd", "attn_bwd"), key=lambda n: kt.get(n, {"avg_ms": 0})["avg_ms"] * kt.get(n, {"launches": 0})["launches"])
     dom_flops = bwd_flops if dom == "attn_bwd" else fwd_flops
     achieved = dom_flops / (kt[dom]["avg_ms"] * 1e-3) / 1e12
-    src = os.path.join(ROOT, "joint_text_image_b200", "csrc", "attn_bwd.cu" if dom == "attn_bwd" else "attn_fwd.cu")
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
-                "frac": achieved / peak_sus, "traffic": cached_traffic(src) if dom == "attn_bwd" else None,
+                "frac": achieved / peak_sus, "traffic": cached_traffic(dom),
                 "peak_kind": f"bf16_tflops_sustained ({pk_kind}): the kernel runs inside a seconds-long loop",
                 "frac_of_burst_peak": achieved / peak_burst,
                 "algorithmic_flops_per_launch": dom_flops}

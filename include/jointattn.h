@@ -219,6 +219,14 @@ int hia_get_device_status(void* stream);
  * kernel returns normally.  timeout_ns in [1, 10^9]. */
 int hia_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 
+/* Test hook for the softmax's FMA-pipe exponential: y[i] = 2^x[i] for n
+ * fp32 device values, computed as the forward kernel computes part of its
+ * exponentials (Cody-Waite range reduction, cubic for 2^f on [0, 1);
+ * relative error <= 1e-4 for x in [-125, 64]; x < -125, -inf included,
+ * gives about 2^-125). Returns HIA_ERR_INVALID_ARG for n < 0 or null
+ * pointers with n > 0; launch errors as HIA_ERR_CUDA. */
+int hia_debug_exp2(const float* x, float* y, int n, void* stream);
+
 const char* hia_status_string(int status);
 
 /* Per-kernel device timing, for benchmarks.  Between hia_profile_begin() and

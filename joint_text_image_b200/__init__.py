@@ -26,7 +26,7 @@ EXPORTED_SYMBOLS = (
     "hia_segments_row_bound", "hia_segments_mask", "hia_segments_tile_classes", "hia_rope2d_tables",
     "hia_attn_fwd_workspace_bytes", "hia_attn_fwd", "hia_attn_bwd_workspace_bytes", "hia_attn_bwd",
     "hia_get_device_status", "hia_debug_wait_timeout", "hia_status_string", "hia_profile_begin",
-    "hia_profile_end", "hia_attn_fwd_noalloc",
+    "hia_profile_end", "hia_attn_fwd_noalloc", "hia_debug_exp2",
 )
 
 
@@ -88,6 +88,7 @@ def lib():
         L.hia_get_device_status.argtypes = [P]
         L.hia_debug_wait_timeout.argtypes = [ctypes.c_uint64, P]
         L.hia_attn_fwd_noalloc.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, T, P, P]
+        L.hia_debug_exp2.argtypes = [P, P, I, P]
         L.hia_profile_begin.argtypes = []
         L.hia_profile_end.argtypes = [ctypes.POINTER(_KernelTime), I, ctypes.POINTER(I)]
         L.hia_status_string.argtypes = [I]

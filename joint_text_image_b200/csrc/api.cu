@@ -313,6 +313,11 @@ extern "C" int hia_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
   return cuda_status(hia::launch_wait_probe(sp, timeout_ns, static_cast<cudaStream_t>(stream)));
 }
 
+extern "C" int hia_debug_exp2(const float* x, float* y, int n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return HIA_ERR_INVALID_ARG;
+  return cuda_status(hia::launch_exp2_probe(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
 extern "C" int hia_attn_bwd(const hia_segments* g, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
                             hia_tensor v, const float* c, const float* s, float scale, hia_tensor o,
                             const float* lse, hia_tensor dout, hia_tensor dq, hia_tensor dk, hia_tensor dv,

@@ -19,13 +19,14 @@
 //                                       shared memory)
 // and dQ^T goes TMEM -> registers -> shared memory -> one bulk fp32
 // reduce-add into the dq accumulator (the reduction runs in L2).
-// Warps (512 threads): 0 TMA producer, 1 TMEM owner + MMA issuer, 4-7 and
+// Warps (512 threads): 0 TMA producer, 1 TMEM owner + S^T/dP^T MMA issuer,
+// 2 dV/dK/dQ^T MMA issuer, 4-7 and
 // 8-11 two softmax warpgroups that take alternate query tiles (one key row
 // per thread; then the dK and dV epilogues), 12-15 dQ writers (one head-dim
 // lane per thread).  setmaxnreg moves registers from the producer/MMA and dQ
 // warpgroups to the softmax warpgroups: 128*80 + 256*168 + 128*96 = 65536 = 512*128.
-// P^T and dS^T become visible to the MMA thread together (one barrier per
-// tile).  TMEM: S^T[2] at 0/64, dP^T[2] at 128/192 (P^T, dS^T written over them as
+// P^T and dS^T become visible to the second MMA thread together (one barrier
+// per tile).  TMEM: S^T[2] at 0/64, dP^T[2] at 128/192 (P^T, dS^T written over them as
 // packed bf16), dV at 256, dK at 256 + D; dQ^T of buffer i is written over
 // dP^T[i] after the dK MMA that read dS^T from there (MMAs run in issue
 // order), so the next S^T never waits for the dQ writers.
@@ -62,6 +63,7 @@ struct BwdSmem {
   uint64_t bar_ds_ready[2];
   uint64_t bar_dq_full[2];
   uint64_t bar_dq_empty[2];
+  uint64_t bar_s_free[2];
   uint64_t bar_final;
   uint32_t tmem_base;
   int abort_flag;
@@ -92,10 +94,6 @@ __device__ __forceinline__ void issue_dq(uint32_t d, uint64_t kt_mn_desc, uint64
   constexpr uint32_t idesc = idesc_bf16_f32(128, BQ, 1, 1);
   constexpr MNMajorSteps<BK / 16> st;
   mma_chain_ss<BK / 16>(d, kt_mn_desc, st.v, ds_desc, st.v, idesc, 0u);
-}
-
-__device__ __forceinline__ void red_add_f32(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 
 template <int D>
@@ -130,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.bar_ds_ready[i], 128);
       mbar_init(&sm.bar_dq_full[i], 1);
       mbar_init(&sm.bar_dq_empty[i], 128);
+      mbar_init(&sm.bar_s_free[i], 1);
     }
     mbar_init(&sm.bar_final, 1);
     sm.abort_flag = 0;
@@ -181,57 +180,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
         mbar_wait_hw(&sm.bar_full[i % kStages], (i / kStages) & 1, wc);
     }
-  } else if (warp == 1) {
-    // =============================== MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // =============================== MMA issuers
+    // Two threads issue MMAs: a wait or fence in an issuing thread lets its
+    // own short MMA queue drain, and the other thread's MMAs keep the tensor
+    // core busy meanwhile.  Warp 1 issues S^T and dP^T (running up to two
+    // query tiles ahead), warp 2 the dV, dK and dQ^T MMAs of each tile.
     if (lane == 0 && n_it > 0) {
-      // descriptor bases; the stages of q / dout and the two dS buffers are adjacent
-      const uint64_t k_km = sdesc_sw128(smem_u32(sm.k), 16, 1024);
-      const uint64_t k_mn = sdesc_sw128(smem_u32(sm.k), D == 128 ? 16384u : smem_u32(sm.v) - smem_u32(sm.k), 1024);
-      const uint64_t v_km = sdesc_sw128(smem_u32(sm.v), 16, 1024);
-      const uint64_t q_km = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
-      const uint64_t q_mn = sdesc_sw128(smem_u32(sm.q[0]), 8192, 1024);
-      const uint64_t o_km = sdesc_sw128(smem_u32(sm.dout[0]), 16, 1024);
-      const uint64_t o_mn = sdesc_sw128(smem_u32(sm.dout[0]), 8192, 1024);
-      const uint64_t ds_mn = sdesc_sw128(smem_u32(sm.ds[0]), 8192, 1024);
       constexpr uint32_t kQStep = (BQ * D * 2u) >> 4, kDsStep = (BK * BQ * 2u) >> 4;
-      bool ok = mbar_wait(&sm.bar_kv, 0, wc) && mbar_wait(&sm.bar_full[0], 0, wc);
-      if (ok) {
-        tc_fence_after();
-        issue_kq<D>(tS[0], k_km, q_km);
-        tc_commit(&sm.bar_s_full[0]);
-        issue_kq<D>(tdP[0], v_km, o_km);
-        tc_commit(&sm.bar_dp_full[0]);
-      }
-      for (int i = 0; ok && i < n_it; ++i) {
-        const int bf = i & 1, s = i % kStages;
-        // Every wait/fence in this thread lets the short MMA queue drain, so the
-        // loop has two synchronisation points per query tile: (1) the next
-        // tile's operands are loaded and its TMEM buffer was read out by the dQ
-        // writers, (2) this tile's dS^T (hence also P^T) is ready.
-        if (i + 1 < n_it) {
-          const int i1 = i + 1, b1 = i1 & 1, s1 = i1 % kStages;
-          // S^T(i+1) reuses the buffer whose P^T(i-1) the dV MMA already read;
-          // dP^T(i+1) reuses the buffer the dQ writers read dQ^T(i-1) from.
-          if (!mbar_wait(&sm.bar_full[s1], (i1 / kStages) & 1, wc)) { ok = false; break; }
-          issue_kq<D>(tS[b1], k_km, q_km + uint32_t(s1) * kQStep);
-          tc_commit(&sm.bar_s_full[b1]);
-          if (i1 >= 2) {
-            if (!mbar_wait(&sm.bar_dq_empty[b1], ((i1 >> 1) - 1) & 1, wc)) { ok = false; break; }
+      bool ok = mbar_wait(&sm.bar_kv, 0, wc);
+      if (warp == 1) {
+        const uint64_t k_km = sdesc_sw128(smem_u32(sm.k), 16, 1024);
+        const uint64_t v_km = sdesc_sw128(smem_u32(sm.v), 16, 1024);
+        const uint64_t q_km = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
+        const uint64_t o_km = sdesc_sw128(smem_u32(sm.dout[0]), 16, 1024);
+        for (int i = 0; ok && i < n_it; ++i) {
+          const int b = i & 1, s = i % kStages;
+          // S^T(i) reuses the buffer whose P^T(i-2) the dV MMA read; dP^T(i)
+          // the buffer the dQ writers read dQ^T(i-2) from.
+          if (!mbar_wait(&sm.bar_full[s], (i / kStages) & 1, wc)) { ok = false; break; }
+          if (i >= 2 && !mbar_wait(&sm.bar_s_free[b], ((i >> 1) - 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          issue_kq<D>(tS[b], k_km, q_km + uint32_t(s) * kQStep);
+          tc_commit(&sm.bar_s_full[b]);
+          if (i >= 2) {
+            if (!mbar_wait(&sm.bar_dq_empty[b], ((i >> 1) - 1) & 1, wc)) { ok = false; break; }
             tc_fence_after();  // TMEM reuse after the dQ writers' loads
           }
-          issue_kq<D>(tdP[b1], v_km, o_km + uint32_t(s1) * kQStep);
-          tc_commit(&sm.bar_dp_full[b1]);
+          issue_kq<D>(tdP[b], v_km, o_km + uint32_t(s) * kQStep);
+          tc_commit(&sm.bar_dp_full[b]);
         }
-        if (!mbar_wait(&sm.bar_ds_ready[bf], (i >> 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        issue_acc<D>(tdV, tS[bf], o_mn + uint32_t(s) * kQStep, i > 0);
-        issue_acc<D>(tdK, tdP[bf], q_mn + uint32_t(s) * kQStep, i > 0);
-        issue_dq(tdP[bf], k_mn, ds_mn + uint32_t(bf) * kDsStep);  // over dS^T, after the dK MMA read it
-        tc_commit(&sm.bar_dq_full[bf]);
-        tc_commit(&sm.bar_empty[s]);
+      } else {
+        const uint64_t k_mn = sdesc_sw128(smem_u32(sm.k), D == 128 ? 16384u : smem_u32(sm.v) - smem_u32(sm.k), 1024);
+        const uint64_t q_mn = sdesc_sw128(smem_u32(sm.q[0]), 8192, 1024);
+        const uint64_t o_mn = sdesc_sw128(smem_u32(sm.dout[0]), 8192, 1024);
+        const uint64_t ds_mn = sdesc_sw128(smem_u32(sm.ds[0]), 8192, 1024);
+        for (int i = 0; ok && i < n_it; ++i) {
+          const int b = i & 1, s = i % kStages;
+          // P^T(i) and dS^T(i) are in TMEM and dS^T(i) in shared memory
+          if (!mbar_wait(&sm.bar_ds_ready[b], (i >> 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          issue_acc<D>(tdV, tS[b], o_mn + uint32_t(s) * kQStep, i > 0);
+          tc_commit(&sm.bar_s_free[b]);
+          issue_acc<D>(tdK, tdP[b], q_mn + uint32_t(s) * kQStep, i > 0);
+          tc_commit(&sm.bar_empty[s]);  // the stage's Q and dO are no longer read
+          issue_dq(tdP[b], k_mn, ds_mn + uint32_t(b) * kDsStep);  // over dS^T, after the dK MMA read it
+          tc_commit(&sm.bar_dq_full[b]);
+        }
+        tc_commit(&sm.bar_final);
+        mbar_wait_hw(&sm.bar_final, 0, wc);
       }
-      tc_commit(&sm.bar_final);
-      mbar_wait_hw(&sm.bar_final, 0, wc);
     }
    }
   } else if (warp < 12) {

@@ -38,6 +38,7 @@ constexpr int kThreads = 384;
 // 128*88 + 256*208 = 64512 = 384*168.  The launcher checks the compiled count first.
 constexpr int kLaunchRegs = 168;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
+constexpr int kFmaExpPairs = 4;           // of every 16 column pairs, this many use exp2_fma2
 
 constexpr int kKStages = 3;  // K(j+1) is awaited together with V(j), so K runs one stage deeper
 constexpr int kVStages = 2;
@@ -248,7 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 8; ++c) mp[c] = __uint_as_float(sr[c]);
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(sr[c]));
+      for (int c = 8; c < 128; c += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mp[k] = fmax3(mp[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
       const float xmax = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                                fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * cs;
       if (j == 0) {
@@ -271,15 +274,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       uint32_t pk[64];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      const float2 cs2 = make_float2(cs, cs), nm2 = make_float2(-m, -m);
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), cs, -m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), cs, -m));
-        ls[c & 3] += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), cs2, nm2);
+        // kFmaExpPairs of every 16 column pairs take exp2 on the FMA pipe, the rest on MUFU
+        const float2 pv = (c & 15) < kFmaExpPairs ? exp2_fma2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        ls[c & 1] = __fadd2_rn(ls[c & 1], pv);
+        pk[c] = pack_bf16x2(pv.x, pv.y);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_st_wait();

@@ -90,5 +90,6 @@ cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st);
 cudaError_t launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const BwdParams& p, int n_blocks, int D, cudaStream_t st);
 cudaError_t launch_wait_probe(int* status, uint64_t timeout_ns, cudaStream_t st);
+cudaError_t launch_exp2_probe(const float* x, float* y, int n, cudaStream_t st);
 
 }  // namespace hia

@@ -293,6 +293,39 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x for a pair of values on the FMA/ALU pipes (packed f32x2 arithmetic),
+// for x <= 64: Cody-Waite split x = j + f with j = floor(x), f in [0, 1); 2^f
+// from a cubic whose coefficients were fitted here to minimise the relative
+// error on [0, 1) (max relative error 7.5e-5, well inside the bf16 rounding of
+// P); 2^j is added to the exponent field.  Inputs are clamped at -125 (the
+// cubic dips just below 1 at f = 0, so the exponent field must stay >= 2):
+// x <= -125, -inf included, gives about 2^-125 = 2.4e-38 instead of 0, which
+// is below anything a softmax row with a visible key can resolve.  Used for
+// part of the softmax exponentials so that the MUFU unit (ex2.approx) is not
+// the only source of exp2.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23: floor(x) lands in the low mantissa bits
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rd(x, make_float2(kShift, kShift));
+  const float2 j = __fadd2_rn(t, make_float2(-kShift, -kShift));  // floor(x), exact
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);     // x - floor(x), exact
+  float2 p = __ffma2_rn(make_float2(0x1.3f95cap-4f, 0x1.3f95cap-4f), f, make_float2(0x1.cefc18p-3f, 0x1.cefc18p-3f));
+  p = __ffma2_rn(p, f, make_float2(0x1.64446cp-1f, 0x1.64446cp-1f));
+  p = __ffma2_rn(p, f, make_float2(0x1.fff62cp-1f, 0x1.fff62cp-1f));
+  // t's low mantissa bits hold floor(x) + 2^22; shifted left by 23 only the
+  // low 9 bits of floor(x) survive: floor(x) << 23 modulo 2^32, the exponent step.
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// max of three (a NaN operand is ignored, as in fmaxf)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

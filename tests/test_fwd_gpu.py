@@ -112,3 +112,24 @@ def test_bounded_wait_expires_and_reports():
     # the context is still usable
     wl = synth.workload("tiny")
     run_fwd(wl)
+
+
+def test_fma_exp2_matches_exp2():
+    """The FMA-pipe exponential used for part of the softmax: relative error
+    <= 1e-4 against 2^x over the range the softmax feeds it (x <= 8 after the
+    lazy rescale), and at most 2^-125 (about 2.4e-38) for x <= -125, -inf
+    included."""
+    x = torch.cat([torch.linspace(-125.0, 8.0, 200001),
+                   torch.tensor([-125.5, -126.0, -127.0, -200.0, -float("inf"), -0.0, 1e-8, -1e-8, 7.9999995])])
+    xd = x.cuda()
+    y = torch.empty_like(xd)
+    assert jt.lib().hia_debug_exp2(xd.data_ptr(), y.data_ptr(), x.numel(), jt._stream()) == 0
+    torch.cuda.synchronize()
+    ref = torch.exp2(x.double())
+    got = y.cpu().double()
+    assert torch.isfinite(got).all()
+    fin = x >= -125.0
+    rel = ((got[fin] - ref[fin]) / ref[fin]).abs()
+    assert rel.max() <= 1e-4, rel.max()
+    low = got[~fin]
+    assert ((low >= 0) & (low <= 2.0 ** -125 * 1.0001)).all(), low
