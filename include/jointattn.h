@@ -208,6 +208,37 @@ int hia_attn_bwd(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, 
                  hia_tensor dk, hia_tensor dv, void* workspace, size_t workspace_bytes,
                  void* stream);
 
+/* ---- One training step from HOST buffers.  (No counterpart on the pages:
+ * a convenience of the library for callers that hold their tensors in host
+ * memory.)  A hia_step owns, on the device current at creation, the device
+ * copies of one step's tensors in the plain contiguous layout (q, dout, o,
+ * dq: [B,S,Hq,D] bf16; k, v, dk, dv: [B,S,Hkv,D] bf16; lse: [B,Hq,S] fp32),
+ * the RoPE tables of `seg` (computed once, at creation, with `rope_base`) and
+ * both workspaces.  `seg` must stay alive and uploaded while the step exists.
+ * Returns HIA_ERR_INVALID_ARG for null pointers, non-positive head counts
+ * or rope_base, HIA_ERR_UNSUPPORTED unless D is 64 or 128 and Hq a multiple
+ * of Hkv, HIA_ERR_NOT_ON_DEVICE if `seg` was not uploaded, HIA_ERR_CUDA if
+ * an allocation fails (nothing is left allocated). */
+typedef struct hia_step hia_step;
+int hia_step_create(const hia_segments* seg, int Hq, int Hkv, int D, double rope_base, hia_step** out);
+/* Waits for the step's own copy stream, then frees everything it owns. */
+void hia_step_destroy(hia_step* st);
+
+/* Enqueue one forward + backward on `stream` from host buffers (all
+ * pointers below are HOST pointers, in the layouts above): copies q, k, v,
+ * dout to the device, runs hia_attn_fwd and hia_attn_bwd, copies o, lse, dq,
+ * dk, dv back.  dout is uploaded, and o and lse downloaded, on the step's own
+ * copy stream so that they overlap the kernels; `stream` waits for that
+ * stream at the end, so once `stream` reaches this point every output is in
+ * host memory.  Asynchronous: host buffers must stay valid until then.
+ * Pinned (page-locked) host memory makes the copies asynchronous; pageable
+ * memory works but the copies then block the calling thread.  Two steps
+ * enqueued on two streams overlap one step's copies with the other's
+ * kernels.  Errors: HIA_ERR_INVALID_ARG (null pointer), the errors of
+ * hia_attn_fwd / hia_attn_bwd, HIA_ERR_CUDA. */
+int hia_attn_step_host(hia_step* st, const void* q, const void* k, const void* v, const void* dout,
+                       float scale, void* o, float* lse, void* dq, void* dk, void* dv, void* stream);
+
 /* Read and clear the device status word of the current device (synchronizes
  * `stream`).  Returns HIA_OK, HIA_ERR_DEVICE_TIMEOUT if any kernel's bounded
  * wait expired since the last call, or HIA_ERR_CUDA. */

@@ -16,7 +16,7 @@ __all__ = [
     "HiaError", "Segments", "lib", "hia_segments_build", "hia_rope2d_tables", "hia_attn_fwd",
     "hia_attn_bwd", "hia_attn_fwd_workspace_bytes", "hia_attn_bwd_workspace_bytes",
     "hia_get_device_status", "hia_debug_wait_timeout", "hia_profile_begin", "hia_profile_end",
-    "LIB_PATH", "EXPORTED_SYMBOLS",
+    "Step", "hia_step_create", "hia_attn_step_host", "LIB_PATH", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libjointattn.so")
@@ -26,7 +26,8 @@ EXPORTED_SYMBOLS = (
     "hia_segments_row_bound", "hia_segments_mask", "hia_segments_tile_classes", "hia_rope2d_tables",
     "hia_attn_fwd_workspace_bytes", "hia_attn_fwd", "hia_attn_bwd_workspace_bytes", "hia_attn_bwd",
     "hia_get_device_status", "hia_debug_wait_timeout", "hia_status_string", "hia_profile_begin",
-    "hia_profile_end", "hia_attn_fwd_noalloc", "hia_debug_exp2",
+    "hia_profile_end", "hia_attn_fwd_noalloc", "hia_debug_exp2", "hia_step_create", "hia_step_destroy",
+    "hia_attn_step_host",
 )
 
 
@@ -89,6 +90,10 @@ def lib():
         L.hia_debug_wait_timeout.argtypes = [ctypes.c_uint64, P]
         L.hia_attn_fwd_noalloc.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, T, P, P]
         L.hia_debug_exp2.argtypes = [P, P, I, P]
+        L.hia_step_create.argtypes = [P, I, I, I, ctypes.c_double, ctypes.POINTER(P)]
+        L.hia_step_destroy.argtypes = [P]
+        L.hia_step_destroy.restype = None
+        L.hia_attn_step_host.argtypes = [P, P, P, P, P, ctypes.c_float, P, P, P, P, P, P]
         L.hia_profile_begin.argtypes = []
         L.hia_profile_end.argtypes = [ctypes.POINTER(_KernelTime), I, ctypes.POINTER(I)]
         L.hia_status_string.argtypes = [I]
@@ -259,6 +264,50 @@ def hia_attn_bwd(seg: Segments, q, k, v, cos, sin, o, lse, dout, scale=None, dq=
                               _t(dout, True, g), _t(dq, True, g), _t(dk, False, 1), _t(dv, False, 1),
                               ws.data_ptr(), nb, _stream()), "hia_attn_bwd")
     return dq, dk, dv
+
+
+class Step:
+    """Owner of a library hia_step: device buffers, RoPE tables and workspaces
+    for training steps fed from host memory (hia_attn_step_host)."""
+
+    def __init__(self, seg: "Segments", Hq, Hkv, D, base=10000.0):
+        self.seg, self.Hq, self.Hkv, self.D = seg, Hq, Hkv, D
+        h = ctypes.c_void_p()
+        _check(lib().hia_step_create(seg.handle, int(Hq), int(Hkv), int(D), float(base), ctypes.byref(h)),
+               "hia_step_create")
+        self.handle = h
+
+    def __del__(self):
+        if getattr(self, "handle", None) and _lib is not None:
+            _lib.hia_step_destroy(self.handle)
+            self.handle = None
+
+
+def hia_step_create(seg: "Segments", Hq, Hkv, D, base=10000.0) -> Step:
+    return Step(seg, Hq, Hkv, D, base)
+
+
+def hia_attn_step_host(step: Step, q, k, v, dout, o, lse, dq, dk, dv, scale=None, stream=None):
+    """One forward + backward from host tensors (contiguous CPU tensors; pin
+    them for asynchronous copies): q, dout [B,S,Hq,D], k, v [B,S,Hkv,D] bf16
+    in; o, dq [B,S,Hq,D], dk, dv [B,S,Hkv,D] bf16 and lse [B,Hq,S] fp32 out.
+    Enqueued on `stream` (default: the current CUDA stream)."""
+    import torch
+    B, S, Hq, Hkv, D = step.seg.B, step.seg.S, step.Hq, step.Hkv, step.D
+    want = ((q, (B, S, Hq, D), torch.bfloat16), (k, (B, S, Hkv, D), torch.bfloat16),
+            (v, (B, S, Hkv, D), torch.bfloat16), (dout, (B, S, Hq, D), torch.bfloat16),
+            (o, (B, S, Hq, D), torch.bfloat16), (lse, (B, Hq, S), torch.float32),
+            (dq, (B, S, Hq, D), torch.bfloat16), (dk, (B, S, Hkv, D), torch.bfloat16),
+            (dv, (B, S, Hkv, D), torch.bfloat16))
+    for t, shape, dt in want:
+        if t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape or t.dtype != dt:
+            raise ValueError(f"hia_attn_step_host takes contiguous host tensors {shape} {dt}")
+    if scale is None:
+        scale = step.D ** -0.5
+    st = _stream() if stream is None else ctypes.c_void_p(stream.cuda_stream)
+    _check(lib().hia_attn_step_host(step.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
+                                    float(scale), o.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                    dv.data_ptr(), st), "hia_attn_step_host")
 
 
 def hia_get_device_status():

@@ -11,7 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libjointattn.so")
 BUILD = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "rope.cu", "attn_fwd.cu", "attn_bwd.cu", "probe.cu", "segments.cpp", "profile.cpp", "fwd_noalloc.cu"]
+SOURCES = ["api.cu", "rope.cu", "attn_fwd.cu", "attn_bwd.cu", "probe.cu", "segments.cpp", "profile.cpp", "fwd_noalloc.cu", "host_step.cpp"]
 HEADERS = ["sm100.cuh", "internal.h", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
