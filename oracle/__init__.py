@@ -44,8 +44,9 @@ def _load():
         lib.oracle_positions.argtypes = [I, I, P, P, P, P, P, P]
         lib.oracle_rope_tables.argtypes = [I, I, I, P, P, P, P, D, P, P]
         lib.oracle_rope_apply.argtypes = [I, I, I, I, P, P, P, P, D, I, P, P]
-        lib.oracle_attn_fwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, D, D, I, P, I, P, P, P, I]
-        lib.oracle_attn_bwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, D, D, I, P, I, P, P, P, P, I]
+        lib.oracle_attn_fwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, D, D, I, P, I, P, P, P, D, P, P, I]
+        lib.oracle_attn_bwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, D, D, I, P, I, P, P, P, D,
+                                        P, P, P, P, P, I]
         _lib = lib
     return _lib
 
@@ -102,12 +103,24 @@ def rope_apply(samples, x: np.ndarray, base: float = 10000.0, inverse: bool = Fa
     return y
 
 
+def _norm_args(qk_norm, D):
+    """qk_norm = (wq [D], wk [D], eps) or None -> (wq, wk, eps) for the C call."""
+    if qk_norm is None:
+        return None, None, 0.0
+    wq, wk, eps = qk_norm
+    wq = np.ascontiguousarray(wq, dtype=np.float64).reshape(D)
+    wk = np.ascontiguousarray(wk, dtype=np.float64).reshape(D)
+    return wq, wk, float(eps)
+
+
 def attn_fwd(samples, q, k, v, scale=None, base=10000.0, rotate=True, rows=None,
-             groups=None, nthreads=0):
+             groups=None, nthreads=0, qk_norm=None):
     """Forward: returns (o [B,S,Hq,D], lse [B,Hq,S], threads_used).
 
     q [B,S,Hq,D], k/v [B,S,Hkv,D] as fp64 (exact copies of the bf16 inputs).
-    rows: optional int list of query rows; groups: optional bool [B, Hkv]."""
+    rows: optional int list of query rows; groups: optional bool [B, Hkv].
+    qk_norm: optional (wq [D], wk [D], eps): per-head RMSNorm of the rotated
+    q and k rows (oracle.c, rms_norm)."""
     g = _geom(samples)
     q = np.ascontiguousarray(q, dtype=np.float64)
     k = np.ascontiguousarray(k, dtype=np.float64)
@@ -118,12 +131,13 @@ def attn_fwd(samples, q, k, v, scale=None, base=10000.0, rotate=True, rows=None,
         scale = 1.0 / np.sqrt(D)
     r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
     gs = None if groups is None else np.ascontiguousarray(groups, dtype=np.uint8).reshape(-1)
+    wq, wk, eps = _norm_args(qk_norm, D)
     o = np.zeros((B, S, Hq, D))
     lse = np.zeros((B, Hq, S))
     used = _load().oracle_attn_fwd(B, S, Hq, Hkv, D, *map(_p, g), _p(q), _p(k), _p(v),
                                    float(scale), float(base), int(rotate), _p(r),
-                                   0 if r is None else len(r), _p(gs), _p(o), _p(lse),
-                                   int(nthreads))
+                                   0 if r is None else len(r), _p(gs), _p(wq), _p(wk), eps,
+                                   _p(o), _p(lse), int(nthreads))
     if used < 0:
         raise ValueError("bad arguments")
     return o, lse, used
@@ -134,6 +148,19 @@ def attn_bwd(samples, q, k, v, dout, scale=None, base=10000.0, rotate=True, grou
     """Backward: returns (dq [B,S,Hq,D], dk, dv [B,S,Hkv,D], threads_used).
 
     rows: optional query-row subset (dq of those rows; dk, dv summed over them)."""
+    dq, dk, dv, _, _, used = _attn_bwd(samples, q, k, v, dout, scale, base, rotate, groups,
+                                       nthreads, rows, None)
+    return dq, dk, dv, used
+
+
+def attn_bwd_qknorm(samples, q, k, v, dout, qk_norm, scale=None, base=10000.0, rotate=True,
+                    groups=None, nthreads=0, rows=None):
+    """Backward with the per-head QK RMSNorm qk_norm = (wq, wk, eps): returns
+    (dq, dk, dv, dwq [D], dwk [D], threads_used) (oracle.c, rms_norm_vjp)."""
+    return _attn_bwd(samples, q, k, v, dout, scale, base, rotate, groups, nthreads, rows, qk_norm)
+
+
+def _attn_bwd(samples, q, k, v, dout, scale, base, rotate, groups, nthreads, rows, qk_norm):
     g = _geom(samples)
     q = np.ascontiguousarray(q, dtype=np.float64)
     k = np.ascontiguousarray(k, dtype=np.float64)
@@ -145,13 +172,16 @@ def attn_bwd(samples, q, k, v, dout, scale=None, base=10000.0, rotate=True, grou
         scale = 1.0 / np.sqrt(D)
     gs = None if groups is None else np.ascontiguousarray(groups, dtype=np.uint8).reshape(-1)
     r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    wq, wk, eps = _norm_args(qk_norm, D)
     dq = np.zeros((B, S, Hq, D))
     dk = np.zeros((B, S, Hkv, D))
     dv = np.zeros((B, S, Hkv, D))
+    dwq = np.zeros(D) if qk_norm is not None else None
+    dwk = np.zeros(D) if qk_norm is not None else None
     used = _load().oracle_attn_bwd(B, S, Hq, Hkv, D, *map(_p, g), _p(q), _p(k), _p(v), _p(dout),
                                    float(scale), float(base), int(rotate), _p(r),
-                                   0 if r is None else len(r), _p(gs), _p(dq),
-                                   _p(dk), _p(dv), int(nthreads))
+                                   0 if r is None else len(r), _p(gs), _p(wq), _p(wk), eps,
+                                   _p(dq), _p(dk), _p(dv), _p(dwq), _p(dwk), int(nthreads))
     if used < 0:
         raise ValueError("bad arguments")
-    return dq, dk, dv, used
+    return dq, dk, dv, dwq, dwk, used

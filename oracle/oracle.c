@@ -35,7 +35,13 @@
  *   - image token i (row r = i / w, column c = i % w) sits at x = I0 + c,
  *     y = I0 + r; even j use x, odd j use y; every other token (text, suffix,
  *     padding) sits at x = y = n, its sequence index;
- *   - scores are scale * <R q, R k>, with scale passed in (1/sqrt(D)).
+ *   - scores are scale * <R q, R k>, with scale passed in (1/sqrt(D));
+ *   - optional per-head QK RMSNorm (HunyuanImage3Attention: RoPE is applied
+ *     before the per-head QK RMSNorm; HunyuanRMSNorm normalizes over the
+ *     last axis with eps, default 1e-5, and multiplies by its weight): with
+ *     weights wq, wk the scores use y = w * x / sqrt(mean(x^2) + eps) of the
+ *     rotated rows x = R q, R k.  In fp64 here; the dtype casts of the
+ *     reference layer are rounding, covered by the parity tolerances.
  *
  * Parity pins: every function here is pinned by the CPU tests (hand-written
  * masks, closed-form pair counts, the 1D-RoPE library routine, relative
@@ -207,8 +213,11 @@ typedef struct {
     const int32_t* rows;        /* query rows to compute, or NULL for all */
     int n_rows;
     const uint8_t* group_sel;   /* [B * Hkv] 1 = compute this (b, kv head) group; NULL = all */
+    const double *wq, *wk;      /* QK RMSNorm weights [D] each, or NULL: no norm */
+    double eps;
     double *o, *lse;            /* fwd outputs */
     double *dq, *dk_h, *dv_h;   /* bwd outputs; dk_h, dv_h per q head [B,S,Hq,D] */
+    double *dwq_h, *dwk_h;      /* bwd, with the norm: weight gradients per (b, q head) [B*Hq][D] */
     int n_tasks;
     int next_task;
     pthread_mutex_t lock;
@@ -218,6 +227,27 @@ static double dot(const double* a, const double* b, int D) {
     double s = 0.0;
     for (int d = 0; d < D; ++d) s += a[d] * b[d];
     return s;
+}
+
+/* HunyuanRMSNorm of one head vector: y = w * x / sqrt(mean(x^2) + eps).
+ * Returns r = 1 / sqrt(mean(x^2) + eps). */
+static double rms_norm(const double* x, const double* w, int D, double eps, double* y) {
+    double ss = 0.0;
+    for (int d = 0; d < D; ++d) ss += x[d] * x[d];
+    double r = 1.0 / sqrt(ss / D + eps);
+    for (int d = 0; d < D; ++d) y[d] = w[d] * x[d] * r;
+    return r;
+}
+
+/* Vector-Jacobian product of rms_norm at x (r from rms_norm): with
+ * xh = r x and a = w * gy, gx = r (a - xh <a, xh> / D); gw += gy * xh. */
+static void rms_norm_vjp(const double* x, const double* w, int D, double r, const double* gy,
+                         double* gx, double* gw) {
+    double ax = 0.0;
+    for (int d = 0; d < D; ++d) ax += w[d] * gy[d] * x[d] * r;
+    for (int d = 0; d < D; ++d) gx[d] = r * (w[d] * gy[d] - x[d] * r * ax / D);
+    if (gw)
+        for (int d = 0; d < D; ++d) gw[d] += gy[d] * x[d] * r;
 }
 
 /* Rotated copy of head h of tensor x [B,S,H,D] for sample b: out [S, D]. */
@@ -242,6 +272,11 @@ static void fwd_task(job_t* J, int b, int h) {
     gather_head(J, J->q, J->Hq, b, h, J->rotate_inputs, qr);
     gather_head(J, J->k, J->Hkv, b, h / g, J->rotate_inputs, kr);
     gather_head(J, J->v, J->Hkv, b, h / g, 0, vv);
+    if (J->wq)
+        for (int64_t n = 0; n < S; ++n) {
+            rms_norm(qr + n * D, J->wq, D, J->eps, qr + n * D);
+            rms_norm(kr + n * D, J->wk, D, J->eps, kr + n * D);
+        }
     int nr = J->rows ? J->n_rows : S;
     for (int ri = 0; ri < nr; ++ri) {
         int64_t q = J->rows ? J->rows[ri] : ri;
@@ -271,7 +306,10 @@ static void fwd_task(job_t* J, int b, int h) {
  *   dP = dO V^T,  Dq = dO . O,  dS = P (dP - Dq),
  *   dQr = scale dS Kr,  dKr += scale dS^T Qr,  dV += P^T dO,
  * and returns dQ = R^T dQr; dk_h/dv_h hold this head's R^T dKr and dV
- * contributions (summed over the heads of a group by the caller). */
+ * contributions (summed over the heads of a group by the caller).  With the
+ * QK RMSNorm, Qr and Kr are the normalized rotated rows and the gradients
+ * pass through the norm's vector-Jacobian product before R^T; the weight
+ * gradients of this head go to dwq_h / dwk_h. */
 static void bwd_task(job_t* J, int b, int h) {
     const int S = J->S, D = J->D, g = J->Hq / J->Hkv;
     osample s = make_sample(J->prefix[b], J->img_h[b], J->img_w[b], J->suffix[b]);
@@ -287,6 +325,24 @@ static void bwd_task(job_t* J, int b, int h) {
     gather_head(J, J->q, J->Hq, b, h, J->rotate_inputs, qr);
     gather_head(J, J->k, J->Hkv, b, h / g, J->rotate_inputs, kr);
     gather_head(J, J->v, J->Hkv, b, h / g, 0, vv);
+    /* with the norm: keep the rotated rows (qx, kx) and normalize qr, kr */
+    double *qx = NULL, *kx = NULL, *rq = NULL, *rk = NULL, *gx = NULL;
+    double *dwq = NULL, *dwk = NULL;
+    if (J->wq) {
+        qx = malloc(sizeof(double) * SD);
+        kx = malloc(sizeof(double) * SD);
+        rq = malloc(sizeof(double) * (size_t)S);
+        rk = malloc(sizeof(double) * (size_t)S);
+        gx = malloc(sizeof(double) * D);
+        memcpy(qx, qr, sizeof(double) * SD);
+        memcpy(kx, kr, sizeof(double) * SD);
+        for (int64_t n = 0; n < S; ++n) {
+            rq[n] = rms_norm(qx + n * D, J->wq, D, J->eps, qr + n * D);
+            rk[n] = rms_norm(kx + n * D, J->wk, D, J->eps, kr + n * D);
+        }
+        dwq = J->dwq_h + ((size_t)b * J->Hq + h) * D;
+        dwk = J->dwk_h + ((size_t)b * J->Hq + h) * D;
+    }
     int nr = J->rows ? J->n_rows : S;
     for (int ri = 0; ri < nr; ++ri) {
         int64_t q = J->rows ? J->rows[ri] : ri;
@@ -320,17 +376,26 @@ static void bwd_task(job_t* J, int b, int h) {
                 dvv[k * D + d] += p * dorow[d];
             }
         }
+        if (J->wq) {
+            rms_norm_vjp(qx + q * D, J->wq, D, rq[q], dqr, gx, dwq);
+            memcpy(dqr, gx, sizeof(double) * D);
+        }
         if (J->rotate_inputs) rotate_t(&s, q, D, J->base, dqr, dqout);
         else memcpy(dqout, dqr, sizeof(double) * D);
     }
     for (int64_t k = 0; k < S; ++k) {
         double* dko = J->dk_h + (((int64_t)b * S + k) * J->Hq + h) * D;
         double* dvo = J->dv_h + (((int64_t)b * S + k) * J->Hq + h) * D;
+        if (J->wq) {
+            rms_norm_vjp(kx + k * D, J->wk, D, rk[k], dkr + k * D, gx, dwk);
+            memcpy(dkr + k * D, gx, sizeof(double) * D);
+        }
         if (J->rotate_inputs) rotate_t(&s, k, D, J->base, dkr + k * D, dko);
         else memcpy(dko, dkr + k * D, sizeof(double) * D);
         memcpy(dvo, dvv + k * D, sizeof(double) * D);
     }
     free(qr); free(kr); free(vv); free(dkr); free(dvv); free(dqr); free(orow); free(sc);
+    free(qx); free(kx); free(rq); free(rk); free(gx);
 }
 
 static int task_selected(const job_t* J, int t) {
@@ -384,14 +449,17 @@ static int check_geom(int B, int S, int Hq, int Hkv, int D, const int32_t* prefi
 
 /* Forward.  q [B,S,Hq,D], k, v [B,S,Hkv,D] (fp64, exact copies of the bf16
  * inputs); o [B,S,Hq,D]; lse [B,Hq,S].  rows/n_rows restrict the query rows;
- * group_sel [B*Hkv] restricts the (b, kv head) groups.  Returns the number of
+ * group_sel [B*Hkv] restricts the (b, kv head) groups; wq, wk [D] (both or
+ * neither) turn on the QK RMSNorm with epsilon eps.  Returns the number of
  * threads used, or -1 on bad arguments. */
 int oracle_attn_fwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
                     const int32_t* img_h, const int32_t* img_w, const int32_t* suffix,
                     const double* q, const double* k, const double* v, double scale,
                     double base, int rotate_inputs, const int32_t* rows, int n_rows,
-                    const uint8_t* group_sel, double* o, double* lse, int nthreads) {
+                    const uint8_t* group_sel, const double* wq, const double* wk, double eps,
+                    double* o, double* lse, int nthreads) {
     if (check_geom(B, S, Hq, Hkv, D, prefix, img_h, img_w, suffix)) return -1;
+    if ((wq == NULL) != (wk == NULL) || (wq && !(eps >= 0.0))) return -1;
     job_t J;
     memset(&J, 0, sizeof(J));
     J.B = B; J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.D = D;
@@ -399,19 +467,24 @@ int oracle_attn_fwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
     J.q = q; J.k = k; J.v = v; J.scale = scale; J.base = base;
     J.rotate_inputs = rotate_inputs; J.rows = rows; J.n_rows = n_rows;
     J.group_sel = group_sel; J.o = o; J.lse = lse;
+    J.wq = wq; J.wk = wk; J.eps = eps;
     return run_job(&J, 0, nthreads);
 }
 
 /* Backward.  dq [B,S,Hq,D]; dk, dv [B,S,Hkv,D].  group_sel as above (dq of
  * unselected groups and their dk/dv are left untouched).  rows/n_rows
  * restrict the query rows: dq is written for those rows only and dk, dv hold
- * the contributions of those rows only (a partial sum over queries). */
+ * the contributions of those rows only (a partial sum over queries).  With
+ * the QK RMSNorm (wq, wk non-NULL) dwq, dwk [D] receive the weight
+ * gradients, summed over the selected groups and rows. */
 int oracle_attn_bwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
                     const int32_t* img_h, const int32_t* img_w, const int32_t* suffix,
                     const double* q, const double* k, const double* v, const double* dout,
                     double scale, double base, int rotate_inputs, const int32_t* rows, int n_rows,
-                    const uint8_t* group_sel, double* dq, double* dk, double* dv, int nthreads) {
+                    const uint8_t* group_sel, const double* wq, const double* wk, double eps,
+                    double* dq, double* dk, double* dv, double* dwq, double* dwk, int nthreads) {
     if (check_geom(B, S, Hq, Hkv, D, prefix, img_h, img_w, suffix)) return -1;
+    if ((wq == NULL) != (wk == NULL) || (wq && (!(eps >= 0.0) || !dwq || !dwk))) return -1;
     size_t n = (size_t)B * S * Hq * D;
     job_t J;
     memset(&J, 0, sizeof(J));
@@ -422,7 +495,24 @@ int oracle_attn_bwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
     J.group_sel = group_sel; J.dq = dq;
     J.dk_h = calloc(n ? n : 1, sizeof(double));
     J.dv_h = calloc(n ? n : 1, sizeof(double));
+    J.wq = wq; J.wk = wk; J.eps = eps;
+    size_t nw = (size_t)B * Hq * D;
+    if (wq) {
+        J.dwq_h = calloc(nw ? nw : 1, sizeof(double));
+        J.dwk_h = calloc(nw ? nw : 1, sizeof(double));
+    }
     int used = run_job(&J, 1, nthreads);
+    if (wq) {
+        /* weight gradients: sum of the per-(b, head) partials, in a fixed order */
+        for (int d = 0; d < D; ++d) { dwq[d] = 0.0; dwk[d] = 0.0; }
+        for (size_t t = 0; t < (size_t)B * Hq; ++t)
+            for (int d = 0; d < D; ++d) {
+                dwq[d] += J.dwq_h[t * D + d];
+                dwk[d] += J.dwk_h[t * D + d];
+            }
+        free(J.dwq_h);
+        free(J.dwk_h);
+    }
     int g = Hq / Hkv;
     for (int b = 0; b < B; ++b)
         for (int hk = 0; hk < Hkv; ++hk) {
