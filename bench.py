@@ -196,6 +196,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD, choices=["tiny", "256px", "1024px", "mixed", "1024px_bwd"],
                     help="synthetic workload (the metric is quoted on 1024px; the others are for profiling)")
+    ap.add_argument("--qk-norm", action="store_true",
+                    help="enable the per-head QK RMSNorm after RoPE (weights seeded, eps 1e-5)")
     ap.add_argument("--source-hash", choices=sorted(KERNEL_SOURCES),
                     help="print the kernel_source_sha256 an ncu summary of this kernel records, and exit")
     args = ap.parse_args()
@@ -244,10 +246,17 @@ def main():
     wsf = torch.empty(jt.hia_attn_fwd_workspace_bytes(seg, wl.Hq, wl.Hkv, wl.D), dtype=torch.uint8, device=dev)
     wsb = torch.empty(jt.hia_attn_bwd_workspace_bytes(seg, wl.Hq, wl.Hkv, wl.D), dtype=torch.uint8, device=dev)
 
+    norm = None
+    if args.qk_norm:
+        # per-head QK RMSNorm after RoPE, seeded weights U[0.5, 1.5), eps 1e-5
+        gw = torch.Generator().manual_seed(args.seed + 7)
+        norm = tuple((torch.rand(wl.D, generator=gw) + 0.5).to(dev) for _ in range(2)) + (1e-5,)
+
     def step(qi, ki, vi, doi):
         c, s = jt.hia_rope2d_tables(seg, wl.D, wl.base, out=cs)
-        jt.hia_attn_fwd(seg, qi, ki, vi, c, s, wl.scale, o=o, lse=lse, workspace=wsf)
-        jt.hia_attn_bwd(seg, qi, ki, vi, c, s, o, lse, doi, wl.scale, dq=dq, dk=dk, dv=dv, workspace=wsb)
+        jt.hia_attn_fwd(seg, qi, ki, vi, c, s, wl.scale, o=o, lse=lse, workspace=wsf, qk_norm=norm)
+        jt.hia_attn_bwd(seg, qi, ki, vi, c, s, o, lse, doi, wl.scale, dq=dq, dk=dk, dv=dv, workspace=wsb,
+                        qk_norm=norm)
 
     for _ in range(args.warmup):
         step(qd, kd, vd, dod)
@@ -360,7 +369,8 @@ def main():
             "config": {"workload": workload_desc(wl), "global_batch": wl.B * world, "seq_len": wl.S,
                        "parallelism": f"replicas x{world} (no cross-GPU exchange in this op)",
                        "l2": f"inputs larger than L2: {(q.numel() + k.numel() + v.numel() + do.numel()) * 2 / 1e6:.0f} MB read per step",
-                       "visible_pairs": pairs, "fwd_flops": fwd_flops, "bwd_flops": bwd_flops},
+                       "visible_pairs": pairs, "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
+                       "qk_norm": ({"eps": 1e-5, "weights": "seeded U[0.5,1.5)"} if args.qk_norm else None)},
             "pct_of_bf16_peak": value / world / peak_burst * 100.0,
             "fwd_tflops": fwd_flops / (fwd_t * 1e-3) / 1e12 if fwd_t else None,
             "bwd_tflops": bwd_flops / (bwd_t * 1e-3) / 1e12 if bwd_t else None,

@@ -166,6 +166,28 @@ int hia_attn_fwd(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, 
                  hia_tensor o, float* lse, void* workspace, size_t workspace_bytes,
                  void* stream);
 
+/* Per-head QK RMSNorm applied after RoPE (HunyuanImage3Attention with
+ * use_qk_norm: RoPE is applied before the per-head QK RMSNorm; HunyuanRMSNorm
+ * normalizes over the last axis with eps and scales by its weight).  With a
+ * norm, the attention uses y = w * x / sqrt(mean(x^2) + eps) of every rotated
+ * q row (w = wq) and k row (w = wk), x = R q or R k, computed in fp32 and
+ * rounded once to bf16.  wq, wk: fp32 [D] device pointers, 16-byte aligned;
+ * eps >= 0 (the layer's default is 1e-5). */
+typedef struct {
+    const float* wq;
+    const float* wk;
+    float eps;
+} hia_qk_norm;
+
+/* hia_attn_fwd with an optional QK RMSNorm (norm == NULL: none, identical to
+ * hia_attn_fwd).  Same workspace.  Extra errors: HIA_ERR_INVALID_ARG for a
+ * null weight or a negative or non-finite eps, HIA_ERR_UNSUPPORTED for a
+ * misaligned weight pointer. */
+int hia_attn_fwd_ex(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                    hia_tensor v, const float* cos_t, const float* sin_t, float scale,
+                    const hia_qk_norm* norm, hia_tensor o, float* lse, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
 /* hia_attn_fwd for callers that cannot allocate device memory.  (No
  * counterpart on the pages: this is a property of the library, not of the
  * method.)  Some callers may not call cudaMalloc at all: a plug-in inside a
@@ -194,7 +216,8 @@ int hia_attn_fwd_noalloc(const hia_segments* seg, int Hq, int Hkv, int D, hia_te
                          hia_tensor v, const float* cos_t, const float* sin_t, float scale,
                          hia_tensor o, float* lse, void* stream);
 
-/* Bytes of device workspace hia_attn_bwd needs. */
+/* Bytes of device workspace hia_attn_bwd and hia_attn_bwd_ex need (the
+ * size covers the QK RMSNorm's extra accumulators either way). */
 size_t hia_attn_bwd_workspace_bytes(const hia_segments* seg, int Hq, int Hkv, int D);
 
 /* Recompute backward of hia_attn_fwd: given o and lse from the forward and
@@ -207,6 +230,20 @@ int hia_attn_bwd(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, 
                  hia_tensor o, const float* lse, hia_tensor dout, hia_tensor dq,
                  hia_tensor dk, hia_tensor dv, void* workspace, size_t workspace_bytes,
                  void* stream);
+
+/* hia_attn_bwd with an optional QK RMSNorm: norm must be the one given to
+ * the forward that produced o and lse.  With a norm, dq and dk are the
+ * gradients with respect to the un-rotated, un-normed q and k (through the
+ * norm and R^T), and dwq, dwk (fp32 [D] device, overwritten) receive the
+ * gradients of wq and wk summed over every row and head, in a fixed order
+ * (deterministic).  norm == NULL: identical to hia_attn_bwd; dwq, dwk are
+ * ignored.  Errors as hia_attn_fwd_ex, plus HIA_ERR_INVALID_ARG for null
+ * dwq/dwk with a norm. */
+int hia_attn_bwd_ex(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                    hia_tensor v, const float* cos_t, const float* sin_t, float scale,
+                    const hia_qk_norm* norm, hia_tensor o, const float* lse, hia_tensor dout,
+                    hia_tensor dq, hia_tensor dk, hia_tensor dv, float* dwq, float* dwk,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---- One training step from HOST buffers.  (No counterpart on the pages:
  * a convenience of the library for callers that hold their tensors in host

@@ -27,7 +27,7 @@ EXPORTED_SYMBOLS = (
     "hia_attn_fwd_workspace_bytes", "hia_attn_fwd", "hia_attn_bwd_workspace_bytes", "hia_attn_bwd",
     "hia_get_device_status", "hia_debug_wait_timeout", "hia_status_string", "hia_profile_begin",
     "hia_profile_end", "hia_attn_fwd_noalloc", "hia_debug_exp2", "hia_step_create", "hia_step_destroy",
-    "hia_attn_step_host",
+    "hia_attn_step_host", "hia_attn_fwd_ex", "hia_attn_bwd_ex",
 )
 
 
@@ -53,6 +53,10 @@ class SegmentsInfo(ctypes.Structure):
                 ("fwd_tiles_full", ctypes.c_int64), ("fwd_tiles_partial", ctypes.c_int64),
                 ("fwd_tiles_skipped", ctypes.c_int64), ("bwd_q_tiles", ctypes.c_int32),
                 ("bwd_kv_tiles", ctypes.c_int32)]
+
+
+class _QkNorm(ctypes.Structure):
+    _fields_ = [("wq", ctypes.c_void_p), ("wk", ctypes.c_void_p), ("eps", ctypes.c_float)]
 
 
 class _KernelTime(ctypes.Structure):
@@ -88,6 +92,10 @@ def lib():
         L.hia_attn_bwd.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, T, P, T, T, T, T, P, Z, P]
         L.hia_get_device_status.argtypes = [P]
         L.hia_debug_wait_timeout.argtypes = [ctypes.c_uint64, P]
+        QN = ctypes.POINTER(_QkNorm)
+        L.hia_attn_fwd_ex.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, QN, T, P, P, Z, P]
+        L.hia_attn_bwd_ex.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, QN, T, P, T, T, T, T, P, P, P,
+                                      Z, P]
         L.hia_attn_fwd_noalloc.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, T, P, P]
         L.hia_debug_exp2.argtypes = [P, P, I, P]
         L.hia_step_create.argtypes = [P, I, I, I, ctypes.c_double, ctypes.POINTER(P)]
@@ -223,9 +231,25 @@ def _ws(nbytes, workspace):
     return torch.empty(max(nbytes, 1), dtype=torch.uint8, device="cuda")
 
 
-def hia_attn_fwd(seg: Segments, q, k, v, cos, sin, scale=None, o=None, lse=None, workspace=None):
+def _norm(qk_norm, D):
+    """qk_norm = (wq, wk, eps) with fp32 [D] CUDA weights -> pointer to a
+    hia_qk_norm (or None); the tensors are kept alive by the caller."""
+    if qk_norm is None:
+        return None
+    wq, wk, eps = qk_norm
+    for w in (wq, wk):
+        if not w.is_cuda or w.dtype.itemsize != 4 or not w.dtype.is_floating_point or w.numel() != D \
+                or not w.is_contiguous():
+            raise ValueError("QK-norm weights must be contiguous fp32 CUDA tensors of D elements")
+    return ctypes.pointer(_QkNorm(wq.data_ptr(), wk.data_ptr(), float(eps)))
+
+
+def hia_attn_fwd(seg: Segments, q, k, v, cos, sin, scale=None, o=None, lse=None, workspace=None,
+                 qk_norm=None):
     """Forward.  q [B,S,Hq,D], k, v [B,S,Hkv,D] bf16 CUDA tensors (or grouped
-    5-D views).  Returns (o [B,S,Hq,D] bf16, lse [B,Hq,S] fp32)."""
+    5-D views).  Returns (o [B,S,Hq,D] bf16, lse [B,Hq,S] fp32).  qk_norm:
+    optional (wq, wk, eps), fp32 [D] CUDA weights of the per-head RMSNorm
+    applied after RoPE (hia_attn_fwd_ex)."""
     import torch
     Hq, Hkv, D = _heads(q), _heads(k), q.shape[-1]
     g = Hq // Hkv
@@ -237,15 +261,23 @@ def hia_attn_fwd(seg: Segments, q, k, v, cos, sin, scale=None, o=None, lse=None,
         lse = torch.empty(seg.B, Hq, seg.S, device=q.device, dtype=torch.float32)
     nb = hia_attn_fwd_workspace_bytes(seg, Hq, Hkv, D)
     ws = _ws(nb, workspace)
-    _check(lib().hia_attn_fwd(seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1),
-                              cos.data_ptr(), sin.data_ptr(), float(scale), _t(o, True, g), lse.data_ptr(),
-                              ws.data_ptr(), nb, _stream()), "hia_attn_fwd")
+    if qk_norm is None:
+        _check(lib().hia_attn_fwd(seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1),
+                                  cos.data_ptr(), sin.data_ptr(), float(scale), _t(o, True, g), lse.data_ptr(),
+                                  ws.data_ptr(), nb, _stream()), "hia_attn_fwd")
+    else:
+        _check(lib().hia_attn_fwd_ex(seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1),
+                                     cos.data_ptr(), sin.data_ptr(), float(scale), _norm(qk_norm, D),
+                                     _t(o, True, g), lse.data_ptr(), ws.data_ptr(), nb, _stream()),
+               "hia_attn_fwd_ex")
     return o, lse
 
 
 def hia_attn_bwd(seg: Segments, q, k, v, cos, sin, o, lse, dout, scale=None, dq=None, dk=None, dv=None,
-                 workspace=None):
-    """Recompute backward.  Returns (dq, dk, dv) bf16."""
+                 workspace=None, qk_norm=None):
+    """Recompute backward.  Returns (dq, dk, dv) bf16; with qk_norm (the
+    forward's (wq, wk, eps)) returns (dq, dk, dv, dwq, dwk), dwq/dwk fp32 [D]
+    (hia_attn_bwd_ex)."""
     import torch
     Hq, Hkv, D = _heads(q), _heads(k), q.shape[-1]
     g = Hq // Hkv
@@ -259,11 +291,20 @@ def hia_attn_bwd(seg: Segments, q, k, v, cos, sin, o, lse, dout, scale=None, dq=
         dv = torch.empty(seg.B, seg.S, Hkv, D, device=q.device, dtype=torch.bfloat16)
     nb = hia_attn_bwd_workspace_bytes(seg, Hq, Hkv, D)
     ws = _ws(nb, workspace)
-    _check(lib().hia_attn_bwd(seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1),
-                              cos.data_ptr(), sin.data_ptr(), float(scale), _t(o, True, g), lse.data_ptr(),
-                              _t(dout, True, g), _t(dq, True, g), _t(dk, False, 1), _t(dv, False, 1),
-                              ws.data_ptr(), nb, _stream()), "hia_attn_bwd")
-    return dq, dk, dv
+    if qk_norm is None:
+        _check(lib().hia_attn_bwd(seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1),
+                                  cos.data_ptr(), sin.data_ptr(), float(scale), _t(o, True, g), lse.data_ptr(),
+                                  _t(dout, True, g), _t(dq, True, g), _t(dk, False, 1), _t(dv, False, 1),
+                                  ws.data_ptr(), nb, _stream()), "hia_attn_bwd")
+        return dq, dk, dv
+    dwq = torch.empty(D, device=q.device, dtype=torch.float32)
+    dwk = torch.empty(D, device=q.device, dtype=torch.float32)
+    _check(lib().hia_attn_bwd_ex(seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1),
+                                 cos.data_ptr(), sin.data_ptr(), float(scale), _norm(qk_norm, D), _t(o, True, g),
+                                 lse.data_ptr(), _t(dout, True, g), _t(dq, True, g), _t(dk, False, 1),
+                                 _t(dv, False, 1), dwq.data_ptr(), dwk.data_ptr(), ws.data_ptr(), nb, _stream()),
+           "hia_attn_bwd_ex")
+    return dq, dk, dv, dwq, dwk
 
 
 class Step:

@@ -135,8 +135,10 @@ FwdWs fwd_ws(const hia_segments* seg, int Hq, int Hkv, int D) {
 int S_pad64(int S) { return (S + 63) / 64 * 64; }
 
 struct BwdWs {
-  size_t q_off, k_off, lse_off, delta_off, dq_off, total;
+  size_t q_off, k_off, lse_off, delta_off, dq_off, dk_off, dw_off, total;
 };
+// The dK accumulator and the weight-gradient partials are used only with the
+// QK RMSNorm; the size always includes them so one workspace serves both.
 BwdWs bwd_ws(const hia_segments* seg, int Hq, int Hkv, int D) {
   BwdWs w{};
   const size_t BS = size_t(seg->B) * seg->S;
@@ -146,15 +148,26 @@ BwdWs bwd_ws(const hia_segments* seg, int Hq, int Hkv, int D) {
   w.lse_off = w.k_off + align256(BS * Hkv * D * 2);
   w.delta_off = w.lse_off + align256(BSp * Hq * 4);
   w.dq_off = w.delta_off + align256(BSp * Hq * 4);
-  w.total = w.dq_off + align256(BSp * Hq * D * 4);
+  w.dk_off = w.dq_off + align256(BSp * Hq * D * 4);
+  w.dw_off = w.dk_off + align256(BSp * Hkv * D * 4);
+  w.total = w.dw_off + align256(size_t(2) * hia::grad_finalize_blocks(seg->B, seg->S) * D * 4);
   return w;
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? HIA_OK : HIA_ERR_CUDA; }
 
+int check_norm(const hia_qk_norm* n) {
+  if (!n) return HIA_OK;
+  if (!n->wq || !n->wk || !std::isfinite(n->eps) || n->eps < 0.f) return HIA_ERR_INVALID_ARG;
+  if (!aligned16(n->wq) || !aligned16(n->wk)) return HIA_ERR_UNSUPPORTED;
+  return HIA_OK;
+}
+
 void rotate_into(const hia_tensor& src, int H, int g, const float* c, const float* s, __nv_bfloat16* dst,
-                 const hia_segments* seg, int D, cudaStream_t st) {
+                 const hia_segments* seg, int D, cudaStream_t st, const float* w = nullptr, float eps = 0.f) {
   hia::RotateArgs a{};
+  a.w = w;
+  a.eps = eps;
   a.src = src.ptr;
   a.src_sb = src.stride_b;
   a.src_ss = src.stride_s;
@@ -240,8 +253,15 @@ extern "C" size_t hia_attn_bwd_workspace_bytes(const hia_segments* g, int Hq, in
 extern "C" int hia_attn_fwd(const hia_segments* g, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
                             hia_tensor v, const float* c, const float* s, float scale, hia_tensor o, float* lse,
                             void* ws, size_t ws_bytes, void* stream) {
+  return hia_attn_fwd_ex(g, Hq, Hkv, D, q, k, v, c, s, scale, nullptr, o, lse, ws, ws_bytes, stream);
+}
+
+extern "C" int hia_attn_fwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                               hia_tensor v, const float* c, const float* s, float scale, const hia_qk_norm* norm,
+                               hia_tensor o, float* lse, void* ws, size_t ws_bytes, void* stream) {
   int rc = check_common(g, Hq, Hkv, D, c, s);
   if (rc) return rc;
+  if ((rc = check_norm(norm))) return rc;
   if (g->B == 0 || g->S == 0) return HIA_OK;
   if (!std::isfinite(scale) || !(scale > 0.f)) return HIA_ERR_INVALID_ARG;
   const int gq = Hq / Hkv;
@@ -263,8 +283,8 @@ extern "C" int hia_attn_fwd(const hia_segments* g, int Hq, int Hkv, int D, hia_t
       !make_kv_map(&tv, v, D, Hkv, g->S, g->B, 128))
     return HIA_ERR_CUDA;
 
-  rotate_into(q, Hq, gq, c, s, qr, g, D, st);
-  rotate_into(k, Hkv, 1, c, s, kr, g, D, st);
+  rotate_into(q, Hq, gq, c, s, qr, g, D, st, norm ? norm->wq : nullptr, norm ? norm->eps : 0.f);
+  rotate_into(k, Hkv, 1, c, s, kr, g, D, st, norm ? norm->wk : nullptr, norm ? norm->eps : 0.f);
 
   hia::FwdParams p{};
   p.samples = g->d_samples;
@@ -322,8 +342,18 @@ extern "C" int hia_attn_bwd(const hia_segments* g, int Hq, int Hkv, int D, hia_t
                             hia_tensor v, const float* c, const float* s, float scale, hia_tensor o,
                             const float* lse, hia_tensor dout, hia_tensor dq, hia_tensor dk, hia_tensor dv,
                             void* ws, size_t ws_bytes, void* stream) {
+  return hia_attn_bwd_ex(g, Hq, Hkv, D, q, k, v, c, s, scale, nullptr, o, lse, dout, dq, dk, dv, nullptr, nullptr,
+                         ws, ws_bytes, stream);
+}
+
+extern "C" int hia_attn_bwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                               hia_tensor v, const float* c, const float* s, float scale, const hia_qk_norm* norm,
+                               hia_tensor o, const float* lse, hia_tensor dout, hia_tensor dq, hia_tensor dk,
+                               hia_tensor dv, float* dwq, float* dwk, void* ws, size_t ws_bytes, void* stream) {
   int rc = check_common(g, Hq, Hkv, D, c, s);
   if (rc) return rc;
+  if ((rc = check_norm(norm))) return rc;
+  if (norm && (!dwq || !dwk)) return HIA_ERR_INVALID_ARG;
   if (g->B == 0 || g->S == 0) return HIA_OK;
   if (!std::isfinite(scale) || !(scale > 0.f)) return HIA_ERR_INVALID_ARG;
   const int gq = Hq / Hkv;
@@ -345,6 +375,8 @@ extern "C" int hia_attn_bwd(const hia_segments* g, int Hq, int Hkv, int D, hia_t
   float* lse2 = reinterpret_cast<float*>(wb + w.lse_off);
   float* delta = reinterpret_cast<float*>(wb + w.delta_off);
   float* dq_acc = reinterpret_cast<float*>(wb + w.dq_off);
+  float* dk_acc = reinterpret_cast<float*>(wb + w.dk_off);
+  float* dw_part = reinterpret_cast<float*>(wb + w.dw_off);
   const int S_pad = S_pad64(g->S);
 
   CUtensorMap tq, tk, tv, tdo;
@@ -352,8 +384,8 @@ extern "C" int hia_attn_bwd(const hia_segments* g, int Hq, int Hkv, int D, hia_t
       !make_kv_map(&tv, v, D, Hkv, g->S, g->B, 128) || !make_q_map(&tdo, dout, D, gq, Hkv, g->S, g->B, 64))
     return HIA_ERR_CUDA;
 
-  rotate_into(q, Hq, gq, c, s, qr, g, D, st);
-  rotate_into(k, Hkv, 1, c, s, kr, g, D, st);
+  rotate_into(q, Hq, gq, c, s, qr, g, D, st, norm ? norm->wq : nullptr, norm ? norm->eps : 0.f);
+  rotate_into(k, Hkv, 1, c, s, kr, g, D, st, norm ? norm->wk : nullptr, norm ? norm->eps : 0.f);
   if (cudaMemsetAsync(dq_acc, 0, size_t(g->B) * Hq * S_pad * D * 4, st) != cudaSuccess) return HIA_ERR_CUDA;
 
   hia::BwdPreParams pp{};
@@ -404,6 +436,7 @@ extern "C" int hia_attn_bwd(const hia_segments* g, int Hq, int Hkv, int D, hia_t
   p.dv_sb = dv.stride_b;
   p.dv_ss = dv.stride_s;
   p.dv_sh = dv.stride_hkv;
+  p.dk_acc = norm ? dk_acc : nullptr;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = status;
@@ -412,12 +445,22 @@ extern "C" int hia_attn_bwd(const hia_segments* g, int Hq, int Hkv, int D, hia_t
   if (n_blocks > (1ll << 31) - 1) return HIA_ERR_UNSUPPORTED;
   if ((rc = cuda_status(hia::launch_attn_bwd(tq, tk, tv, tdo, p, int(n_blocks), D, st)))) return rc;
 
-  hia::DqFinalArgs fa{};
+  // dq = R^T (norm backward of) scale * dq_acc; with the norm also dk from dk_acc and the weight gradients
+  const int nblk = hia::grad_finalize_blocks(g->B, g->S);
+  hia::GradFinalArgs fa{};
   fa.acc = dq_acc;
   fa.S_pad = S_pad;
   fa.scale = scale;
   fa.cos_t = c;
   fa.sin_t = s;
+  fa.x = q.ptr;
+  fa.x_sb = q.stride_b;
+  fa.x_ss = q.stride_s;
+  fa.x_shkv = q.stride_hkv;
+  fa.x_shq = q.stride_hq;
+  fa.w = norm ? norm->wq : nullptr;
+  fa.eps = norm ? norm->eps : 0.f;
+  fa.dw_part = dw_part;
   fa.dst = dq.ptr;
   fa.dst_sb = dq.stride_b;
   fa.dst_ss = dq.stride_s;
@@ -427,6 +470,28 @@ extern "C" int hia_attn_bwd(const hia_segments* g, int Hq, int Hkv, int D, hia_t
   fa.B = g->B;
   fa.S = g->S;
   fa.H = Hq;
-  hia::launch_dq_finalize(fa, D, st);
+  hia::launch_grad_finalize(fa, D, st);
+  if (norm) {
+    hia::launch_dw_reduce(dw_part, nblk, D, dwq, st);
+    hia::GradFinalArgs fk = fa;
+    fk.acc = dk_acc;
+    fk.scale = 1.f;  // the epilogue already applied the softmax scale
+    fk.x = k.ptr;
+    fk.x_sb = k.stride_b;
+    fk.x_ss = k.stride_s;
+    fk.x_shkv = k.stride_hkv;
+    fk.x_shq = 0;
+    fk.w = norm->wk;
+    fk.dw_part = dw_part + size_t(nblk) * D;
+    fk.dst = dk.ptr;
+    fk.dst_sb = dk.stride_b;
+    fk.dst_ss = dk.stride_s;
+    fk.dst_shkv = dk.stride_hkv;
+    fk.dst_shq = 0;
+    fk.g = 1;
+    fk.H = Hkv;
+    hia::launch_grad_finalize(fk, D, st);
+    hia::launch_dw_reduce(dw_part + size_t(nblk) * D, nblk, D, dwk, st);
+  }
   return cuda_status(cudaGetLastError());
 }

@@ -308,7 +308,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (have) have = __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, wc));
     if (have) tc_fence_after();
     const bool store = key < p.S;
-    if (bf == 0) {
+    if (bf == 0 && p.dk_acc) {
+      // QK RMSNorm: the norm's backward needs the whole row, so write
+      // scale * dK_n (gradient w.r.t. the normed rotated key row) in fp32 and
+      // let the gradient epilogue kernel finish it
+      float* arow = p.dk_acc + ((int64_t(b) * p.Hkv + hkv) * p.S_pad + key) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        if (have) {
+          tmem_ld32(tdK + lane_off + c * 32, ov);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = 0u;
+        }
+        if (store) {
+          float4* d0 = reinterpret_cast<float4*>(arow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            d0[i] = make_float4(__uint_as_float(ov[4 * i]) * p.scale, __uint_as_float(ov[4 * i + 1]) * p.scale,
+                                __uint_as_float(ov[4 * i + 2]) * p.scale, __uint_as_float(ov[4 * i + 3]) * p.scale);
+        }
+      }
+    } else if (bf == 0) {
       const int kc = store ? key : p.S - 1;
       const float* cp = p.cos_t + (int64_t(b) * p.S + kc) * D;
       const float* sp = p.sin_t + (int64_t(b) * p.S + kc) * D;

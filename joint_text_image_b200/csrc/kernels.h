@@ -14,17 +14,24 @@ struct RotateArgs {
   int g;            // heads per stride_hkv group (1 for k)
   const float* cos_t;
   const float* sin_t;
+  const float* w;   // QK RMSNorm weight [D], or nullptr: no norm
+  float eps;
   __nv_bfloat16* dst;  // [B][H][S][D]
   int B, S, H;
 };
 
-struct DqFinalArgs {
-  const float* acc;  // fp32 [B][H][S_pad][D]
+struct GradFinalArgs {
+  const float* acc;  // fp32 [B][H][S_pad][D]: gradient w.r.t. the attention's input rows (times 1/scale)
   int S_pad;
   float scale;
   const float* cos_t;
   const float* sin_t;
-  void* dst;
+  const void* x;     // the layer input rows (q or k), bf16 with strides; read only with the norm
+  int64_t x_sb, x_ss, x_shkv, x_shq;
+  const float* w;    // QK RMSNorm weight [D], or nullptr: no norm
+  float eps;
+  float* dw_part;    // [grad_finalize_blocks][D] per-block weight-gradient partials (with the norm)
+  void* dst;         // bf16 with strides
   int64_t dst_sb, dst_ss, dst_shkv, dst_shq;
   int g;
   int B, S, H;
@@ -67,6 +74,7 @@ struct BwdParams {
   const float* sin_t;
   __nv_bfloat16* dk;
   int64_t dk_sb, dk_ss, dk_sh;
+  float* dk_acc;      // non-null (QK RMSNorm): write scale * dK_n rows fp32 [B][Hkv][S_pad][D] here instead of dk
   __nv_bfloat16* dv;
   int64_t dv_sb, dv_ss, dv_sh;
   float scale;        // softmax scale
@@ -76,14 +84,16 @@ struct BwdParams {
 };
 
 // Profiling brackets around one kernel launch (no-ops unless profiling is on).
-enum KernelId { kRopeTables = 0, kRopeRotate, kAttnFwd, kBwdPre, kAttnBwd, kDqFinalize, kNumKernels };
+enum KernelId { kRopeTables = 0, kRopeRotate, kAttnFwd, kBwdPre, kAttnBwd, kGradFinalize, kDwReduce, kNumKernels };
 void prof_begin(KernelId id, cudaStream_t st);
 void prof_end(KernelId id, cudaStream_t st);
 
 void launch_rope2d_tables(const SampleDev* samples, int B, int S, int D, double base, float* cos_out,
                           float* sin_out, cudaStream_t st);
 void launch_rope_rotate(const RotateArgs& a, int D, cudaStream_t st);
-void launch_dq_finalize(const DqFinalArgs& a, int D, cudaStream_t st);
+int grad_finalize_blocks(int B, int S);
+void launch_grad_finalize(const GradFinalArgs& a, int D, cudaStream_t st);
+void launch_dw_reduce(const float* part, int nblk, int D, float* dw, cudaStream_t st);
 cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int n_blocks, int D, cudaStream_t st);
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st);

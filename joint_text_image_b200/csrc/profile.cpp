@@ -11,7 +11,7 @@
 namespace {
 
 const char* kNames[hia::kNumKernels] = {"rope2d_tables", "rope_rotate", "attn_fwd",
-                                        "bwd_pre", "attn_bwd", "dq_finalize"};
+                                        "bwd_pre", "attn_bwd", "grad_finalize", "dw_reduce"};
 
 struct Rec {
   int id;

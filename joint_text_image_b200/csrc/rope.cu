@@ -47,99 +47,218 @@ __global__ void rope2d_tables_kernel(const SampleDev* __restrict__ samples, int 
   }
 }
 
-// Rotation pre-pass: dst[b][h][s][:] = R(b,s) src[b,s,h,:] in fp32, rounded
-// to bf16.  One warp per (b, s): each lane owns 8 channels of the low half
-// and the matching 8 of the high half of one head; the cos/sin of the row are
-// read once and reused for every head.  inverse = 1 applies R^T instead and
-// reads fp32 input (used for dq).
+// Row helpers shared by the rotation pre-pass and the gradient epilogue.  A
+// warp owns one (b, s) row; lane = hs * CPH + c owns channels c*8 .. c*8+7 of
+// the low half and the matching 8 of the high half of one head (CPH = D/16
+// lanes per head, HPI = 32/CPH heads per pass).  A sum over one head's
+// channels is a butterfly over the CPH lanes of the head's lane group.
 template <int D>
-__global__ void __launch_bounds__(256) rope_rotate_kernel(RotateArgs a) {
-  constexpr int CPH = D / 16;  // 8-channel chunks per half-head
-  constexpr int HPI = 32 / CPH;  // heads per warp iteration
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= a.B * a.S) return;
-  const int b = warp / a.S, s = warp % a.S;
-  const int c = lane % CPH, hs = lane / CPH;
-  const float* cp = a.cos_t + (int64_t(b) * a.S + s) * D + c * 8;
-  const float* sp = a.sin_t + (int64_t(b) * a.S + s) * D + c * 8;
-  const float4 c0 = __ldg(reinterpret_cast<const float4*>(cp)), c1 = __ldg(reinterpret_cast<const float4*>(cp) + 1);
-  const float4 s0 = __ldg(reinterpret_cast<const float4*>(sp)), s1 = __ldg(reinterpret_cast<const float4*>(sp) + 1);
-  const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-  const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-  for (int h = hs; h < a.H; h += HPI) {
-    const int64_t so = int64_t(b) * a.src_sb + int64_t(s) * a.src_ss + int64_t(h / a.g) * a.src_shkv +
-                       int64_t(h % a.g) * a.src_shq;
-    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.src) + so;
-    const uint4 lo4 = *reinterpret_cast<const uint4*>(src + c * 8);
-    const uint4 hi4 = *reinterpret_cast<const uint4*>(src + D / 2 + c * 8);
-    const __nv_bfloat162* lo2 = reinterpret_cast<const __nv_bfloat162*>(&lo4);
-    const __nv_bfloat162* hi2 = reinterpret_cast<const __nv_bfloat162*>(&hi4);
-    uint4 olo, ohi;
-    __nv_bfloat162* ol = reinterpret_cast<__nv_bfloat162*>(&olo);
-    __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&ohi);
+struct RowLanes {
+  static constexpr int CPH = D / 16;
+  static constexpr int HPI = 32 / CPH;
+  int c, hs;
+  unsigned gmask;
+  __device__ explicit RowLanes(int lane) : c(lane % CPH), hs(lane / CPH) {
+    gmask = (CPH == 32 ? 0xffffffffu : ((1u << CPH) - 1u)) << (hs * CPH);
+  }
+  __device__ float head_sum(float v) const {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 l = __bfloat1622float2(lo2[i]);
-      const float2 u = __bfloat1622float2(hi2[i]);
-      const float cA = cs[2 * i], cB = cs[2 * i + 1], sA = sn[2 * i], sB = sn[2 * i + 1];
-      const float nlA = fmaf(l.x, cA, -u.x * sA), nlB = fmaf(l.y, cB, -u.y * sB);
-      const float nuA = fmaf(u.x, cA, l.x * sA), nuB = fmaf(u.y, cB, l.y * sB);
-      ol[i] = __floats2bfloat162_rn(nlA, nlB);
-      oh[i] = __floats2bfloat162_rn(nuA, nuB);
-    }
-    __nv_bfloat16* dst = a.dst + ((int64_t(b) * a.H + h) * a.S + s) * D;
-    *reinterpret_cast<uint4*>(dst + c * 8) = olo;
-    *reinterpret_cast<uint4*>(dst + D / 2 + c * 8) = ohi;
+    for (int o = 1; o < CPH; o <<= 1) v += __shfl_xor_sync(gmask, v, o);
+    return v;
+  }
+};
+
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 x0 = __ldg(reinterpret_cast<const float4*>(p)), x1 = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w; v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+}
+
+__device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h2[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
   }
 }
 
-// dq epilogue: dq[b,s,h,:] = R(b,s)^T (scale * acc[b][h][s][:]) in fp32,
-// rounded to bf16 and written with the caller's strides.
+__device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8]) {
+  uint4 u;
+  __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h2[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  return u;
+}
+
+// Rotation pre-pass: dst[b][h][s][:] = R(b,s) src[b,s,h,:] in fp32, rounded
+// to bf16.  With QK RMSNorm weights (a.w != nullptr) the rotated row x is
+// replaced by w * x / sqrt(mean(x^2) + eps) before the rounding
+// (HunyuanImage3Attention applies RoPE, then the per-head QK RMSNorm).  The
+// cos/sin of the row are read once and reused for every head.
 template <int D>
-__global__ void __launch_bounds__(256) dq_finalize_kernel(DqFinalArgs a) {
-  constexpr int CPH = D / 16;
-  constexpr int HPI = 32 / CPH;
+__global__ void __launch_bounds__(256) rope_rotate_kernel(RotateArgs a) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= a.B * a.S) return;
   const int b = warp / a.S, s = warp % a.S;
-  const int c = lane % CPH, hs = lane / CPH;
-  const float* cp = a.cos_t + (int64_t(b) * a.S + s) * D + c * 8;
-  const float* sp = a.sin_t + (int64_t(b) * a.S + s) * D + c * 8;
-  const float4 c0 = __ldg(reinterpret_cast<const float4*>(cp)), c1 = __ldg(reinterpret_cast<const float4*>(cp) + 1);
-  const float4 s0 = __ldg(reinterpret_cast<const float4*>(sp)), s1 = __ldg(reinterpret_cast<const float4*>(sp) + 1);
-  const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-  const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-  for (int h = hs; h < a.H; h += HPI) {
-    const float* src = a.acc + ((int64_t(b) * a.H + h) * a.S_pad + s) * D;
-    float lo[8], hi[8];
-    *reinterpret_cast<float4*>(lo) = *reinterpret_cast<const float4*>(src + c * 8);
-    *reinterpret_cast<float4*>(lo + 4) = *reinterpret_cast<const float4*>(src + c * 8 + 4);
-    *reinterpret_cast<float4*>(hi) = *reinterpret_cast<const float4*>(src + D / 2 + c * 8);
-    *reinterpret_cast<float4*>(hi + 4) = *reinterpret_cast<const float4*>(src + D / 2 + c * 8 + 4);
-    uint4 olo, ohi;
-    __nv_bfloat162* ol = reinterpret_cast<__nv_bfloat162*>(&olo);
-    __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&ohi);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float r[4];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int k = 2 * i + e;
-        const float l = lo[k] * a.scale, u = hi[k] * a.scale;
-        r[e] = fmaf(l, cs[k], u * sn[k]);        // (R^T v)_j
-        r[2 + e] = fmaf(u, cs[k], -l * sn[k]);   // (R^T v)_{j+D/2}
-      }
-      ol[i] = __floats2bfloat162_rn(r[0], r[1]);
-      oh[i] = __floats2bfloat162_rn(r[2], r[3]);
-    }
-    const int64_t so = int64_t(b) * a.dst_sb + int64_t(s) * a.dst_ss + int64_t(h / a.g) * a.dst_shkv +
-                       int64_t(h % a.g) * a.dst_shq;
-    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.dst) + so;
-    *reinterpret_cast<uint4*>(dst + c * 8) = olo;
-    *reinterpret_cast<uint4*>(dst + D / 2 + c * 8) = ohi;
+  const RowLanes<D> L(lane);
+  float cs[8], sn[8], wl[8], wh[8];
+  load8(a.cos_t + (int64_t(b) * a.S + s) * D + L.c * 8, cs);
+  load8(a.sin_t + (int64_t(b) * a.S + s) * D + L.c * 8, sn);
+  const bool norm = a.w != nullptr;
+  if (norm) {
+    load8(a.w + L.c * 8, wl);
+    load8(a.w + D / 2 + L.c * 8, wh);
   }
+  for (int h = L.hs; h < a.H; h += RowLanes<D>::HPI) {
+    const int64_t so = int64_t(b) * a.src_sb + int64_t(s) * a.src_ss + int64_t(h / a.g) * a.src_shkv +
+                       int64_t(h % a.g) * a.src_shq;
+    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.src) + so;
+    float l[8], u[8], xl[8], xu[8];
+    load8_bf16(src + L.c * 8, l);
+    load8_bf16(src + D / 2 + L.c * 8, u);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      xl[k] = fmaf(l[k], cs[k], -u[k] * sn[k]);
+      xu[k] = fmaf(u[k], cs[k], l[k] * sn[k]);
+    }
+    if (norm) {
+      float ss = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ss = fmaf(xl[k], xl[k], fmaf(xu[k], xu[k], ss));
+      const float r = rsqrtf(L.head_sum(ss) * (1.0f / D) + a.eps);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        xl[k] = wl[k] * (xl[k] * r);
+        xu[k] = wh[k] * (xu[k] * r);
+      }
+    }
+    __nv_bfloat16* dst = a.dst + ((int64_t(b) * a.H + h) * a.S + s) * D;
+    *reinterpret_cast<uint4*>(dst + L.c * 8) = pack8_bf16(xl);
+    *reinterpret_cast<uint4*>(dst + D / 2 + L.c * 8) = pack8_bf16(xu);
+  }
+}
+
+// Gradient epilogue for dq (and, with the QK RMSNorm, dk): for every row,
+// v = scale * acc[b][h][s][:] is the gradient with respect to the attention's
+// input row y.  Without the norm y = R x_in and the result is R^T v.  With it,
+// y = w * xh, xh = x r, x = R x_in, r = 1/sqrt(mean(x^2) + eps): the gradient
+// with respect to x is r (w v - xh <w v, xh> / D), then R^T; the weight
+// gradient w += v * xh is summed per block into dw_part[blockIdx.x][:] in a
+// fixed order (deterministic), and dw_reduce_kernel adds the blocks.
+template <int D>
+__global__ void __launch_bounds__(256) grad_finalize_kernel(GradFinalArgs a) {
+  constexpr int CPH = RowLanes<D>::CPH, HPI = RowLanes<D>::HPI;
+  __shared__ float red[8][32][16];
+  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = blockIdx.x * 8 + wib;
+  const RowLanes<D> L(lane);
+  const bool norm = a.w != nullptr;
+  float dwl[8], dwh[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) dwl[k] = dwh[k] = 0.f;
+  if (warp < a.B * a.S) {
+    const int b = warp / a.S, s = warp % a.S;
+    float cs[8], sn[8], wl[8], wh[8];
+    load8(a.cos_t + (int64_t(b) * a.S + s) * D + L.c * 8, cs);
+    load8(a.sin_t + (int64_t(b) * a.S + s) * D + L.c * 8, sn);
+    if (norm) {
+      load8(a.w + L.c * 8, wl);
+      load8(a.w + D / 2 + L.c * 8, wh);
+    }
+    for (int h = L.hs; h < a.H; h += HPI) {
+      const float* src = a.acc + ((int64_t(b) * a.H + h) * a.S_pad + s) * D;
+      float vl[8], vu[8];
+      *reinterpret_cast<float4*>(vl) = *reinterpret_cast<const float4*>(src + L.c * 8);
+      *reinterpret_cast<float4*>(vl + 4) = *reinterpret_cast<const float4*>(src + L.c * 8 + 4);
+      *reinterpret_cast<float4*>(vu) = *reinterpret_cast<const float4*>(src + D / 2 + L.c * 8);
+      *reinterpret_cast<float4*>(vu + 4) = *reinterpret_cast<const float4*>(src + D / 2 + L.c * 8 + 4);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        vl[k] *= a.scale;
+        vu[k] *= a.scale;
+      }
+      if (norm) {
+        const int64_t xo = int64_t(b) * a.x_sb + int64_t(s) * a.x_ss + int64_t(h / a.g) * a.x_shkv +
+                           int64_t(h % a.g) * a.x_shq;
+        const __nv_bfloat16* xin = reinterpret_cast<const __nv_bfloat16*>(a.x) + xo;
+        float l[8], u[8], xl[8], xu[8];
+        load8_bf16(xin + L.c * 8, l);
+        load8_bf16(xin + D / 2 + L.c * 8, u);
+        float ss = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          xl[k] = fmaf(l[k], cs[k], -u[k] * sn[k]);
+          xu[k] = fmaf(u[k], cs[k], l[k] * sn[k]);
+          ss = fmaf(xl[k], xl[k], fmaf(xu[k], xu[k], ss));
+        }
+        const float r = rsqrtf(L.head_sum(ss) * (1.0f / D) + a.eps);
+        float dot = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          xl[k] *= r;  // xh
+          xu[k] *= r;
+          dwl[k] = fmaf(vl[k], xl[k], dwl[k]);
+          dwh[k] = fmaf(vu[k], xu[k], dwh[k]);
+          vl[k] *= wl[k];  // w v
+          vu[k] *= wh[k];
+          dot = fmaf(vl[k], xl[k], fmaf(vu[k], xu[k], dot));
+        }
+        const float m = L.head_sum(dot) * (1.0f / D);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          vl[k] = r * fmaf(-xl[k], m, vl[k]);
+          vu[k] = r * fmaf(-xu[k], m, vu[k]);
+        }
+      }
+      float ol[8], ou[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        ol[k] = fmaf(vl[k], cs[k], vu[k] * sn[k]);   // (R^T v)_j
+        ou[k] = fmaf(vu[k], cs[k], -vl[k] * sn[k]);  // (R^T v)_{j+D/2}
+      }
+      const int64_t so = int64_t(b) * a.dst_sb + int64_t(s) * a.dst_ss + int64_t(h / a.g) * a.dst_shkv +
+                         int64_t(h % a.g) * a.dst_shq;
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.dst) + so;
+      *reinterpret_cast<uint4*>(dst + L.c * 8) = pack8_bf16(ol);
+      *reinterpret_cast<uint4*>(dst + D / 2 + L.c * 8) = pack8_bf16(ou);
+    }
+  }
+  if (!norm) return;  // uniform across the block
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    red[wib][lane][k] = dwl[k];
+    red[wib][lane][8 + k] = dwh[k];
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    const int j = d % (D / 2), c = j / 8, k = (j % 8) + (d >= D / 2 ? 8 : 0);
+    float t = 0.f;
+    for (int w8 = 0; w8 < 8; ++w8)
+      for (int h2 = 0; h2 < HPI; ++h2) t += red[w8][c + CPH * h2][k];
+    a.dw_part[int64_t(blockIdx.x) * D + d] = t;
+  }
+}
+
+// dw[d] = sum over blocks of dw_part[blk][d]: 32 channels x 32 block rows per
+// CTA, a fixed strided split and a fixed tree (deterministic).
+__global__ void __launch_bounds__(1024) dw_reduce_kernel(const float* __restrict__ part, int nblk, int D,
+                                                         float* __restrict__ dw) {
+  __shared__ float t[32][33];
+  const int cx = threadIdx.x & 31, ry = threadIdx.x >> 5;
+  const int d = blockIdx.x * 32 + cx;
+  float s = 0.f;
+  if (d < D)
+    for (int i = ry; i < nblk; i += 32) s += part[int64_t(i) * D + d];
+  t[ry][cx] = s;
+  __syncthreads();
+  for (int o = 16; o > 0; o >>= 1) {
+    if (ry < o) t[ry][cx] += t[ry + o][cx];
+    __syncthreads();
+  }
+  if (ry == 0 && d < D) dw[d] = t[0][cx];
 }
 
 void launch_rope2d_tables(const SampleDev* samples, int B, int S, int D, double base, float* cos_out,
@@ -164,14 +283,21 @@ void launch_rope_rotate(const RotateArgs& a, int D, cudaStream_t st) {
   prof_end(kRopeRotate, st);
 }
 
-void launch_dq_finalize(const DqFinalArgs& a, int D, cudaStream_t st) {
-  const int64_t warps = int64_t(a.B) * a.S;
-  if (warps == 0) return;
-  const int blocks = int((warps + 7) / 8);
-  prof_begin(kDqFinalize, st);
-  if (D == 128) dq_finalize_kernel<128><<<blocks, 256, 0, st>>>(a);
-  else dq_finalize_kernel<64><<<blocks, 256, 0, st>>>(a);
-  prof_end(kDqFinalize, st);
+int grad_finalize_blocks(int B, int S) { return int((int64_t(B) * S + 7) / 8); }
+
+void launch_grad_finalize(const GradFinalArgs& a, int D, cudaStream_t st) {
+  const int blocks = grad_finalize_blocks(a.B, a.S);
+  if (blocks == 0) return;
+  prof_begin(kGradFinalize, st);
+  if (D == 128) grad_finalize_kernel<128><<<blocks, 256, 0, st>>>(a);
+  else grad_finalize_kernel<64><<<blocks, 256, 0, st>>>(a);
+  prof_end(kGradFinalize, st);
+}
+
+void launch_dw_reduce(const float* part, int nblk, int D, float* dw, cudaStream_t st) {
+  prof_begin(kDwReduce, st);
+  dw_reduce_kernel<<<(D + 31) / 32, 1024, 0, st>>>(part, nblk, D, dw);
+  prof_end(kDwReduce, st);
 }
 
 }  // namespace hia

@@ -46,9 +46,10 @@ def sample_rows(wl, n_per_segment=6, seed=0):
     return sorted(r for r in rows if 0 <= r < wl.S)
 
 
-def check_fwd(oracle_mod, wl, q, k, v, o, lse, rows=None, groups=None):
+def check_fwd(oracle_mod, wl, q, k, v, o, lse, rows=None, groups=None, qk_norm=None):
     o_ref, lse_ref, _ = oracle_mod.attn_fwd(wl.samples, q.double().numpy(), k.double().numpy(),
-                                            v.double().numpy(), wl.scale, wl.base, rows=rows, groups=groups)
+                                            v.double().numpy(), wl.scale, wl.base, rows=rows, groups=groups,
+                                            qk_norm=qk_norm)
     sel_r = slice(None) if rows is None else np.asarray(rows)
     g = wl.Hq // wl.Hkv
     if groups is None:
@@ -92,11 +93,23 @@ def run_fwd_bwd(wl, seed=0):
     return (q, k, v, do), (f(dq), f(dk), f(dv))
 
 
-def check_bwd(oracle_mod, wl, inputs, grads, groups=None):
+def check_bwd(oracle_mod, wl, inputs, grads, groups=None, qk_norm=None, dw=None):
+    """dq, dk, dv against the oracle by relative Frobenius norm; with qk_norm
+    also the weight gradients dw = (dwq, dwk) (full problems only)."""
     q, k, v, do = inputs
     f64 = lambda t: t.double().numpy()
-    ref = oracle_mod.attn_bwd(wl.samples, f64(q), f64(k), f64(v), f64(do), wl.scale, wl.base,
-                              groups=groups)[:3]
+    if qk_norm is None:
+        ref = oracle_mod.attn_bwd(wl.samples, f64(q), f64(k), f64(v), f64(do), wl.scale, wl.base,
+                                  groups=groups)[:3]
+    else:
+        full = oracle_mod.attn_bwd_qknorm(wl.samples, f64(q), f64(k), f64(v), f64(do), qk_norm, wl.scale,
+                                          wl.base, groups=groups)
+        ref = full[:3]
+        if dw is not None:
+            for name, got, r in zip(("dwq", "dwk"), dw, full[3:5]):
+                rel = np.linalg.norm(np.asarray(got, dtype=np.float64) - r) / np.linalg.norm(r)
+                assert rel <= GRAD_REL, f"{name} relative Frobenius {rel:.3e}"
+                print(f"[parity-bwd] {wl.name}: {name} {rel:.3e}")
     g = wl.Hq // wl.Hkv
     gsel = np.ones((wl.B, wl.Hkv), dtype=bool) if groups is None else np.asarray(groups, dtype=bool)
     out = {}
