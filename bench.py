@@ -196,6 +196,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD, choices=["tiny", "256px", "1024px", "mixed", "1024px_bwd"],
                     help="synthetic workload (the metric is quoted on 1024px; the others are for profiling)")
+    ap.add_argument("--packed", action="store_true",
+                    help="packed (varlen) layout: no padded rows (no e2e line: the host step is padded-only)")
     ap.add_argument("--qk-norm", action="store_true",
                     help="enable the per-head QK RMSNorm after RoPE (weights seeded, eps 1e-5)")
     ap.add_argument("--source-hash", choices=sorted(KERNEL_SOURCES),
@@ -231,7 +233,14 @@ def main():
 
     wl = synth.workload(args.workload, seed=args.seed)
     q, k, v, do = synth.tensors(wl, args.seed + rank, grad=True)
-    seg = jt.hia_segments_build(wl.samples, wl.S)
+    padded_inputs = (q, k, v, do)
+    if args.packed:
+        # the same draws in the packed (varlen) layout: each sample's rows back to back
+        seg = jt.hia_segments_build_packed(wl.samples)
+        packf = lambda x: torch.cat([x[b, :L] for b, L in enumerate(seg.lengths)], 0).contiguous()
+        q, k, v, do = (packf(t) for t in (q, k, v, do))
+    else:
+        seg = jt.hia_segments_build(wl.samples, wl.S)
     info = seg.info()
     pairs = info.visible_pairs
     fwd_flops = 4.0 * wl.D * wl.Hq * pairs
@@ -239,9 +248,9 @@ def main():
     step_flops = fwd_flops + bwd_flops
 
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
-    cs = (torch.empty(wl.B, wl.S, wl.D, device=dev), torch.empty(wl.B, wl.S, wl.D, device=dev))
+    cs = (torch.empty(wl.B, seg.S, wl.D, device=dev), torch.empty(wl.B, seg.S, wl.D, device=dev))
     o = torch.empty_like(qd)
-    lse = torch.empty(wl.B, wl.Hq, wl.S, device=dev)
+    lse = torch.empty((wl.Hq, seg.total_rows) if args.packed else (wl.B, wl.Hq, wl.S), device=dev)
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
     wsf = torch.empty(jt.hia_attn_fwd_workspace_bytes(seg, wl.Hq, wl.Hkv, wl.D), dtype=torch.uint8, device=dev)
     wsb = torch.empty(jt.hia_attn_bwd_workspace_bytes(seg, wl.Hq, wl.Hkv, wl.D), dtype=torch.uint8, device=dev)
@@ -317,7 +326,7 @@ def main():
     # the other's kernels, as a training loop feeding the op from host memory
     # would run it.
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and not args.packed:  # the host-buffer step uses the padded layout
         hin = [tuple(t.pin_memory() for t in (q, k, v, do)) for _ in range(2)]
         mk = lambda t, dt=torch.bfloat16: torch.empty(t.shape, dtype=dt, pin_memory=True)
         hout = [(mk(o), mk(lse, torch.float32), mk(dq), mk(dk), mk(dv)) for _ in range(2)]
@@ -354,7 +363,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = sample_rows(wl.S, args.ref_row_stride)
-        dt, fl, used = oracle_sample_step(wl, q, k, v, do, rows)
+        dt, fl, used = oracle_sample_step(wl, *padded_inputs, rows)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOPS", "cores": used, "kind": "oracle",
                "sample": SAMPLE_DESC.format(g=wl.Hq // wl.Hkv, stride=args.ref_row_stride, n=len(rows))
                          + f", one step of {dt:.2f} s"}
@@ -370,7 +379,8 @@ def main():
                        "parallelism": f"replicas x{world} (no cross-GPU exchange in this op)",
                        "l2": f"inputs larger than L2: {(q.numel() + k.numel() + v.numel() + do.numel()) * 2 / 1e6:.0f} MB read per step",
                        "visible_pairs": pairs, "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
-                       "qk_norm": ({"eps": 1e-5, "weights": "seeded U[0.5,1.5)"} if args.qk_norm else None)},
+                       "qk_norm": ({"eps": 1e-5, "weights": "seeded U[0.5,1.5)"} if args.qk_norm else None),
+                       "layout": f"packed ({seg.total_rows} rows)" if args.packed else "padded"},
             "pct_of_bf16_peak": value / world / peak_burst * 100.0,
             "fwd_tflops": fwd_flops / (fwd_t * 1e-3) / 1e12 if fwd_t else None,
             "bwd_tflops": bwd_flops / (bwd_t * 1e-3) / 1e12 if bwd_t else None,

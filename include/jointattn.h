@@ -89,6 +89,9 @@ typedef struct {
     int64_t fwd_tiles_skipped;   /* fully masked, incl. padded keys: never loaded */
     int32_t bwd_q_tiles;         /* ceil(S / 64) */
     int32_t bwd_kv_tiles;        /* ceil(S / 128) */
+    int32_t packed;              /* 1: built by hia_segments_build_packed */
+    int32_t reserved;
+    int64_t total_rows;          /* rows of a tensor in this layout: B*S, or the sum of L when packed */
 } hia_segments_info_t;
 
 /* Tile classes reported by hia_segments_tile_classes. */
@@ -113,6 +116,17 @@ enum {
  * lengths, exactly one of img_h/img_w zero, L > S, S >= 2^24). */
 int hia_segments_build(const hia_sample* samples, int B, int S, hia_segments** out);
 
+/* The same descriptor for the PACKED (varlen) layout: the samples are stored
+ * back to back with no padding rows, sample b's rows starting at row
+ * off_b = L_0 + ... + L_{b-1} of a [total_rows, heads, D] tensor
+ * (total_rows = sum of L).  Every hia_tensor passed with such a descriptor
+ * addresses row s of sample b at ptr + (off_b + s) * stride_s (stride_b is
+ * ignored), lse is fp32 [Hq, total_rows], and the RoPE tables stay
+ * [B, S, D] with S = max L.  There are no padded query rows: nothing is
+ * computed, read or written past a sample's L.  Errors as hia_segments_build
+ * (S >= 2^24 or total_rows >= 2^31 refused). */
+int hia_segments_build_packed(const hia_sample* samples, int B, hia_segments** out);
+
 /* Copy the per-sample bounds, tile tables and work lists to the current
  * device (allocated once per object; asynchronous on `stream`).  Must
  * precede hia_rope2d_tables / hia_attn_fwd / hia_attn_bwd. */
@@ -129,6 +143,11 @@ int hia_segments_info(const hia_segments* seg, hia_segments_info_t* info);
  * from e, for a bit-exact comparison with the reference rule.  classes:
  * uint8 [B, fwd_q_tiles, fwd_kv_tiles] with HIA_TILE_* values. */
 int hia_segments_row_bound(const hia_segments* seg, int32_t* row_bound);
+/* Per-sample layout, int32 [B] each: rows = the sample's rows in a tensor of
+ * this layout (S padded, L packed) and offsets = its first row (0 padded,
+ * L_0 + ... + L_{b-1} packed).  The packed offsets are what a caller uses to
+ * cut its packed tensors per sample. */
+int hia_segments_layout(const hia_segments* seg, int32_t* rows, int32_t* offsets);
 int hia_segments_mask(const hia_segments* seg, uint8_t* mask);
 int hia_segments_tile_classes(const hia_segments* seg, uint8_t* classes);
 

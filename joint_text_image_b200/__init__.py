@@ -16,7 +16,8 @@ __all__ = [
     "HiaError", "Segments", "lib", "hia_segments_build", "hia_rope2d_tables", "hia_attn_fwd",
     "hia_attn_bwd", "hia_attn_fwd_workspace_bytes", "hia_attn_bwd_workspace_bytes",
     "hia_get_device_status", "hia_debug_wait_timeout", "hia_profile_begin", "hia_profile_end",
-    "Step", "hia_step_create", "hia_attn_step_host", "LIB_PATH", "EXPORTED_SYMBOLS",
+    "Step", "hia_step_create", "hia_attn_step_host", "hia_segments_build_packed", "LIB_PATH",
+    "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libjointattn.so")
@@ -27,7 +28,8 @@ EXPORTED_SYMBOLS = (
     "hia_attn_fwd_workspace_bytes", "hia_attn_fwd", "hia_attn_bwd_workspace_bytes", "hia_attn_bwd",
     "hia_get_device_status", "hia_debug_wait_timeout", "hia_status_string", "hia_profile_begin",
     "hia_profile_end", "hia_attn_fwd_noalloc", "hia_debug_exp2", "hia_step_create", "hia_step_destroy",
-    "hia_attn_step_host", "hia_attn_fwd_ex", "hia_attn_bwd_ex",
+    "hia_attn_step_host", "hia_attn_fwd_ex", "hia_attn_bwd_ex", "hia_segments_build_packed",
+    "hia_segments_layout",
 )
 
 
@@ -52,7 +54,8 @@ class SegmentsInfo(ctypes.Structure):
                 ("fwd_q_tiles", ctypes.c_int32), ("fwd_kv_tiles", ctypes.c_int32),
                 ("fwd_tiles_full", ctypes.c_int64), ("fwd_tiles_partial", ctypes.c_int64),
                 ("fwd_tiles_skipped", ctypes.c_int64), ("bwd_q_tiles", ctypes.c_int32),
-                ("bwd_kv_tiles", ctypes.c_int32)]
+                ("bwd_kv_tiles", ctypes.c_int32), ("packed", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("total_rows", ctypes.c_int64)]
 
 
 class _QkNorm(ctypes.Structure):
@@ -76,11 +79,13 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         P, I, Z, T = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, _Tensor
         L.hia_segments_build.argtypes = [ctypes.POINTER(_Sample), I, I, ctypes.POINTER(P)]
+        L.hia_segments_build_packed.argtypes = [ctypes.POINTER(_Sample), I, ctypes.POINTER(P)]
         L.hia_segments_upload.argtypes = [P, P]
         L.hia_segments_destroy.argtypes = [P]
         L.hia_segments_destroy.restype = None
         L.hia_segments_info.argtypes = [P, ctypes.POINTER(SegmentsInfo)]
         L.hia_segments_row_bound.argtypes = [P, P]
+        L.hia_segments_layout.argtypes = [P, P, P]
         L.hia_segments_mask.argtypes = [P, P]
         L.hia_segments_tile_classes.argtypes = [P, P]
         L.hia_rope2d_tables.argtypes = [P, I, ctypes.c_double, P, P, P]
@@ -130,13 +135,21 @@ def _stream(device=None):
 class Segments:
     """Owner of a library hia_segments object (host tables + device copies)."""
 
-    def __init__(self, samples, S):
+    def __init__(self, samples, S, packed=False):
         arr = (_Sample * max(1, len(samples)))(*[_Sample(*map(int, s)) for s in samples])
         h = ctypes.c_void_p()
-        _check(lib().hia_segments_build(arr, len(samples), int(S), ctypes.byref(h)), "hia_segments_build")
+        if packed:
+            _check(lib().hia_segments_build_packed(arr, len(samples), ctypes.byref(h)), "hia_segments_build_packed")
+        else:
+            _check(lib().hia_segments_build(arr, len(samples), int(S), ctypes.byref(h)), "hia_segments_build")
         self.handle = h
         self.samples = [tuple(map(int, s)) for s in samples]
-        self.B, self.S = len(samples), int(S)
+        inf = self.info()
+        self.B, self.S = len(samples), int(inf.S)
+        self.packed = bool(inf.packed)
+        self.total_rows = int(inf.total_rows)
+        self.lengths = [p + hh * ww + sf for (p, hh, ww, sf) in self.samples]
+        self.rows, self.offsets = self.layout()
         self.on_device = False
 
     def upload(self):
@@ -148,6 +161,16 @@ class Segments:
         out = SegmentsInfo()
         _check(lib().hia_segments_info(self.handle, ctypes.byref(out)), "hia_segments_info")
         return out
+
+    def layout(self):
+        """(rows, offsets) per sample, from the library: a sample's rows in a
+        tensor of this layout and its first row."""
+        import numpy as np
+        r = np.zeros(max(self.B, 1), dtype=np.int32)
+        o = np.zeros(max(self.B, 1), dtype=np.int32)
+        _check(lib().hia_segments_layout(self.handle, r.ctypes.data_as(ctypes.c_void_p),
+                                         o.ctypes.data_as(ctypes.c_void_p)), "hia_segments_layout")
+        return [int(x) for x in r[:self.B]], [int(x) for x in o[:self.B]]
 
     def row_bound(self):
         import numpy as np
@@ -179,6 +202,18 @@ def hia_segments_build(samples, S, upload=True) -> Segments:
     """Segment descriptor for samples [(prefix, img_h, img_w, suffix)] padded to S."""
     seg = Segments(samples, S)
     return seg.upload() if upload else seg
+
+
+def hia_segments_build_packed(samples, upload=True) -> Segments:
+    """Segment descriptor for the packed (varlen) layout: samples back to back,
+    tensors [total_rows, heads, D], lse [Hq, total_rows]."""
+    seg = Segments(samples, 0, packed=True)
+    return seg.upload() if upload else seg
+
+
+def _view(seg, x):
+    """A packed [T,H,D] (or grouped [T,Hkv,g,D]) tensor as one batch row."""
+    return x.unsqueeze(0) if (x is not None and seg.packed) else x
 
 
 def _t(x, q_heads, g):
@@ -251,14 +286,18 @@ def hia_attn_fwd(seg: Segments, q, k, v, cos, sin, scale=None, o=None, lse=None,
     optional (wq, wk, eps), fp32 [D] CUDA weights of the per-head RMSNorm
     applied after RoPE (hia_attn_fwd_ex)."""
     import torch
-    Hq, Hkv, D = _heads(q), _heads(k), q.shape[-1]
+    Hq, Hkv, D = _heads(_view(seg, q)), _heads(_view(seg, k)), q.shape[-1]
     g = Hq // Hkv
     if scale is None:
         scale = D ** -0.5
     if o is None:
-        o = torch.empty(seg.B, seg.S, Hq, D, device=q.device, dtype=torch.bfloat16)
+        shape = (seg.total_rows, Hq, D) if seg.packed else (seg.B, seg.S, Hq, D)
+        o = torch.empty(shape, device=q.device, dtype=torch.bfloat16)
     if lse is None:
-        lse = torch.empty(seg.B, Hq, seg.S, device=q.device, dtype=torch.float32)
+        shape = (Hq, seg.total_rows) if seg.packed else (seg.B, Hq, seg.S)
+        lse = torch.empty(shape, device=q.device, dtype=torch.float32)
+    o_ret = o
+    q, k, v, o = (_view(seg, x) for x in (q, k, v, o))
     nb = hia_attn_fwd_workspace_bytes(seg, Hq, Hkv, D)
     ws = _ws(nb, workspace)
     if qk_norm is None:
@@ -270,7 +309,7 @@ def hia_attn_fwd(seg: Segments, q, k, v, cos, sin, scale=None, o=None, lse=None,
                                      cos.data_ptr(), sin.data_ptr(), float(scale), _norm(qk_norm, D),
                                      _t(o, True, g), lse.data_ptr(), ws.data_ptr(), nb, _stream()),
                "hia_attn_fwd_ex")
-    return o, lse
+    return o_ret, lse
 
 
 def hia_attn_bwd(seg: Segments, q, k, v, cos, sin, o, lse, dout, scale=None, dq=None, dk=None, dv=None,
@@ -279,16 +318,19 @@ def hia_attn_bwd(seg: Segments, q, k, v, cos, sin, o, lse, dout, scale=None, dq=
     forward's (wq, wk, eps)) returns (dq, dk, dv, dwq, dwk), dwq/dwk fp32 [D]
     (hia_attn_bwd_ex)."""
     import torch
-    Hq, Hkv, D = _heads(q), _heads(k), q.shape[-1]
+    Hq, Hkv, D = _heads(_view(seg, q)), _heads(_view(seg, k)), q.shape[-1]
     g = Hq // Hkv
     if scale is None:
         scale = D ** -0.5
+    lead = (seg.total_rows,) if seg.packed else (seg.B, seg.S)
     if dq is None:
-        dq = torch.empty(seg.B, seg.S, Hq, D, device=q.device, dtype=torch.bfloat16)
+        dq = torch.empty(*lead, Hq, D, device=q.device, dtype=torch.bfloat16)
     if dk is None:
-        dk = torch.empty(seg.B, seg.S, Hkv, D, device=q.device, dtype=torch.bfloat16)
+        dk = torch.empty(*lead, Hkv, D, device=q.device, dtype=torch.bfloat16)
     if dv is None:
-        dv = torch.empty(seg.B, seg.S, Hkv, D, device=q.device, dtype=torch.bfloat16)
+        dv = torch.empty(*lead, Hkv, D, device=q.device, dtype=torch.bfloat16)
+    ret = (dq, dk, dv)
+    q, k, v, o, dout, dq, dk, dv = (_view(seg, x) for x in (q, k, v, o, dout, dq, dk, dv))
     nb = hia_attn_bwd_workspace_bytes(seg, Hq, Hkv, D)
     ws = _ws(nb, workspace)
     if qk_norm is None:
@@ -296,7 +338,7 @@ def hia_attn_bwd(seg: Segments, q, k, v, cos, sin, o, lse, dout, scale=None, dq=
                                   cos.data_ptr(), sin.data_ptr(), float(scale), _t(o, True, g), lse.data_ptr(),
                                   _t(dout, True, g), _t(dq, True, g), _t(dk, False, 1), _t(dv, False, 1),
                                   ws.data_ptr(), nb, _stream()), "hia_attn_bwd")
-        return dq, dk, dv
+        return ret
     dwq = torch.empty(D, device=q.device, dtype=torch.float32)
     dwk = torch.empty(D, device=q.device, dtype=torch.float32)
     _check(lib().hia_attn_bwd_ex(seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1),
@@ -304,7 +346,7 @@ def hia_attn_bwd(seg: Segments, q, k, v, cos, sin, o, lse, dout, scale=None, dq=
                                  lse.data_ptr(), _t(dout, True, g), _t(dq, True, g), _t(dk, False, 1),
                                  _t(dv, False, 1), dwq.data_ptr(), dwk.data_ptr(), ws.data_ptr(), nb, _stream()),
            "hia_attn_bwd_ex")
-    return dq, dk, dv, dwq, dwk
+    return (*ret, dwq, dwk)
 
 
 class Step:

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <initializer_list>
 #include <cstring>
 #include <mutex>
 
@@ -75,10 +76,17 @@ bool make_ws_map(CUtensorMap* m, const void* base, int D, int S, int BH, uint32_
   return make_map(m, base, 3, dims, st, box);
 }
 
-// User tensor with Hkv heads: dims (D, Hkv, S, B), box rows along S.
+// Batch stride of a map: a packed tensor is one batch of total_rows rows (its
+// stride_b is 0, so the map gets the extent of the whole tensor instead).
+uint64_t batch_stride_bytes(const hia_tensor& t, int S, int B) {
+  return (B == 1 && t.stride_b == 0) ? uint64_t(S) * uint64_t(t.stride_s) * 2 : uint64_t(t.stride_b) * 2;
+}
+
+// User tensor with Hkv heads: dims (D, Hkv, S, B), box rows along S.  A packed
+// tensor is mapped with S = total_rows and B = 1.
 bool make_kv_map(CUtensorMap* m, const hia_tensor& t, int D, int Hkv, int S, int B, uint32_t rows) {
   uint64_t dims[4] = {uint64_t(D), uint64_t(Hkv), uint64_t(S), uint64_t(B)};
-  uint64_t st[3] = {uint64_t(t.stride_hkv) * 2, uint64_t(t.stride_s) * 2, uint64_t(t.stride_b) * 2};
+  uint64_t st[3] = {uint64_t(t.stride_hkv) * 2, uint64_t(t.stride_s) * 2, batch_stride_bytes(t, S, B)};
   uint32_t box[4] = {64, 1, rows, 1};
   return make_map(m, t.ptr, 4, dims, st, box);
 }
@@ -87,7 +95,7 @@ bool make_kv_map(CUtensorMap* m, const hia_tensor& t, int D, int Hkv, int S, int
 bool make_q_map(CUtensorMap* m, const hia_tensor& t, int D, int g, int Hkv, int S, int B, uint32_t rows) {
   uint64_t dims[5] = {uint64_t(D), uint64_t(g), uint64_t(Hkv), uint64_t(S), uint64_t(B)};
   uint64_t st[4] = {uint64_t(t.stride_hq) * 2, uint64_t(t.stride_hkv) * 2, uint64_t(t.stride_s) * 2,
-                    uint64_t(t.stride_b) * 2};
+                    batch_stride_bytes(t, S, B)};
   uint32_t box[5] = {64, 1, 1, rows, 1};
   return make_map(m, t.ptr, 5, dims, st, box);
 }
@@ -166,6 +174,7 @@ int check_norm(const hia_qk_norm* n) {
 void rotate_into(const hia_tensor& src, int H, int g, const float* c, const float* s, __nv_bfloat16* dst,
                  const hia_segments* seg, int D, cudaStream_t st, const float* w = nullptr, float eps = 0.f) {
   hia::RotateArgs a{};
+  a.samples = seg->d_samples;
   a.w = w;
   a.eps = eps;
   a.src = src.ptr;
@@ -182,6 +191,17 @@ void rotate_into(const hia_tensor& src, int H, int g, const float* c, const floa
   a.H = H;
   hia::launch_rope_rotate(a, D, st);
 }
+
+// Packed layout: row s of sample b is at (off_b + s) * stride_s; the batch
+// stride is not used.
+void packed_view(const hia_segments* g, std::initializer_list<hia_tensor*> ts) {
+  if (!g->packed) return;
+  for (hia_tensor* t : ts) t->stride_b = 0;
+}
+
+// The tensor maps' sequence extent and batch count.
+int map_rows(const hia_segments* g) { return g->packed ? int(g->total_rows) : g->S; }
+int map_batches(const hia_segments* g) { return g->packed ? 1 : g->B; }
 
 }  // namespace
 
@@ -269,6 +289,7 @@ extern "C" int hia_attn_fwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
       (rc = check_tensor(v, false, g->B, g->S, 1)) || (rc = check_tensor(o, true, g->B, g->S, gq)))
     return rc;
   if (!q.ptr || !k.ptr || !v.ptr || !o.ptr || !lse || !ws) return HIA_ERR_INVALID_ARG;
+  packed_view(g, {&q, &k, &v, &o});
   const FwdWs w = fwd_ws(g, Hq, Hkv, D);
   if (ws_bytes < w.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return HIA_ERR_INVALID_ARG;
   int* status = status_ptr();
@@ -280,7 +301,7 @@ extern "C" int hia_attn_fwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
 
   CUtensorMap tq, tk, tv;
   if (!make_ws_map(&tq, qr, D, g->S, g->B * Hq) || !make_ws_map(&tk, kr, D, g->S, g->B * Hkv) ||
-      !make_kv_map(&tv, v, D, Hkv, g->S, g->B, 128))
+      !make_kv_map(&tv, v, D, Hkv, map_rows(g), map_batches(g), 128))
     return HIA_ERR_CUDA;
 
   rotate_into(q, Hq, gq, c, s, qr, g, D, st, norm ? norm->wq : nullptr, norm ? norm->eps : 0.f);
@@ -303,6 +324,9 @@ extern "C" int hia_attn_fwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
   p.o_shkv = o.stride_hkv;
   p.o_shq = o.stride_hq;
   p.lse = lse;
+  p.lse_sb = g->packed ? 0 : int64_t(Hq) * g->S;
+  p.lse_sh = g->packed ? g->total_rows : g->S;
+  p.packed = g->packed ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = status;
   p.timeout_ns = kDefaultTimeoutNs;
@@ -364,6 +388,7 @@ extern "C" int hia_attn_bwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
     return rc;
   if (!q.ptr || !k.ptr || !v.ptr || !o.ptr || !lse || !dout.ptr || !dq.ptr || !dk.ptr || !dv.ptr || !ws)
     return HIA_ERR_INVALID_ARG;
+  packed_view(g, {&q, &k, &v, &o, &dout, &dq, &dk, &dv});
   const BwdWs w = bwd_ws(g, Hq, Hkv, D);
   if (ws_bytes < w.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return HIA_ERR_INVALID_ARG;
   int* status = status_ptr();
@@ -381,7 +406,8 @@ extern "C" int hia_attn_bwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
 
   CUtensorMap tq, tk, tv, tdo;
   if (!make_ws_map(&tq, qr, D, g->S, g->B * Hq, 64) || !make_ws_map(&tk, kr, D, g->S, g->B * Hkv, 128) ||
-      !make_kv_map(&tv, v, D, Hkv, g->S, g->B, 128) || !make_q_map(&tdo, dout, D, gq, Hkv, g->S, g->B, 64))
+      !make_kv_map(&tv, v, D, Hkv, map_rows(g), map_batches(g), 128) ||
+      !make_q_map(&tdo, dout, D, gq, Hkv, map_rows(g), map_batches(g), 64))
     return HIA_ERR_CUDA;
 
   rotate_into(q, Hq, gq, c, s, qr, g, D, st, norm ? norm->wq : nullptr, norm ? norm->eps : 0.f);
@@ -399,7 +425,10 @@ extern "C" int hia_attn_bwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
   pp.d_ss = dout.stride_s;
   pp.d_shkv = dout.stride_hkv;
   pp.d_shq = dout.stride_hq;
+  pp.samples = g->d_samples;
   pp.lse = lse;
+  pp.lse_sb = g->packed ? 0 : int64_t(Hq) * g->S;
+  pp.lse_sh = g->packed ? g->total_rows : g->S;
   pp.lse2 = lse2;
   pp.delta = delta;
   pp.dq_acc = dq_acc;
@@ -437,6 +466,7 @@ extern "C" int hia_attn_bwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
   p.dv_ss = dv.stride_s;
   p.dv_sh = dv.stride_hkv;
   p.dk_acc = norm ? dk_acc : nullptr;
+  p.packed = g->packed ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = status;
@@ -448,6 +478,7 @@ extern "C" int hia_attn_bwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
   // dq = R^T (norm backward of) scale * dq_acc; with the norm also dk from dk_acc and the weight gradients
   const int nblk = hia::grad_finalize_blocks(g->B, g->S);
   hia::GradFinalArgs fa{};
+  fa.samples = g->d_samples;
   fa.acc = dq_acc;
   fa.S_pad = S_pad;
   fa.scale = scale;

@@ -112,9 +112,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = p.work[2 * bid], kt = p.work[2 * bid + 1];
   const int qt_first = p.tiles[2 * (b * p.bKT + kt)];
   const int qt_full = p.tiles[2 * (b * p.bKT + kt) + 1];
-  const int n_qt = p.bQT - qt_first;
-  const int n_it = n_qt * p.g;  // iteration i: head hkv*g + i / n_qt, query tile qt_first + i % n_qt
   const SampleDev smp = p.samples[b];
+  // query tiles [qt_first, ceil(rows / 64)): ceil(S / 64) = bQT for the padded layout
+  const int n_qt = max((smp.rows + BQ - 1) / BQ - qt_first, 0);
+  const int n_it = n_qt * p.g;  // iteration i: head hkv*g + i / n_qt, query tile qt_first + i % n_qt
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_kv, 1);
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(&sm.bar_kv, 2 * kv_bytes);
       for (int c = 0; c < D / 64; ++c) {
         tma_load_3d(&sm.k[c * BK * 64], &tm_k, &sm.bar_kv, c * 64, kt * BK, b * p.Hkv + hkv);
-        tma_load_4d(&sm.v[c * BK * 64], &tm_v, &sm.bar_kv, c * 64, hkv, kt * BK, b);
+        tma_load_4d(&sm.v[c * BK * 64], &tm_v, &sm.bar_kv, c * 64, hkv, smp.off + kt * BK, p.packed ? 0 : b);
       }
       int issued = 0;
       for (int i = 0; i < n_it; ++i) {
@@ -169,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&sm.bar_full[s], 2 * qd_bytes + 2 * BQ * 4);
         for (int c = 0; c < D / 64; ++c) {
           tma_load_3d(&sm.q[s][c * BQ * 64], &tm_q, &sm.bar_full[s], c * 64, qt * BQ, b * p.Hq + h);
-          tma_load_5d(&sm.dout[s][c * BQ * 64], &tm_do, &sm.bar_full[s], c * 64, hi, hkv, qt * BQ, b);
+          tma_load_5d(&sm.dout[s][c * BQ * 64], &tm_do, &sm.bar_full[s], c * 64, hi, hkv, smp.off + qt * BQ,
+                      p.packed ? 0 : b);
         }
         const int64_t row = (int64_t(b) * p.Hq + h) * p.S_pad + int64_t(qt) * BQ;
         bulk_load(sm.lse2[s], p.lse2 + row, BQ * 4, &sm.bar_full[s]);
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = bf; i < n_it; i += 2) {
       const int s = i % kStages;
       const int qt = qt_first + i % n_qt;
-      const bool partial = qt < qt_full || (qt + 1) * BQ > p.S;
+      const bool partial = qt < qt_full || (qt + 1) * BQ > smp.rows;
       // the stage's lse2/delta were written by TMA: acquire them through its barrier
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_full[s], (i / kStages) & 1, wc) &&
                                        mbar_wait(&sm.bar_s_full[bf], (i >> 1) & 1, wc));
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q0 = qt * BQ;
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if (key > row_bound(smp.I0, smp.I1, smp.L, q0 + c) || q0 + c >= p.S) pv[c] = 0.f;
+          if (key > row_bound(smp.I0, smp.I1, smp.L, q0 + c) || q0 + c >= smp.rows) pv[c] = 0.f;
       }
       uint32_t pk[32];
 #pragma unroll
@@ -307,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool have = n_it > 0 && ok;
     if (have) have = __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, wc));
     if (have) tc_fence_after();
-    const bool store = key < p.S;
+    const bool store = key < smp.rows;
     if (bf == 0 && p.dk_acc) {
       // QK RMSNorm: the norm's backward needs the whole row, so write
       // scale * dK_n (gradient w.r.t. the normed rotated key row) in fp32 and
@@ -332,10 +334,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else if (bf == 0) {
-      const int kc = store ? key : p.S - 1;
+      const int kc = store ? key : 0;  // read only when storing
       const float* cp = p.cos_t + (int64_t(b) * p.S + kc) * D;
       const float* sp = p.sin_t + (int64_t(b) * p.S + kc) * D;
-      __nv_bfloat16* dkrow = p.dk + int64_t(b) * p.dk_sb + int64_t(key) * p.dk_ss + int64_t(hkv) * p.dk_sh;
+      __nv_bfloat16* dkrow = p.dk + int64_t(b) * p.dk_sb + int64_t(smp.off + key) * p.dk_ss + int64_t(hkv) * p.dk_sh;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t lo[32], hi[32];
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else {
-      __nv_bfloat16* dvrow = p.dv + int64_t(b) * p.dv_sb + int64_t(key) * p.dv_ss + int64_t(hkv) * p.dv_sh;
+      __nv_bfloat16* dvrow = p.dv + int64_t(b) * p.dv_sb + int64_t(smp.off + key) * p.dv_ss + int64_t(hkv) * p.dv_sh;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -455,19 +457,20 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreParams p) {
   if (warp >= p.B * p.S_pad) return;
   const int b = warp / p.S_pad, q = warp % p.S_pad;
   const int per = p.D / 32;  // elements per lane: 4 (D=128) or 2 (D=64)
+  const SampleDev t = p.samples[b];
   for (int h = 0; h < p.Hq; ++h) {
     const int64_t orow = (int64_t(b) * p.Hq + h) * p.S_pad + q;
-    if (q >= p.S) {
+    if (q >= t.rows) {  // beyond the sample's rows (padding past S, or past L when packed)
       if (lane == 0) {
         p.delta[orow] = 0.f;
         p.lse2[orow] = INFINITY;
       }
       continue;
     }
-    const __nv_bfloat16* o = p.o + int64_t(b) * p.o_sb + int64_t(q) * p.o_ss + int64_t(h / p.g) * p.o_shkv +
+    const __nv_bfloat16* o = p.o + int64_t(b) * p.o_sb + int64_t(t.off + q) * p.o_ss + int64_t(h / p.g) * p.o_shkv +
                              int64_t(h % p.g) * p.o_shq;
-    const __nv_bfloat16* d = p.dout + int64_t(b) * p.d_sb + int64_t(q) * p.d_ss + int64_t(h / p.g) * p.d_shkv +
-                             int64_t(h % p.g) * p.d_shq;
+    const __nv_bfloat16* d = p.dout + int64_t(b) * p.d_sb + int64_t(t.off + q) * p.d_ss +
+                             int64_t(h / p.g) * p.d_shkv + int64_t(h % p.g) * p.d_shq;
     float acc = 0.f;
     if (per == 4) {
       const uint2 ov = *reinterpret_cast<const uint2*>(o + lane * 4);
@@ -489,7 +492,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreParams p) {
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) {
       p.delta[orow] = acc;
-      p.lse2[orow] = p.lse[(int64_t(b) * p.Hq + h) * p.S + q] * 1.4426950408889634f;
+      p.lse2[orow] = p.lse[int64_t(b) * p.lse_sb + int64_t(h) * p.lse_sh + t.off + q] * 1.4426950408889634f;
     }
   }
 }

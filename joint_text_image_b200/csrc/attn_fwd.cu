@@ -79,6 +79,22 @@ __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint64_t vdes
   mma_chain_ts<8>(tO, tP, 8u, vdesc, st.v, idesc, accumulate ? 1u : 0u);
 }
 
+// P = exp2(S * scale*log2e - m) for one row of 128 scores, packed to bf16
+// pairs, with the row sum.  kFma: kFmaExpPairs of every 16 column pairs take
+// exp2 on the FMA pipe, the rest on MUFU.
+template <bool kFma>
+__device__ __forceinline__ void exp_pack(const uint32_t (&sr)[128], float2 cs2, float2 nm2, uint32_t (&pk)[64],
+                                         float2 (&ls)[2]) {
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), cs2, nm2);
+    const float2 pv = (kFma && (c & 15) < kFmaExpPairs) ? exp2_fma2(x)
+                                                        : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    ls[c & 1] = __fadd2_rn(ls[c & 1], pv);
+    pk[c] = pack_bf16x2(pv.x, pv.y);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -153,7 +169,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= kVStages && !mbar_wait(&sm.bar_v_empty[vs], ((j / kVStages) - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(&sm.bar_v_full[vs], tile_bytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(&sm.v[vs][c * 128 * 64], &tm_v, &sm.bar_v_full[vs], c * 64, hkv, j * 128, b);
+          tma_load_4d(&sm.v[vs][c * 128 * 64], &tm_v, &sm.bar_v_full[vs], c * 64, hkv, smp.off + j * 128,
+                      p.packed ? 0 : b);
         viss = j + 1;
       }
       // Drain: the copies this CTA issued must land before its shared memory
@@ -276,14 +293,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pk[64];
       float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       const float2 cs2 = make_float2(cs, cs), nm2 = make_float2(-m, -m);
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), cs2, nm2);
-        // kFmaExpPairs of every 16 column pairs take exp2 on the FMA pipe, the rest on MUFU
-        const float2 pv = (c & 15) < kFmaExpPairs ? exp2_fma2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
-        ls[c & 1] = __fadd2_rn(ls[c & 1], pv);
-        pk[c] = pack_bf16x2(pv.x, pv.y);
-      }
+      // FULL tiles have no masked entry: part of their exponentials run on the
+      // FMA pipe.  PARTIAL tiles use MUFU only, whose ex2(-inf) is exactly 0,
+      // so a masked key adds nothing (exp2_fma2 bottoms out at 2^-125).
+      if (j < n_full)
+        exp_pack<true>(sr, cs2, nm2, pk, ls);
+      else
+        exp_pack<false>(sr, cs2, nm2, pk, ls);
       l += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
@@ -296,8 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool have = n_vis > 0 && ok;
       if (have) have = __all_sync(0xffffffffu, mbar_wait(&sm.bar_o_final[t], 0, wc));
       if (have) tc_fence_after();
-      const bool store = q < p.S;
-      __nv_bfloat16* orow = p.o + int64_t(b) * p.o_sb + int64_t(q) * p.o_ss + int64_t(h / p.g) * p.o_shkv +
+      const bool store = q < smp.rows;
+      __nv_bfloat16* orow = p.o + int64_t(b) * p.o_sb + int64_t(smp.off + q) * p.o_ss + int64_t(h / p.g) * p.o_shkv +
                             int64_t(h % p.g) * p.o_shq;
       const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
@@ -321,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (store)
-        p.lse[(int64_t(b) * p.Hq + h) * p.S + q] =
+        p.lse[int64_t(b) * p.lse_sb + int64_t(h) * p.lse_sh + smp.off + q] =
             (have && l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }

@@ -68,6 +68,7 @@ extern "C" int hia_step_create(const hia_segments* seg, int Hq, int Hkv, int D, 
                                hia_step** out) {
   if (!seg || !out || Hq <= 0 || Hkv <= 0 || !(rope_base > 0)) return HIA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0 || (D != 64 && D != 128)) return HIA_ERR_UNSUPPORTED;
+  if (seg->packed) return HIA_ERR_UNSUPPORTED;  // the step's buffers use the padded layout
   if (!seg->dbuf) return HIA_ERR_NOT_ON_DEVICE;
   *out = nullptr;
   hia_step* st = new hia_step;

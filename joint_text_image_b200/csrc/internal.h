@@ -21,9 +21,13 @@ constexpr int kBwdBK = 128;
 constexpr int kBwdBQ = 64;
 
 // Per-sample bounds on the device: I0 = image start, I1 = image end,
-// L = valid length, w = image width (unused by the attention kernels).
+// L = valid length, w = image width (unused by the attention kernels),
+// rows = the sample's rows in the caller's tensors (S for the padded layout,
+// L for the packed one), off = the sample's first row in a packed tensor
+// (0 for the padded layout).  Row s of sample b sits at
+// b * stride_b + (off + s) * stride_s; a packed layout has stride_b = 0.
 struct SampleDev {
-  int32_t I0, I1, L, w;
+  int32_t I0, I1, L, w, rows, off;
 };
 
 // Row bound e(q): the last visible key of query q (keys k <= e(q) visible).
@@ -37,6 +41,8 @@ HIA_HD inline int32_t row_bound(int32_t I0, int32_t I1, int32_t L, int32_t q) {
 
 struct hia_segments {
   int B = 0, S = 0;
+  bool packed = false;      // samples stored back to back (no padding rows); S = max L
+  int64_t total_rows = 0;   // packed: sum of L; padded: B * S
   std::vector<hia::SampleDev> samples;
   // forward tile table [B][nQT]: (n_full, n_visible) over 128-key tiles.
   int nQT = 0, nKT = 0;

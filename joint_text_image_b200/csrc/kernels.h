@@ -9,6 +9,7 @@
 namespace hia {
 
 struct RotateArgs {
+  const SampleDev* samples;  // rows / off of every sample (layout of src)
   const void* src;  // bf16 [B,S,heads,D] with strides (elements)
   int64_t src_sb, src_ss, src_shkv, src_shq;
   int g;            // heads per stride_hkv group (1 for k)
@@ -21,6 +22,7 @@ struct RotateArgs {
 };
 
 struct GradFinalArgs {
+  const SampleDev* samples;  // rows / off of every sample (layout of x and dst)
   const float* acc;  // fp32 [B][H][S_pad][D]: gradient w.r.t. the attention's input rows (times 1/scale)
   int S_pad;
   float scale;
@@ -44,7 +46,9 @@ struct FwdParams {
   int B, S, Hq, Hkv, g, nQT, n_hp;
   __nv_bfloat16* o;
   int64_t o_sb, o_ss, o_shkv, o_shq;
-  float* lse;
+  float* lse;        // element b * lse_sb + h * lse_sh + off + q
+  int64_t lse_sb, lse_sh;
+  int packed;        // 1: V is a packed tensor map (row = off + s, batch coordinate 0)
   float scale_log2;  // softmax scale * log2(e)
   int* status;
   uint64_t timeout_ns;
@@ -55,7 +59,9 @@ struct BwdPreParams {
   int64_t o_sb, o_ss, o_shkv, o_shq;
   const __nv_bfloat16* dout;
   int64_t d_sb, d_ss, d_shkv, d_shq;
-  const float* lse;     // [B][Hq][S]
+  const SampleDev* samples;
+  const float* lse;     // element b * lse_sb + h * lse_sh + off + q
+  int64_t lse_sb, lse_sh;
   float* lse2;          // [B][Hq][S_pad]: lse * log2(e); +inf beyond S
   float* delta;         // [B][Hq][S_pad]: rowsum(dout * o); 0 beyond S
   float* dq_acc;        // [B][Hq][S_pad][D] zeroed
@@ -75,6 +81,7 @@ struct BwdParams {
   __nv_bfloat16* dk;
   int64_t dk_sb, dk_ss, dk_sh;
   float* dk_acc;      // non-null (QK RMSNorm): write scale * dK_n rows fp32 [B][Hkv][S_pad][D] here instead of dk
+  int packed;         // 1: V and dO are packed tensor maps (row = off + s, batch coordinate 0)
   __nv_bfloat16* dv;
   int64_t dv_sb, dv_ss, dv_sh;
   float scale;        // softmax scale

@@ -104,6 +104,15 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(RotateArgs a) {
   if (warp >= a.B * a.S) return;
   const int b = warp / a.S, s = warp % a.S;
   const RowLanes<D> L(lane);
+  const SampleDev t = a.samples[b];
+  if (s >= t.rows) {  // packed layout: the sample has no row s; keep the slab finite
+    for (int h = L.hs; h < a.H; h += RowLanes<D>::HPI) {
+      __nv_bfloat16* dst = a.dst + ((int64_t(b) * a.H + h) * a.S + s) * D;
+      *reinterpret_cast<uint4*>(dst + L.c * 8) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(dst + D / 2 + L.c * 8) = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
   float cs[8], sn[8], wl[8], wh[8];
   load8(a.cos_t + (int64_t(b) * a.S + s) * D + L.c * 8, cs);
   load8(a.sin_t + (int64_t(b) * a.S + s) * D + L.c * 8, sn);
@@ -113,7 +122,7 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(RotateArgs a) {
     load8(a.w + D / 2 + L.c * 8, wh);
   }
   for (int h = L.hs; h < a.H; h += RowLanes<D>::HPI) {
-    const int64_t so = int64_t(b) * a.src_sb + int64_t(s) * a.src_ss + int64_t(h / a.g) * a.src_shkv +
+    const int64_t so = int64_t(b) * a.src_sb + int64_t(t.off + s) * a.src_ss + int64_t(h / a.g) * a.src_shkv +
                        int64_t(h % a.g) * a.src_shq;
     const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(a.src) + so;
     float l[8], u[8], xl[8], xu[8];
@@ -159,8 +168,9 @@ __global__ void __launch_bounds__(256) grad_finalize_kernel(GradFinalArgs a) {
   float dwl[8], dwh[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) dwl[k] = dwh[k] = 0.f;
-  if (warp < a.B * a.S) {
-    const int b = warp / a.S, s = warp % a.S;
+  const int b = warp / max(a.S, 1), s = warp % max(a.S, 1);
+  if (warp < a.B * a.S && s < a.samples[b].rows) {
+    const int off = a.samples[b].off;
     float cs[8], sn[8], wl[8], wh[8];
     load8(a.cos_t + (int64_t(b) * a.S + s) * D + L.c * 8, cs);
     load8(a.sin_t + (int64_t(b) * a.S + s) * D + L.c * 8, sn);
@@ -181,7 +191,7 @@ __global__ void __launch_bounds__(256) grad_finalize_kernel(GradFinalArgs a) {
         vu[k] *= a.scale;
       }
       if (norm) {
-        const int64_t xo = int64_t(b) * a.x_sb + int64_t(s) * a.x_ss + int64_t(h / a.g) * a.x_shkv +
+        const int64_t xo = int64_t(b) * a.x_sb + int64_t(off + s) * a.x_ss + int64_t(h / a.g) * a.x_shkv +
                            int64_t(h % a.g) * a.x_shq;
         const __nv_bfloat16* xin = reinterpret_cast<const __nv_bfloat16*>(a.x) + xo;
         float l[8], u[8], xl[8], xu[8];
@@ -219,7 +229,7 @@ __global__ void __launch_bounds__(256) grad_finalize_kernel(GradFinalArgs a) {
         ol[k] = fmaf(vl[k], cs[k], vu[k] * sn[k]);   // (R^T v)_j
         ou[k] = fmaf(vu[k], cs[k], -vl[k] * sn[k]);  // (R^T v)_{j+D/2}
       }
-      const int64_t so = int64_t(b) * a.dst_sb + int64_t(s) * a.dst_ss + int64_t(h / a.g) * a.dst_shkv +
+      const int64_t so = int64_t(b) * a.dst_sb + int64_t(off + s) * a.dst_ss + int64_t(h / a.g) * a.dst_shkv +
                          int64_t(h % a.g) * a.dst_shq;
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.dst) + so;
       *reinterpret_cast<uint4*>(dst + L.c * 8) = pack8_bf16(ol);

@@ -20,15 +20,19 @@ using hia::row_bound;
 
 static int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-extern "C" int hia_segments_build(const hia_sample* s, int B, int S, hia_segments** out) {
-  if (!out || B < 0 || S < 0 || (B > 0 && !s)) return HIA_ERR_INVALID_ARG;
-  *out = nullptr;
-  if (S >= (1 << 24) || B >= (1 << 20)) return HIA_ERR_INVALID_ARG;
+// Shared by the padded and the packed layouts.  A sample's query and key
+// rows are [0, rows) with rows = S (padded: rows >= L are padding) or L
+// (packed: the next sample follows at once); every loop over rows below stops
+// at rows, so a packed descriptor has no padded query rows and no work on
+// them.
+static int build(const hia_sample* s, int B, int S, bool packed, hia_segments** out) {
   hia_segments* g = new (std::nothrow) hia_segments();
   if (!g) return HIA_ERR_INVALID_ARG;
   g->B = B;
   g->S = S;
+  g->packed = packed;
   g->samples.resize(B);
+  int64_t off = 0;
   for (int b = 0; b < B; ++b) {
     const hia_sample& x = s[b];
     if (x.prefix_len < 0 || x.img_h < 0 || x.img_w < 0 || x.suffix_len < 0 || ((x.img_h == 0) != (x.img_w == 0))) {
@@ -41,14 +45,23 @@ extern "C" int hia_segments_build(const hia_sample* s, int B, int S, hia_segment
       delete g;
       return HIA_ERR_INVALID_ARG;
     }
-    g->samples[b] = {x.prefix_len, int32_t(x.prefix_len + n), int32_t(L), x.img_w};
+    const int32_t rows = packed ? int32_t(L) : S;
+    // the padded layout addresses sample b through stride_b: its first row is row 0
+    g->samples[b] = {x.prefix_len, int32_t(x.prefix_len + n), int32_t(L), x.img_w, rows,
+                     packed ? int32_t(off) : 0};
+    off += rows;
   }
+  if (off >= (int64_t(1) << 31)) {
+    delete g;
+    return HIA_ERR_INVALID_ARG;
+  }
+  g->total_rows = off;
 
-  // visible pairs: sum over real query rows of e(q) + 1
+  // visible pairs: sum over the sample's query rows of e(q) + 1
   int64_t pairs = 0;
   for (int b = 0; b < B; ++b) {
     const auto& t = g->samples[b];
-    for (int q = 0; q < S; ++q) pairs += row_bound(t.I0, t.I1, t.L, q) + 1;
+    for (int q = 0; q < t.rows; ++q) pairs += row_bound(t.I0, t.I1, t.L, q) + 1;
   }
   g->pairs = pairs;
 
@@ -62,7 +75,11 @@ extern "C" int hia_segments_build(const hia_sample* s, int B, int S, hia_segment
   for (int b = 0; b < B; ++b) {
     const auto& t = g->samples[b];
     for (int qt = 0; qt < g->nQT; ++qt) {
-      int q0 = qt * kFwdBM, q1 = std::min(q0 + kFwdBM, S) - 1;
+      int q0 = qt * kFwdBM, q1 = std::min(q0 + kFwdBM, int(t.rows)) - 1;
+      if (q0 >= t.rows) {  // packed: no rows here
+        nskip += g->nKT;
+        continue;
+      }
       int e0 = row_bound(t.I0, t.I1, t.L, q0), e1 = row_bound(t.I0, t.I1, t.L, q1);
       int n_vis = e1 < 0 ? 0 : ceil_div(e1 + 1, kFwdBN);
       int n_full = e0 < 0 ? 0 : (e0 + 1) / kFwdBN;
@@ -85,8 +102,9 @@ extern "C" int hia_segments_build(const hia_sample* s, int B, int S, hia_segment
   }
 
   // backward tiles: 128 keys x 64 query rows.  For kv tile kt the visited
-  // query tiles are [qt_first, bQT) (a suffix, by monotone e); those from
-  // qt_full on are FULL (all rows < S and e(first row) >= last key).
+  // query tiles are [qt_first, ceil(rows / 64)) (a suffix, by monotone e);
+  // those from qt_full on are FULL (all rows < rows and e(first row) >= last
+  // key).
   using hia::kBwdBK;
   using hia::kBwdBQ;
   g->bQT = ceil_div(S, kBwdBQ);
@@ -95,15 +113,16 @@ extern "C" int hia_segments_build(const hia_sample* s, int B, int S, hia_segment
   std::vector<int64_t> bwd_cost(size_t(B) * g->bKT, 0);
   for (int b = 0; b < B; ++b) {
     const auto& t = g->samples[b];
+    const int R = t.rows, nq = ceil_div(R, kBwdBQ);
     int first = 0, full = 0;  // non-decreasing in kt: two pointers
     for (int kt = 0; kt < g->bKT; ++kt) {
       int k0 = kt * kBwdBK, k1 = k0 + kBwdBK - 1;
-      while (first < g->bQT && row_bound(t.I0, t.I1, t.L, std::min((first + 1) * kBwdBQ, S) - 1) < k0) ++first;
-      while (full < g->bQT && !((full + 1) * kBwdBQ <= S && row_bound(t.I0, t.I1, t.L, full * kBwdBQ) >= k1)) ++full;
+      while (first < nq && row_bound(t.I0, t.I1, t.L, std::min((first + 1) * kBwdBQ, R) - 1) < k0) ++first;
+      while (full < nq && !((full + 1) * kBwdBQ <= R && row_bound(t.I0, t.I1, t.L, full * kBwdBQ) >= k1)) ++full;
       int f = std::max(full, first);
       g->bwd_tiles[(size_t(b) * g->bKT + kt) * 2 + 0] = first;
       g->bwd_tiles[(size_t(b) * g->bKT + kt) * 2 + 1] = f;
-      bwd_cost[size_t(b) * g->bKT + kt] = g->bQT - first;
+      bwd_cost[size_t(b) * g->bKT + kt] = nq - first;
     }
   }
   order.assign(size_t(B) * g->bKT, 0);
@@ -126,13 +145,51 @@ extern "C" int hia_segments_build(const hia_sample* s, int B, int S, hia_segment
   in.fwd_tiles_skipped = nskip;
   in.bwd_q_tiles = g->bQT;
   in.bwd_kv_tiles = g->bKT;
+  in.packed = packed ? 1 : 0;
+  in.total_rows = g->total_rows;
   *out = g;
   return HIA_OK;
+}
+
+static int check_args(const hia_sample* s, int B, hia_segments** out) {
+  if (!out || B < 0 || (B > 0 && !s)) return HIA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (B >= (1 << 20)) return HIA_ERR_INVALID_ARG;
+  return HIA_OK;
+}
+
+extern "C" int hia_segments_build(const hia_sample* s, int B, int S, hia_segments** out) {
+  int rc = check_args(s, B, out);
+  if (rc) return rc;
+  if (S < 0 || S >= (1 << 24)) return HIA_ERR_INVALID_ARG;
+  return build(s, B, S, false, out);
+}
+
+extern "C" int hia_segments_build_packed(const hia_sample* s, int B, hia_segments** out) {
+  int rc = check_args(s, B, out);
+  if (rc) return rc;
+  int64_t S = 0;
+  for (int b = 0; b < B; ++b) {
+    const hia_sample& x = s[b];
+    if (x.prefix_len < 0 || x.img_h < 0 || x.img_w < 0 || x.suffix_len < 0) return HIA_ERR_INVALID_ARG;
+    S = std::max(S, int64_t(x.prefix_len) + int64_t(x.img_h) * x.img_w + x.suffix_len);
+  }
+  if (S >= (1 << 24)) return HIA_ERR_INVALID_ARG;
+  return build(s, B, int(S), true, out);
 }
 
 extern "C" int hia_segments_info(const hia_segments* g, hia_segments_info_t* info) {
   if (!g || !info) return HIA_ERR_INVALID_ARG;
   *info = g->info;
+  return HIA_OK;
+}
+
+extern "C" int hia_segments_layout(const hia_segments* g, int32_t* rows, int32_t* offsets) {
+  if (!g || (g->B > 0 && (!rows || !offsets))) return HIA_ERR_INVALID_ARG;
+  for (int b = 0; b < g->B; ++b) {
+    rows[b] = g->samples[b].rows;
+    offsets[b] = g->samples[b].off;
+  }
   return HIA_OK;
 }
 
