@@ -40,21 +40,43 @@ def _load():
         P = ctypes.c_void_p
         I = ctypes.c_int
         D = ctypes.c_double
-        lib.oracle_mask.argtypes = [I, I, P, P, P, P, P]
-        lib.oracle_positions.argtypes = [I, I, P, P, P, P, P, P]
-        lib.oracle_rope_tables.argtypes = [I, I, I, P, P, P, P, D, P, P]
-        lib.oracle_rope_apply.argtypes = [I, I, I, I, P, P, P, P, D, I, P, P]
-        lib.oracle_attn_fwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, D, D, I, P, I, P, P, P, D, P, P, I]
-        lib.oracle_attn_bwd.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, D, D, I, P, I, P, P, P, D,
+        G = [P, P, P, P, P]  # flat geometry: n_img, text_before, img_h, img_w, suffix
+        lib.oracle_mask.argtypes = [I, I, *G, P]
+        lib.oracle_positions.argtypes = [I, I, *G, P, P]
+        lib.oracle_rope_tables.argtypes = [I, I, I, *G, D, P, P]
+        lib.oracle_rope_apply.argtypes = [I, I, I, I, *G, D, I, P, P]
+        lib.oracle_attn_fwd.argtypes = [I, I, I, I, I, *G, P, P, P, D, D, I, P, I, P, P, P, D, P, P, I]
+        lib.oracle_attn_bwd.argtypes = [I, I, I, I, I, *G, P, P, P, P, D, D, I, P, I, P, P, P, D,
                                         P, P, P, P, P, I]
         _lib = lib
     return _lib
 
 
 def _geom(samples):
-    """samples: list of (prefix, img_h, img_w, suffix) -> four int32 arrays."""
-    a = np.asarray(samples, dtype=np.int32).reshape(-1, 4)
-    return [np.ascontiguousarray(a[:, i]) for i in range(4)]
+    """Flat geometry (oracle.c, ogeom) from samples given either as
+    (prefix, img_h, img_w, suffix) -- one image, or text only when h = w = 0 --
+    or as (images, suffix) with images a list of (text_before, img_h, img_w):
+    returns the int32 arrays n_img, text_before, img_h, img_w, suffix."""
+    n_img, tb, hh, ww, suf = [], [], [], [], []
+    for smp in samples:
+        if len(smp) == 2:
+            images, suffix = smp
+        else:
+            p, h, w, sfx = smp
+            if min(p, h, w, sfx) < 0 or (h == 0) != (w == 0):
+                images, suffix = [(-1, 0, 0)], -1  # bad geometry: refused by the C side
+            elif h == 0:
+                images, suffix = [], p + sfx
+            else:
+                images, suffix = [(p, h, w)], sfx
+        n_img.append(len(images))
+        for (t, h, w) in images:
+            tb.append(t)
+            hh.append(h)
+            ww.append(w)
+        suf.append(suffix)
+    arr = lambda x: np.ascontiguousarray(np.asarray(x if x else [0], dtype=np.int32))
+    return [arr(n_img), arr(tb), arr(hh), arr(ww), arr(suf)]
 
 
 def _p(a):
@@ -64,8 +86,8 @@ def _p(a):
 def mask(samples, S: int) -> np.ndarray:
     """uint8 [B, S, S] indexed [b, query, key] from the literal rule."""
     g = _geom(samples)
-    out = np.zeros((len(g[0]), S, S), dtype=np.uint8)
-    if _load().oracle_mask(len(g[0]), S, *map(_p, g), _p(out)) != 0:
+    out = np.zeros((len(samples), S, S), dtype=np.uint8)
+    if _load().oracle_mask(len(samples), S, *map(_p, g), _p(out)) != 0:
         raise ValueError("bad sample geometry")
     return out
 
@@ -73,7 +95,7 @@ def mask(samples, S: int) -> np.ndarray:
 def positions(samples, S: int):
     """(x, y) int64 [B, S] 2D RoPE positions."""
     g = _geom(samples)
-    B = len(g[0])
+    B = len(samples)
     x = np.zeros((B, S), dtype=np.int64)
     y = np.zeros((B, S), dtype=np.int64)
     if _load().oracle_positions(B, S, *map(_p, g), _p(x), _p(y)) != 0:
@@ -84,7 +106,7 @@ def positions(samples, S: int):
 def rope_tables(samples, S: int, D: int, base: float = 10000.0):
     """(cos, sin) fp64 [B, S, D]."""
     g = _geom(samples)
-    B = len(g[0])
+    B = len(samples)
     c = np.zeros((B, S, D))
     s = np.zeros((B, S, D))
     if _load().oracle_rope_tables(B, S, D, *map(_p, g), float(base), _p(c), _p(s)) != 0:

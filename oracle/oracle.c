@@ -58,37 +58,80 @@
 /* Sample geometry                                                          */
 /* ------------------------------------------------------------------------ */
 
-/* One sample: prefix P (text incl. <timestep>), image h x w, suffix s.
- * I0 = P, I1 = P + h*w, L = I1 + s.  Padding is [L, S). */
+/* One sample: text and images in order, then suffix text.  Image i spans
+ * [I0_i, I1_i) (I1_i = I0_i + h_i * w_i, row-major, width w_i); L is the
+ * sample's length; padding is [L, S).  The single-image layout of the Cache
+ * Contract is prefix P, one image, suffix s: I0 = P, I1 = P + h*w,
+ * L = I1 + s. */
+#define OMAX_IMG 64
 typedef struct {
-    int64_t I0, I1, L, w;
+    int64_t I0, I1, w;
+} oimage;
+typedef struct {
+    int64_t L;
+    int n;
+    oimage img[OMAX_IMG];
 } osample;
 
-static osample make_sample(int32_t prefix, int32_t h, int32_t w, int32_t suffix) {
-    osample s;
-    s.I0 = prefix;
-    s.I1 = (int64_t)prefix + (int64_t)h * (int64_t)w;
-    s.L = s.I1 + suffix;
-    s.w = w;
-    return s;
-}
+/* Flat batch geometry: sample b holds n_img[b] images, entries
+ * first_b .. first_b + n_img[b] - 1 of text_before / img_h / img_w (first_b
+ * the running sum of n_img); image j is preceded by text_before[j] text
+ * tokens; after the last image come suffix[b] text tokens. */
+typedef struct {
+    int B;
+    const int32_t *n_img, *text_before, *img_h, *img_w, *suffix;
+} ogeom;
 
-/* The literal mask rule (build_joint_attention_mask; 3.1.2; 3.3):
- *   key k visible from query q  <=>  k < L  and  ( k <= q  or
- *                                   (I0 <= q < I1 and I0 <= k < I1) ). */
-static int visible(const osample* s, int64_t q, int64_t k) {
-    if (k >= s->L) return 0;
-    if (k <= q) return 1;
-    if (s->I0 <= q && q < s->I1 && s->I0 <= k && k < s->I1) return 1;
+static int make_sample(const ogeom* g, int b, osample* s) {
+    int64_t first = 0;
+    for (int i = 0; i < b; ++i) first += g->n_img[i];
+    int n = g->n_img[b];
+    if (n < 0 || n > OMAX_IMG || g->suffix[b] < 0) return -1;
+    int64_t pos = 0;
+    s->n = n;
+    for (int j = 0; j < n; ++j) {
+        int64_t t = g->text_before[first + j], h = g->img_h[first + j], w = g->img_w[first + j];
+        if (t < 0 || h <= 0 || w <= 0) return -1;
+        s->img[j].I0 = pos + t;
+        s->img[j].I1 = s->img[j].I0 + h * w;
+        s->img[j].w = w;
+        pos = s->img[j].I1;
+    }
+    s->L = pos + g->suffix[b];
     return 0;
 }
 
+static int image_of(const osample* s, int64_t n) {
+    for (int j = 0; j < s->n; ++j)
+        if (s->img[j].I0 <= n && n < s->img[j].I1) return j;
+    return -1;
+}
+
+/* The literal mask rule (build_joint_attention_mask; 3.1.2; 3.3), with the
+ * multi-image rule of 3.1.2 (images in context are masked from subsequent
+ * tokens; read here as: every image but the sample's last is hidden from all
+ * tokens after its span, the last image follows the one-image rule):
+ *   key k visible from query q  <=>  k < L  and  ( q, k in the same image  or
+ *                                   ( k <= q  and  k not in a context image ) ),
+ * a context image being one of images 0 .. n-2 (any k <= q outside q's own
+ * image lies before q's image, so it is hidden exactly when its image is a
+ * context image). */
+static int visible(const osample* s, int64_t q, int64_t k) {
+    if (k >= s->L) return 0;
+    int iq = image_of(s, q), ik = image_of(s, k);
+    if (iq >= 0 && iq == ik) return 1;
+    if (k > q) return 0;
+    if (ik >= 0 && ik < s->n - 1) return 0;
+    return 1;
+}
+
 /* mask: uint8 [B, S, S] indexed [b, q, k]. */
-int oracle_mask(int B, int S, const int32_t* prefix, const int32_t* img_h,
+int oracle_mask(int B, int S, const int32_t* n_img, const int32_t* text_before, const int32_t* img_h,
                 const int32_t* img_w, const int32_t* suffix, uint8_t* mask) {
+    ogeom g = {B, n_img, text_before, img_h, img_w, suffix};
+    osample s;
     for (int b = 0; b < B; ++b) {
-        osample s = make_sample(prefix[b], img_h[b], img_w[b], suffix[b]);
-        if (s.L > S) return -1;
+        if (make_sample(&g, b, &s) || s.L > S) return -1;
         for (int64_t q = 0; q < S; ++q)
             for (int64_t k = 0; k < S; ++k)
                 mask[((int64_t)b * S + q) * S + k] = (uint8_t)visible(&s, q, k);
@@ -100,13 +143,17 @@ int oracle_mask(int B, int S, const int32_t* prefix, const int32_t* img_h,
 /* Generalized 2D RoPE (3.4 of the paper review)                             */
 /* ------------------------------------------------------------------------ */
 
-/* 2D position (x, y) of token n of sample s. */
+/* 2D position (x, y) of token n of sample s: a token of image j at row r,
+ * column c of its grid sits at (I0_j + c, I0_j + r); any other token at
+ * (n, n).  (With several images the pages also shift the positions after a
+ * generated image, 3.1.3, by an amount they do not give: not modelled.) */
 static void position(const osample* s, int64_t n, double* x, double* y) {
-    if (s->I0 <= n && n < s->I1) {
-        int64_t i = n - s->I0;
-        int64_t r = i / s->w, c = i % s->w;
-        *x = (double)(s->I0 + c);
-        *y = (double)(s->I0 + r);
+    int j = image_of(s, n);
+    if (j >= 0) {
+        int64_t i = n - s->img[j].I0;
+        int64_t r = i / s->img[j].w, c = i % s->img[j].w;
+        *x = (double)(s->img[j].I0 + c);
+        *y = (double)(s->img[j].I0 + r);
     } else {
         *x = (double)n;
         *y = (double)n;
@@ -122,11 +169,12 @@ static double angle(const osample* s, int64_t n, int j, int D, double base) {
 }
 
 /* positions: int64 [B, S] x and y. */
-int oracle_positions(int B, int S, const int32_t* prefix, const int32_t* img_h,
+int oracle_positions(int B, int S, const int32_t* n_img, const int32_t* text_before, const int32_t* img_h,
                      const int32_t* img_w, const int32_t* suffix, int64_t* xs, int64_t* ys) {
+    ogeom g = {B, n_img, text_before, img_h, img_w, suffix};
+    osample s;
     for (int b = 0; b < B; ++b) {
-        osample s = make_sample(prefix[b], img_h[b], img_w[b], suffix[b]);
-        if (s.L > S) return -1;
+        if (make_sample(&g, b, &s) || s.L > S) return -1;
         for (int64_t n = 0; n < S; ++n) {
             double x, y;
             position(&s, n, &x, &y);
@@ -138,13 +186,14 @@ int oracle_positions(int B, int S, const int32_t* prefix, const int32_t* img_h,
 }
 
 /* cos, sin fp64 [B, S, D]: entry j and j + D/2 both hold angle_j. */
-int oracle_rope_tables(int B, int S, int D, const int32_t* prefix, const int32_t* img_h,
-                       const int32_t* img_w, const int32_t* suffix, double base,
+int oracle_rope_tables(int B, int S, int D, const int32_t* n_img, const int32_t* text_before,
+                       const int32_t* img_h, const int32_t* img_w, const int32_t* suffix, double base,
                        double* cos_t, double* sin_t) {
     if (D % 2) return -1;
+    ogeom g = {B, n_img, text_before, img_h, img_w, suffix};
+    osample s;
     for (int b = 0; b < B; ++b) {
-        osample s = make_sample(prefix[b], img_h[b], img_w[b], suffix[b]);
-        if (s.L > S) return -1;
+        if (make_sample(&g, b, &s) || s.L > S) return -1;
         for (int64_t n = 0; n < S; ++n)
             for (int j = 0; j < D / 2; ++j) {
                 double a = angle(&s, n, j, D, base);
@@ -183,13 +232,14 @@ static void rotate_t(const osample* s, int64_t n, int D, double base, const doub
 }
 
 /* Apply R (inverse = 0) or R^T (inverse = 1) to x [B, S, H, D] in place of y. */
-int oracle_rope_apply(int B, int S, int H, int D, const int32_t* prefix, const int32_t* img_h,
-                      const int32_t* img_w, const int32_t* suffix, double base, int inverse,
-                      const double* x, double* y) {
+int oracle_rope_apply(int B, int S, int H, int D, const int32_t* n_img, const int32_t* text_before,
+                      const int32_t* img_h, const int32_t* img_w, const int32_t* suffix, double base,
+                      int inverse, const double* x, double* y) {
     if (D % 2) return -1;
+    ogeom g = {B, n_img, text_before, img_h, img_w, suffix};
+    osample s;
     for (int b = 0; b < B; ++b) {
-        osample s = make_sample(prefix[b], img_h[b], img_w[b], suffix[b]);
-        if (s.L > S) return -1;
+        if (make_sample(&g, b, &s) || s.L > S) return -1;
         for (int64_t n = 0; n < S; ++n)
             for (int h = 0; h < H; ++h) {
                 int64_t o = (((int64_t)b * S + n) * H + h) * D;
@@ -206,7 +256,7 @@ int oracle_rope_apply(int B, int S, int H, int D, const int32_t* prefix, const i
 
 typedef struct {
     int B, S, Hq, Hkv, D;
-    const int32_t *prefix, *img_h, *img_w, *suffix;
+    const osample* samples;     /* [B], built from the flat geometry */
     const double *q, *k, *v, *dout;
     double scale, base;
     int rotate_inputs;          /* 1: apply R to q, k here; 0: inputs already rotated */
@@ -252,10 +302,10 @@ static void rms_norm_vjp(const double* x, const double* w, int D, double r, cons
 
 /* Rotated copy of head h of tensor x [B,S,H,D] for sample b: out [S, D]. */
 static void gather_head(const job_t* J, const double* x, int H, int b, int h, int rot, double* out) {
-    osample s = make_sample(J->prefix[b], J->img_h[b], J->img_w[b], J->suffix[b]);
+    const osample* sp = &J->samples[b];
     for (int64_t n = 0; n < J->S; ++n) {
         const double* src = x + (((int64_t)b * J->S + n) * H + h) * J->D;
-        if (rot) rotate(&s, n, J->D, J->base, src, out + n * J->D);
+        if (rot) rotate(sp, n, J->D, J->base, src, out + n * J->D);
         else memcpy(out + n * J->D, src, sizeof(double) * J->D);
     }
 }
@@ -264,7 +314,7 @@ static void gather_head(const job_t* J, const double* x, int H, int b, int h, in
  * of exp(scaled score)). */
 static void fwd_task(job_t* J, int b, int h) {
     const int S = J->S, D = J->D, g = J->Hq / J->Hkv;
-    osample s = make_sample(J->prefix[b], J->img_h[b], J->img_w[b], J->suffix[b]);
+    const osample* sp = &J->samples[b];
     double* qr = malloc(sizeof(double) * (size_t)S * D);
     double* kr = malloc(sizeof(double) * (size_t)S * D);
     double* vv = malloc(sizeof(double) * (size_t)S * D);
@@ -282,7 +332,7 @@ static void fwd_task(job_t* J, int b, int h) {
         int64_t q = J->rows ? J->rows[ri] : ri;
         double m = -INFINITY;
         for (int64_t k = 0; k < S; ++k) {
-            sc[k] = visible(&s, q, k) ? J->scale * dot(qr + q * D, kr + k * D, D) : -INFINITY;
+            sc[k] = visible(sp, q, k) ? J->scale * dot(qr + q * D, kr + k * D, D) : -INFINITY;
             if (sc[k] > m) m = sc[k];
         }
         double* orow = J->o + (((int64_t)b * S + q) * J->Hq + h) * D;
@@ -312,7 +362,7 @@ static void fwd_task(job_t* J, int b, int h) {
  * gradients of this head go to dwq_h / dwk_h. */
 static void bwd_task(job_t* J, int b, int h) {
     const int S = J->S, D = J->D, g = J->Hq / J->Hkv;
-    osample s = make_sample(J->prefix[b], J->img_h[b], J->img_w[b], J->suffix[b]);
+    const osample* sp = &J->samples[b];
     size_t SD = (size_t)S * D;
     double* qr = malloc(sizeof(double) * SD);
     double* kr = malloc(sizeof(double) * SD);
@@ -350,7 +400,7 @@ static void bwd_task(job_t* J, int b, int h) {
         double* dqout = J->dq + (((int64_t)b * S + q) * J->Hq + h) * D;
         double m = -INFINITY;
         for (int64_t k = 0; k < S; ++k) {
-            sc[k] = visible(&s, q, k) ? J->scale * dot(qr + q * D, kr + k * D, D) : -INFINITY;
+            sc[k] = visible(sp, q, k) ? J->scale * dot(qr + q * D, kr + k * D, D) : -INFINITY;
             if (sc[k] > m) m = sc[k];
         }
         if (m == -INFINITY) { for (int d = 0; d < D; ++d) dqout[d] = 0.0; continue; }
@@ -380,7 +430,7 @@ static void bwd_task(job_t* J, int b, int h) {
             rms_norm_vjp(qx + q * D, J->wq, D, rq[q], dqr, gx, dwq);
             memcpy(dqr, gx, sizeof(double) * D);
         }
-        if (J->rotate_inputs) rotate_t(&s, q, D, J->base, dqr, dqout);
+        if (J->rotate_inputs) rotate_t(sp, q, D, J->base, dqr, dqout);
         else memcpy(dqout, dqr, sizeof(double) * D);
     }
     for (int64_t k = 0; k < S; ++k) {
@@ -390,7 +440,7 @@ static void bwd_task(job_t* J, int b, int h) {
             rms_norm_vjp(kx + k * D, J->wk, D, rk[k], dkr + k * D, gx, dwk);
             memcpy(dkr + k * D, gx, sizeof(double) * D);
         }
-        if (J->rotate_inputs) rotate_t(&s, k, D, J->base, dkr + k * D, dko);
+        if (J->rotate_inputs) rotate_t(sp, k, D, J->base, dkr + k * D, dko);
         else memcpy(dko, dkr + k * D, sizeof(double) * D);
         memcpy(dvo, dvv + k * D, sizeof(double) * D);
     }
@@ -436,14 +486,12 @@ static int run_job(job_t* J, int is_bwd, int nthreads) {
     return nthreads;
 }
 
-static int check_geom(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
-                      const int32_t* img_h, const int32_t* img_w, const int32_t* suffix) {
-    if (B < 0 || S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || D % 2) return -1;
-    for (int b = 0; b < B; ++b) {
-        if (prefix[b] < 0 || img_h[b] < 0 || img_w[b] < 0 || suffix[b] < 0) return -1;
-        if ((img_h[b] == 0) != (img_w[b] == 0)) return -1;
-        if (make_sample(prefix[b], img_h[b], img_w[b], suffix[b]).L > S) return -1;
-    }
+/* Builds J->samples from the flat geometry; -1 on bad geometry. */
+static int load_geom(job_t* J, osample* buf, const ogeom* g, int S, int Hq, int Hkv, int D) {
+    if (g->B < 0 || S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || D % 2) return -1;
+    for (int b = 0; b < g->B; ++b)
+        if (make_sample(g, b, &buf[b]) || buf[b].L > S) return -1;
+    J->samples = buf;
     return 0;
 }
 
@@ -452,23 +500,26 @@ static int check_geom(int B, int S, int Hq, int Hkv, int D, const int32_t* prefi
  * group_sel [B*Hkv] restricts the (b, kv head) groups; wq, wk [D] (both or
  * neither) turn on the QK RMSNorm with epsilon eps.  Returns the number of
  * threads used, or -1 on bad arguments. */
-int oracle_attn_fwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
+int oracle_attn_fwd(int B, int S, int Hq, int Hkv, int D, const int32_t* n_img, const int32_t* text_before,
                     const int32_t* img_h, const int32_t* img_w, const int32_t* suffix,
                     const double* q, const double* k, const double* v, double scale,
                     double base, int rotate_inputs, const int32_t* rows, int n_rows,
                     const uint8_t* group_sel, const double* wq, const double* wk, double eps,
                     double* o, double* lse, int nthreads) {
-    if (check_geom(B, S, Hq, Hkv, D, prefix, img_h, img_w, suffix)) return -1;
     if ((wq == NULL) != (wk == NULL) || (wq && !(eps >= 0.0))) return -1;
     job_t J;
     memset(&J, 0, sizeof(J));
+    ogeom g = {B, n_img, text_before, img_h, img_w, suffix};
+    osample* smp = malloc(sizeof(osample) * (B > 0 ? B : 1));
+    if (load_geom(&J, smp, &g, S, Hq, Hkv, D)) { free(smp); return -1; }
     J.B = B; J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.D = D;
-    J.prefix = prefix; J.img_h = img_h; J.img_w = img_w; J.suffix = suffix;
     J.q = q; J.k = k; J.v = v; J.scale = scale; J.base = base;
     J.rotate_inputs = rotate_inputs; J.rows = rows; J.n_rows = n_rows;
     J.group_sel = group_sel; J.o = o; J.lse = lse;
     J.wq = wq; J.wk = wk; J.eps = eps;
-    return run_job(&J, 0, nthreads);
+    int used = run_job(&J, 0, nthreads);
+    free(smp);
+    return used;
 }
 
 /* Backward.  dq [B,S,Hq,D]; dk, dv [B,S,Hkv,D].  group_sel as above (dq of
@@ -477,19 +528,20 @@ int oracle_attn_fwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
  * the contributions of those rows only (a partial sum over queries).  With
  * the QK RMSNorm (wq, wk non-NULL) dwq, dwk [D] receive the weight
  * gradients, summed over the selected groups and rows. */
-int oracle_attn_bwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
+int oracle_attn_bwd(int B, int S, int Hq, int Hkv, int D, const int32_t* n_img, const int32_t* text_before,
                     const int32_t* img_h, const int32_t* img_w, const int32_t* suffix,
                     const double* q, const double* k, const double* v, const double* dout,
                     double scale, double base, int rotate_inputs, const int32_t* rows, int n_rows,
                     const uint8_t* group_sel, const double* wq, const double* wk, double eps,
                     double* dq, double* dk, double* dv, double* dwq, double* dwk, int nthreads) {
-    if (check_geom(B, S, Hq, Hkv, D, prefix, img_h, img_w, suffix)) return -1;
     if ((wq == NULL) != (wk == NULL) || (wq && (!(eps >= 0.0) || !dwq || !dwk))) return -1;
     size_t n = (size_t)B * S * Hq * D;
     job_t J;
     memset(&J, 0, sizeof(J));
+    ogeom geom = {B, n_img, text_before, img_h, img_w, suffix};
+    osample* smp = malloc(sizeof(osample) * (B > 0 ? B : 1));
+    if (load_geom(&J, smp, &geom, S, Hq, Hkv, D)) { free(smp); return -1; }
     J.B = B; J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.D = D;
-    J.prefix = prefix; J.img_h = img_h; J.img_w = img_w; J.suffix = suffix;
     J.q = q; J.k = k; J.v = v; J.dout = dout; J.scale = scale; J.base = base;
     J.rotate_inputs = rotate_inputs; J.rows = rows; J.n_rows = n_rows;
     J.group_sel = group_sel; J.dq = dq;
@@ -531,5 +583,6 @@ int oracle_attn_bwd(int B, int S, int Hq, int Hkv, int D, const int32_t* prefix,
         }
     free(J.dk_h);
     free(J.dv_h);
+    free(smp);
     return used;
 }
