@@ -78,9 +78,8 @@ def oracle_sample_step(wl, q, k, v, do, rows, nthreads=0):
     _, _, _, used2 = oracle.attn_bwd(smp, qq, kk, vv, dd, wl.scale, wl.base, rows=rows, groups=groups,
                                      nthreads=nthreads)
     dt = time.perf_counter() - t0
-    P, h, w, s = smp[0]
-    I0, I1, L = P, P + h * w, P + h * w + s
-    pairs = sum(min(L - 1, I1 - 1 if I0 <= r < I1 else r) + 1 for r in rows)
+    # the sample rows' visible pairs, from the oracle's literal mask (outside the timed part)
+    pairs = int(oracle.mask(smp, q.shape[1])[0][np.asarray(rows)].sum(dtype=np.int64))
     g = wl.Hq // wl.Hkv
     flops = 14.0 * wl.D * g * pairs
     return dt, flops, min(max(used, used2), g)
@@ -194,7 +193,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--ref-row-stride", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default=WORKLOAD, choices=["tiny", "256px", "1024px", "mixed", "1024px_bwd"],
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=["tiny", "256px", "1024px", "mixed", "1024px_bwd", "multi_image"],
                     help="synthetic workload (the metric is quoted on 1024px; the others are for profiling)")
     ap.add_argument("--packed", action="store_true",
                     help="packed (varlen) layout: no padded rows (no e2e line: the host step is padded-only)")

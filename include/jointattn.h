@@ -58,6 +58,14 @@ typedef struct {
     int32_t suffix_len;
 } hia_sample;
 
+/* One image of a sample with several images: text_before text tokens, then
+ * an img_h x img_w image (row-major, img_h, img_w > 0). */
+typedef struct {
+    int32_t text_before;
+    int32_t img_h;
+    int32_t img_w;
+} hia_image;
+
 /* A strided [B, S, heads, D] bf16 (or fp32) device tensor.  Strides are in
  * elements; the last dimension is contiguous.  For a tensor with Hq heads,
  * head h lives at ptr + (h / g) * stride_hkv + (h % g) * stride_hq, which
@@ -126,6 +134,22 @@ int hia_segments_build(const hia_sample* samples, int B, int S, hia_segments** o
  * computed, read or written past a sample's L.  Errors as hia_segments_build
  * (S >= 2^24 or total_rows >= 2^31 refused). */
 int hia_segments_build_packed(const hia_sample* samples, int B, hia_segments** out);
+
+/* Samples with any number of images (technical report summary 3.1.2: in
+ * a training sequence with several generated images, an image already in
+ * context is masked from the tokens after it; positions 3.1.3).  Sample b is
+ * n_images[b] entries of `images` (consecutive, in order: each is its text
+ * then its image), then suffix_len[b] text tokens.  Reading of the pages:
+ * every image of a sample but its last is a context image, hidden from all
+ * tokens after its span; the last image follows the one-image rule, so one
+ * image per sample is exactly hia_segments_build.  Each image sits on its own
+ * 2D grid (x = I0 + column, y = I0 + row); text keeps x = y = its index (the
+ * pages also shift positions after a generated image, by an amount they do
+ * not give: not modelled).  packed != 0 builds the packed layout (S is then
+ * computed as max L and ignored).  Errors: HIA_ERR_INVALID_ARG (null
+ * arrays, negative counts or lengths, an image with h or w <= 0, L > S). */
+int hia_segments_build_multi(const hia_image* images, const int32_t* n_images, const int32_t* suffix_len,
+                             int B, int S, int packed, hia_segments** out);
 
 /* Copy the per-sample bounds, tile tables and work lists to the current
  * device (allocated once per object; asynchronous on `stream`).  Must

@@ -16,7 +16,8 @@ __all__ = [
     "HiaError", "Segments", "lib", "hia_segments_build", "hia_rope2d_tables", "hia_attn_fwd",
     "hia_attn_bwd", "hia_attn_fwd_workspace_bytes", "hia_attn_bwd_workspace_bytes",
     "hia_get_device_status", "hia_debug_wait_timeout", "hia_profile_begin", "hia_profile_end",
-    "Step", "hia_step_create", "hia_attn_step_host", "hia_segments_build_packed", "LIB_PATH",
+    "Step", "hia_step_create", "hia_attn_step_host", "hia_segments_build_packed", "hia_segments_build_multi",
+    "LIB_PATH",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -29,7 +30,7 @@ EXPORTED_SYMBOLS = (
     "hia_get_device_status", "hia_debug_wait_timeout", "hia_status_string", "hia_profile_begin",
     "hia_profile_end", "hia_attn_fwd_noalloc", "hia_debug_exp2", "hia_step_create", "hia_step_destroy",
     "hia_attn_step_host", "hia_attn_fwd_ex", "hia_attn_bwd_ex", "hia_segments_build_packed",
-    "hia_segments_layout",
+    "hia_segments_layout", "hia_segments_build_multi",
 )
 
 
@@ -62,6 +63,10 @@ class _QkNorm(ctypes.Structure):
     _fields_ = [("wq", ctypes.c_void_p), ("wk", ctypes.c_void_p), ("eps", ctypes.c_float)]
 
 
+class _Image(ctypes.Structure):
+    _fields_ = [("text_before", ctypes.c_int32), ("img_h", ctypes.c_int32), ("img_w", ctypes.c_int32)]
+
+
 class _KernelTime(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_double)]
 
@@ -80,6 +85,7 @@ def lib():
         P, I, Z, T = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, _Tensor
         L.hia_segments_build.argtypes = [ctypes.POINTER(_Sample), I, I, ctypes.POINTER(P)]
         L.hia_segments_build_packed.argtypes = [ctypes.POINTER(_Sample), I, ctypes.POINTER(P)]
+        L.hia_segments_build_multi.argtypes = [ctypes.POINTER(_Image), P, P, I, I, I, ctypes.POINTER(P)]
         L.hia_segments_upload.argtypes = [P, P]
         L.hia_segments_destroy.argtypes = [P]
         L.hia_segments_destroy.restype = None
@@ -136,19 +142,37 @@ class Segments:
     """Owner of a library hia_segments object (host tables + device copies)."""
 
     def __init__(self, samples, S, packed=False):
-        arr = (_Sample * max(1, len(samples)))(*[_Sample(*map(int, s)) for s in samples])
+        """samples: (prefix, img_h, img_w, suffix) per sample, or, for several
+        images, (images, suffix) with images a list of (text_before, h, w)."""
         h = ctypes.c_void_p()
-        if packed:
-            _check(lib().hia_segments_build_packed(arr, len(samples), ctypes.byref(h)), "hia_segments_build_packed")
+        multi = any(len(x) == 2 for x in samples)
+        if multi:
+            norm = [x if len(x) == 2 else (([(x[0], x[1], x[2])], x[3]) if x[1] * x[2] > 0 else ([], x[0] + x[3]))
+                    for x in samples]
+            imgs = [im for (ims, _) in norm for im in ims]
+            iarr = (_Image * max(1, len(imgs)))(*[_Image(*map(int, im)) for im in imgs])
+            import numpy as np
+            n_img = np.asarray([len(ims) for (ims, _) in norm] or [0], dtype=np.int32)
+            suf = np.asarray([sf for (_, sf) in norm] or [0], dtype=np.int32)
+            _check(lib().hia_segments_build_multi(iarr, n_img.ctypes.data_as(ctypes.c_void_p),
+                                                  suf.ctypes.data_as(ctypes.c_void_p), len(samples), int(S),
+                                                  int(bool(packed)), ctypes.byref(h)), "hia_segments_build_multi")
+            self.samples = [([tuple(map(int, im)) for im in ims], int(sf)) for (ims, sf) in norm]
+            self.lengths = [sum(t + hh * ww for (t, hh, ww) in ims) + sf for (ims, sf) in self.samples]
         else:
-            _check(lib().hia_segments_build(arr, len(samples), int(S), ctypes.byref(h)), "hia_segments_build")
+            arr = (_Sample * max(1, len(samples)))(*[_Sample(*map(int, x)) for x in samples])
+            if packed:
+                _check(lib().hia_segments_build_packed(arr, len(samples), ctypes.byref(h)),
+                       "hia_segments_build_packed")
+            else:
+                _check(lib().hia_segments_build(arr, len(samples), int(S), ctypes.byref(h)), "hia_segments_build")
+            self.samples = [tuple(map(int, x)) for x in samples]
+            self.lengths = [p + hh * ww + sf for (p, hh, ww, sf) in self.samples]
         self.handle = h
-        self.samples = [tuple(map(int, s)) for s in samples]
         inf = self.info()
         self.B, self.S = len(samples), int(inf.S)
         self.packed = bool(inf.packed)
         self.total_rows = int(inf.total_rows)
-        self.lengths = [p + hh * ww + sf for (p, hh, ww, sf) in self.samples]
         self.rows, self.offsets = self.layout()
         self.on_device = False
 
@@ -208,6 +232,14 @@ def hia_segments_build_packed(samples, upload=True) -> Segments:
     """Segment descriptor for the packed (varlen) layout: samples back to back,
     tensors [total_rows, heads, D], lse [Hq, total_rows]."""
     seg = Segments(samples, 0, packed=True)
+    return seg.upload() if upload else seg
+
+
+def hia_segments_build_multi(samples, S=0, packed=False, upload=True) -> Segments:
+    """Segment descriptor for samples with any number of images: each sample
+    (images, suffix), images a list of (text_before, img_h, img_w); every
+    image but a sample's last is hidden from all tokens after it."""
+    seg = Segments([x if len(x) == 2 else x for x in samples], S, packed=packed)
     return seg.upload() if upload else seg
 
 

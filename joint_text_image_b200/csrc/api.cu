@@ -211,11 +211,12 @@ extern "C" int hia_segments_upload(hia_segments* g, void* stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return HIA_ERR_CUDA;
   if (g->dbuf && g->device != dev) return HIA_ERR_INVALID_ARG;
-  const size_t n_s = g->samples.size() * sizeof(SampleDev);
-  const size_t n_ft = g->fwd_tiles.size() * 4, n_fw = g->fwd_work.size() * 4;
+  const size_t n_s = g->samples.size() * sizeof(SampleDev), n_i = g->images.size() * sizeof(hia::ImageDev);
+  const size_t n_ft = g->fwd_tiles.size() * 4, n_fl = g->fwd_list.size() * 4, n_fw = g->fwd_work.size() * 4;
   const size_t n_bt = g->bwd_tiles.size() * 4, n_bw = g->bwd_work.size() * 4;
-  const size_t o_s = 0, o_ft = align256(n_s), o_fw = o_ft + align256(n_ft), o_bt = o_fw + align256(n_fw),
-               o_bw = o_bt + align256(n_bt), total = o_bw + align256(n_bw) + 256;
+  const size_t o_s = 0, o_i = align256(n_s), o_ft = o_i + align256(n_i), o_fl = o_ft + align256(n_ft),
+               o_fw = o_fl + align256(n_fl), o_bt = o_fw + align256(n_fw), o_bw = o_bt + align256(n_bt),
+               total = o_bw + align256(n_bw) + 256;
   if (!g->dbuf) {
     if (cudaMalloc(&g->dbuf, total) != cudaSuccess) {
       g->dbuf = nullptr;
@@ -225,14 +226,18 @@ extern "C" int hia_segments_upload(hia_segments* g, void* stream) {
   char* base = static_cast<char*>(g->dbuf);
   cudaError_t e = cudaSuccess;
   if (n_s) e = cudaMemcpyAsync(base + o_s, g->samples.data(), n_s, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && n_i) e = cudaMemcpyAsync(base + o_i, g->images.data(), n_i, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess && n_ft) e = cudaMemcpyAsync(base + o_ft, g->fwd_tiles.data(), n_ft, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && n_fl) e = cudaMemcpyAsync(base + o_fl, g->fwd_list.data(), n_fl, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess && n_fw) e = cudaMemcpyAsync(base + o_fw, g->fwd_work.data(), n_fw, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess && n_bt) e = cudaMemcpyAsync(base + o_bt, g->bwd_tiles.data(), n_bt, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess && n_bw) e = cudaMemcpyAsync(base + o_bw, g->bwd_work.data(), n_bw, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return HIA_ERR_CUDA;
   g->device = dev;
   g->d_samples = reinterpret_cast<const SampleDev*>(base + o_s);
+  g->d_images = reinterpret_cast<const hia::ImageDev*>(base + o_i);
   g->d_fwd_tiles = reinterpret_cast<const int32_t*>(base + o_ft);
+  g->d_fwd_list = reinterpret_cast<const int32_t*>(base + o_fl);
   g->d_fwd_work = reinterpret_cast<const int32_t*>(base + o_fw);
   g->d_bwd_tiles = reinterpret_cast<const int32_t*>(base + o_bt);
   g->d_bwd_work = reinterpret_cast<const int32_t*>(base + o_bw);
@@ -256,7 +261,7 @@ extern "C" int hia_rope2d_tables(const hia_segments* g, int D, double base, floa
   if (g->B == 0 || g->S == 0) return HIA_OK;
   if (!c || !s) return HIA_ERR_INVALID_ARG;
   if (g->device < 0) return HIA_ERR_NOT_ON_DEVICE;
-  hia::launch_rope2d_tables(g->d_samples, g->B, g->S, D, base, c, s, static_cast<cudaStream_t>(stream));
+  hia::launch_rope2d_tables(g->d_samples, g->d_images, g->B, g->S, D, base, c, s, static_cast<cudaStream_t>(stream));
   return cuda_status(cudaGetLastError());
 }
 
@@ -309,7 +314,9 @@ extern "C" int hia_attn_fwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
 
   hia::FwdParams p{};
   p.samples = g->d_samples;
+  p.images = g->d_images;
   p.tiles = g->d_fwd_tiles;
+  p.list = g->d_fwd_list;
   p.work = g->d_fwd_work;
   p.B = g->B;
   p.S = g->S;
@@ -442,6 +449,7 @@ extern "C" int hia_attn_bwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
 
   hia::BwdParams p{};
   p.samples = g->d_samples;
+  p.images = g->d_images;
   p.tiles = g->d_bwd_tiles;
   p.work = g->d_bwd_work;
   p.B = g->B;

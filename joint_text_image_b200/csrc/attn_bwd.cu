@@ -110,11 +110,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hkv = bid % p.Hkv;
   bid /= p.Hkv;
   const int b = p.work[2 * bid], kt = p.work[2 * bid + 1];
-  const int qt_first = p.tiles[2 * (b * p.bKT + kt)];
-  const int qt_full = p.tiles[2 * (b * p.bKT + kt) + 1];
+  // the query tiles [qt_first, qt_end) see this kv tile; [full_first, full_end) see all of it
+  const int32_t* te = p.tiles + 4 * (b * p.bKT + kt);
+  const int qt_first = te[0], qt_end = te[1], full_first = te[2], full_end = te[3];
   const SampleDev smp = p.samples[b];
-  // query tiles [qt_first, ceil(rows / 64)): ceil(S / 64) = bQT for the padded layout
-  const int n_qt = max((smp.rows + BQ - 1) / BQ - qt_first, 0);
+  const int n_qt = max(qt_end - qt_first, 0);
   const int n_it = n_qt * p.g;  // iteration i: head hkv*g + i / n_qt, query tile qt_first + i % n_qt
 
   if (threadIdx.x == 0) {
@@ -241,13 +241,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int key = kt * BK + r;
+    // this key is visible exactly to the query rows [vis_lo, vis_hi)
+    const ImageDev* im = p.images + smp.img0;
+    const int vis_lo = first_row(im, smp.n_img, smp.L, key);
+    const int vis_hi = min(int(smp.rows), hidden_from(im, smp.n_img, key));
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const float cs = p.scale_log2;
     bool ok = true;
     for (int i = bf; i < n_it; i += 2) {
       const int s = i % kStages;
       const int qt = qt_first + i % n_qt;
-      const bool partial = qt < qt_full || (qt + 1) * BQ > smp.rows;
+      const bool partial = qt < full_first || qt >= full_end || (qt + 1) * BQ > smp.rows;
       // the stage's lse2/delta were written by TMA: acquire them through its barrier
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_full[s], (i / kStages) & 1, wc) &&
                                        mbar_wait(&sm.bar_s_full[bf], (i >> 1) & 1, wc));
@@ -271,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q0 = qt * BQ;
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if (key > row_bound(smp.I0, smp.I1, smp.L, q0 + c) || q0 + c >= smp.rows) pv[c] = 0.f;
+          if (q0 + c < vis_lo || q0 + c >= vis_hi) pv[c] = 0.f;
       }
       uint32_t pk[32];
 #pragma unroll

@@ -111,7 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hkv = bid % p.Hkv;
   bid /= p.Hkv;
   const int b = p.work[2 * bid], qt = p.work[2 * bid + 1];
-  const int n_full = p.tiles[2 * (b * p.nQT + qt)];
+  // the visible kv tiles of this query tile: entries kt | FULL << 16, in order
+  const int32_t* tlist = p.list + p.tiles[2 * (b * p.nQT + qt)];
   const int n_vis = p.tiles[2 * (b * p.nQT + qt) + 1];
   const int h0 = hkv * p.g + 2 * hp;
   const int n_tiles = (2 * hp + 1 < p.g) ? 2 : 1;
@@ -161,15 +162,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       int kiss = 0, viss = 0;
       for (int j = 0; j < n_vis; ++j) {
         const int ks = j % kKStages, vs = j % kVStages;
+        const int kt = __ldg(tlist + j) & 0xffff;
         if (j >= kKStages && !mbar_wait(&sm.bar_k_empty[ks], ((j / kKStages) - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(&sm.bar_k_full[ks], tile_bytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(&sm.k[ks][c * 128 * 64], &tm_k, &sm.bar_k_full[ks], c * 64, j * 128, b * p.Hkv + hkv);
+          tma_load_3d(&sm.k[ks][c * 128 * 64], &tm_k, &sm.bar_k_full[ks], c * 64, kt * 128, b * p.Hkv + hkv);
         kiss = j + 1;
         if (j >= kVStages && !mbar_wait(&sm.bar_v_empty[vs], ((j / kVStages) - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(&sm.bar_v_full[vs], tile_bytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(&sm.v[vs][c * 128 * 64], &tm_v, &sm.bar_v_full[vs], c * 64, hkv, smp.off + j * 128,
+          tma_load_4d(&sm.v[vs][c * 128 * 64], &tm_v, &sm.bar_v_full[vs], c * 64, hkv, smp.off + kt * 128,
                       p.packed ? 0 : b);
         viss = j + 1;
       }
@@ -243,7 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t tS = tmem + uint32_t(t * 128) + lane_off;
     const uint32_t tO = tmem + 256u + uint32_t(t * D) + lane_off;
-    const int e = row_bound(smp.I0, smp.I1, smp.L, q);
+    const ImageDev* im = p.images + smp.img0;
+    const int e = row_bound(im, smp.n_img, smp.L, q);
+    // context images this row no longer sees (only samples with several images)
+    int n_hidden = 0;
+    for (int i = 0; i < smp.n_img; ++i) n_hidden += (im[i].hidden && im[i].I1 <= q) ? 1 : 0;
     const float cs = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = active;
@@ -255,11 +261,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_ld_wait();
-      if (j >= n_full) {
-        const int lim = e - j * 128;  // key j*128 + c is visible iff c <= lim
+      const int32_t ent = __ldg(tlist + j);
+      const bool full = (ent >> 16) != 0;
+      if (!full) {
+        const int k0 = (ent & 0xffff) * 128;
+        const int lim = e - k0;  // key k0 + c is visible iff c <= lim and not hidden
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c > lim) sr[c] = __float_as_uint(-INFINITY);
+        for (int i = 0; n_hidden > 0 && i < smp.n_img; ++i) {
+          if (!im[i].hidden || im[i].I1 > q) continue;
+          const int lo = im[i].I0 - k0, n = im[i].I1 - im[i].I0;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (unsigned(c - lo) < unsigned(n)) sr[c] = __float_as_uint(-INFINITY);
+        }
       }
       // row max with 8 independent partial maxima (short dependency chains)
       float mp[8];
@@ -296,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // FULL tiles have no masked entry: part of their exponentials run on the
       // FMA pipe.  PARTIAL tiles use MUFU only, whose ex2(-inf) is exactly 0,
       // so a masked key adds nothing (exp2_fma2 bottoms out at 2^-125).
-      if (j < n_full)
+      if (full)
         exp_pack<true>(sr, cs2, nm2, pk, ls);
       else
         exp_pack<false>(sr, cs2, nm2, pk, ls);

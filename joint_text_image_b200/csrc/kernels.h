@@ -41,7 +41,9 @@ struct GradFinalArgs {
 
 struct FwdParams {
   const SampleDev* samples;
-  const int32_t* tiles;  // [B][nQT][2]
+  const ImageDev* images;
+  const int32_t* tiles;  // [B][nQT][2]: (first entry of list, count)
+  const int32_t* list;   // kv tile entries kt | FULL << 16
   const int32_t* work;   // [n_work][2]
   int B, S, Hq, Hkv, g, nQT, n_hp;
   __nv_bfloat16* o;
@@ -70,7 +72,8 @@ struct BwdPreParams {
 
 struct BwdParams {
   const SampleDev* samples;
-  const int32_t* tiles;  // [B][bKT][2]
+  const ImageDev* images;
+  const int32_t* tiles;  // [B][bKT][4]: (qt_first, qt_end, full_first, full_end)
   const int32_t* work;   // [n_work][2]
   int B, S, S_pad, Hq, Hkv, g, bQT, bKT;
   const float* lse2;
@@ -95,7 +98,8 @@ enum KernelId { kRopeTables = 0, kRopeRotate, kAttnFwd, kBwdPre, kAttnBwd, kGrad
 void prof_begin(KernelId id, cudaStream_t st);
 void prof_end(KernelId id, cudaStream_t st);
 
-void launch_rope2d_tables(const SampleDev* samples, int B, int S, int D, double base, float* cos_out,
+void launch_rope2d_tables(const SampleDev* samples, const ImageDev* images, int B, int S, int D, double base,
+                          float* cos_out,
                           float* sin_out, cudaStream_t st);
 void launch_rope_rotate(const RotateArgs& a, int D, cudaStream_t st);
 int grad_finalize_blocks(int B, int S);

@@ -18,8 +18,9 @@ namespace hia {
 
 // K1: one thread per (b, n, j < D/2).  Angle and cos/sin in fp64, rounded
 // once to fp32: a text-only sample reproduces the 1D tables exactly.
-__global__ void rope2d_tables_kernel(const SampleDev* __restrict__ samples, int B, int S, int D, double base,
-                                     float* __restrict__ cos_out, float* __restrict__ sin_out) {
+__global__ void rope2d_tables_kernel(const SampleDev* __restrict__ samples, const ImageDev* __restrict__ images,
+                                     int B, int S, int D, double base, float* __restrict__ cos_out,
+                                     float* __restrict__ sin_out) {
   const int half = D / 2;
   const int64_t total = int64_t(B) * S * half;
   for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
@@ -30,10 +31,12 @@ __global__ void rope2d_tables_kernel(const SampleDev* __restrict__ samples, int 
     const int b = int(bn / S);
     const SampleDev t = samples[b];
     double x = n, y = n;
-    if (n >= t.I0 && n < t.I1) {
-      const int i = n - t.I0;
-      x = double(t.I0 + i % t.w);
-      y = double(t.I0 + i / t.w);
+    const int im = image_of(images + t.img0, t.n_img, n);
+    if (im >= 0) {  // each image on its own grid, origin at its first token
+      const ImageDev g = images[t.img0 + im];
+      const int i = n - g.I0;
+      x = double(g.I0 + i % g.w);
+      y = double(g.I0 + i / g.w);
     }
     const double theta = pow(base, -2.0 * double(j) / double(D));
     const double a = ((j & 1) ? y : x) * theta;
@@ -271,15 +274,15 @@ __global__ void __launch_bounds__(1024) dw_reduce_kernel(const float* __restrict
   if (ry == 0 && d < D) dw[d] = t[0][cx];
 }
 
-void launch_rope2d_tables(const SampleDev* samples, int B, int S, int D, double base, float* cos_out,
-                          float* sin_out, cudaStream_t st) {
+void launch_rope2d_tables(const SampleDev* samples, const ImageDev* images, int B, int S, int D, double base,
+                          float* cos_out, float* sin_out, cudaStream_t st) {
   const int64_t total = int64_t(B) * S * (D / 2);
   if (total == 0) return;
   const int threads = 256;
   int64_t blocks = (total + threads - 1) / threads;
   if (blocks > 148 * 64) blocks = 148 * 64;
   prof_begin(kRopeTables, st);
-  rope2d_tables_kernel<<<int(blocks), threads, 0, st>>>(samples, B, S, D, base, cos_out, sin_out);
+  rope2d_tables_kernel<<<int(blocks), threads, 0, st>>>(samples, images, B, S, D, base, cos_out, sin_out);
   prof_end(kRopeTables, st);
 }
 

@@ -2,30 +2,49 @@
 //
 // Replaces the dense [B,1,S,S] boolean mask of build_joint_attention_mask
 // (hunyuan_image3.model: causal text, bidirectional image span, padded keys
-// masked out; technical report summary 3.1.2) by per-sample bounds and a
-// per-tile classification.  The rule "k < L and (k <= q or q, k both in the
-// image span)" equals "k <= e(q)" with the non-decreasing row bound
-// e(q) = min(L-1, q in [I0,I1) ? I1-1 : q): text rows end at themselves,
-// image rows at the image's last token, suffix rows at themselves, padded
-// rows at L-1.  Monotone e makes every row's visible set a prefix, so a
-// (q-tile, k-tile) pair is FULL when its last key is <= e(first row), skipped
-// when its first key is > e(last row), and PARTIAL otherwise.
+// masked out; technical report summary 3.1.2) by per-sample bounds and
+// per-tile work lists.  The rule "k < L and (k <= q or q, k in one image)"
+// equals "k <= e(q)" with the non-decreasing row bound
+// e(q) = min(L-1, q in an image ? the image's last token : q): text rows end
+// at themselves, image rows at their image's last token, padded rows at L-1.
+// With several images per sample, every image but the last is a context
+// image, masked from all tokens after its span (3.1.2, training sequences
+// with several generated images): k is then also hidden from q when k lies
+// in a context image that ends at or before q.  The builder counts the
+// visible pairs of every (q-tile, kv-tile) pair: FULL when all are visible,
+// skipped when none is, PARTIAL otherwise.
 #include <algorithm>
 #include <cstring>
 #include <new>
 
 #include "internal.h"
 
+using hia::ImageDev;
 using hia::row_bound;
 
 static int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// Shared by the padded and the packed layouts.  A sample's query and key
-// rows are [0, rows) with rows = S (padded: rows >= L are padding) or L
-// (packed: the next sample follows at once); every loop over rows below stops
-// at rows, so a packed descriptor has no padded query rows and no work on
-// them.
-static int build(const hia_sample* s, int B, int S, bool packed, hia_segments** out) {
+namespace {
+
+// One sample before layout: images (text before each, h, w) in order, then
+// the suffix.
+struct SampleSpec {
+  std::vector<hia_image> images;
+  int32_t suffix = 0;
+};
+
+// Visible keys of row q in [k0, k1]: [0, e(q)] minus the context images that
+// end at or before q.
+int64_t visible_in(const ImageDev* im, int n, int32_t L, int32_t q, int32_t k0, int32_t k1) {
+  const int32_t e = row_bound(im, n, L, q);
+  int64_t c = std::max<int64_t>(0, int64_t(std::min(k1, e)) - k0 + 1);
+  for (int i = 0; i < n; ++i)
+    if (im[i].hidden && im[i].I1 <= q) c -= std::max(0, std::min(k1 + 1, im[i].I1) - std::max(k0, im[i].I0));
+  return c;
+}
+
+int build(const std::vector<SampleSpec>& spec, int S, bool packed, hia_segments** out) {
+  const int B = int(spec.size());
   hia_segments* g = new (std::nothrow) hia_segments();
   if (!g) return HIA_ERR_INVALID_ARG;
   g->B = B;
@@ -34,21 +53,32 @@ static int build(const hia_sample* s, int B, int S, bool packed, hia_segments** 
   g->samples.resize(B);
   int64_t off = 0;
   for (int b = 0; b < B; ++b) {
-    const hia_sample& x = s[b];
-    if (x.prefix_len < 0 || x.img_h < 0 || x.img_w < 0 || x.suffix_len < 0 || ((x.img_h == 0) != (x.img_w == 0))) {
-      delete g;
-      return HIA_ERR_INVALID_ARG;
+    const SampleSpec& x = spec[b];
+    const int n = int(x.images.size());
+    int64_t pos = 0;
+    const int32_t img0 = int32_t(g->images.size());
+    for (int j = 0; j < n; ++j) {
+      const hia_image& im = x.images[j];
+      if (im.text_before < 0 || im.img_h <= 0 || im.img_w <= 0) {
+        delete g;
+        return HIA_ERR_INVALID_ARG;
+      }
+      const int64_t I0 = pos + im.text_before, I1 = I0 + int64_t(im.img_h) * im.img_w;
+      if (I1 > S) {
+        delete g;
+        return HIA_ERR_INVALID_ARG;
+      }
+      g->images.push_back({int32_t(I0), int32_t(I1), im.img_w, j < n - 1 ? 1 : 0});
+      pos = I1;
     }
-    int64_t n = int64_t(x.img_h) * x.img_w;
-    int64_t L = int64_t(x.prefix_len) + n + x.suffix_len;
-    if (L > S) {
+    const int64_t L = pos + x.suffix;
+    if (x.suffix < 0 || L > S) {
       delete g;
       return HIA_ERR_INVALID_ARG;
     }
     const int32_t rows = packed ? int32_t(L) : S;
     // the padded layout addresses sample b through stride_b: its first row is row 0
-    g->samples[b] = {x.prefix_len, int32_t(x.prefix_len + n), int32_t(L), x.img_w, rows,
-                     packed ? int32_t(off) : 0};
+    g->samples[b] = {int32_t(L), rows, packed ? int32_t(off) : 0, img0, n, 0};
     off += rows;
   }
   if (off >= (int64_t(1) << 31)) {
@@ -56,16 +86,17 @@ static int build(const hia_sample* s, int B, int S, bool packed, hia_segments** 
     return HIA_ERR_INVALID_ARG;
   }
   g->total_rows = off;
+  auto imgs = [&](int b) { return g->images.data() + g->samples[b].img0; };
 
-  // visible pairs: sum over the sample's query rows of e(q) + 1
+  // visible pairs: sum over the sample's query rows of its visible keys
   int64_t pairs = 0;
   for (int b = 0; b < B; ++b) {
     const auto& t = g->samples[b];
-    for (int q = 0; q < t.rows; ++q) pairs += row_bound(t.I0, t.I1, t.L, q) + 1;
+    for (int q = 0; q < t.rows; ++q) pairs += visible_in(imgs(b), t.n_img, t.L, q, 0, S - 1);
   }
   g->pairs = pairs;
 
-  // forward tiles: 128 x 128
+  // forward tiles: 128 x 128; per (b, qt) the list of visible kv tiles
   using hia::kFwdBM;
   using hia::kFwdBN;
   g->nQT = ceil_div(S, kFwdBM);
@@ -75,20 +106,21 @@ static int build(const hia_sample* s, int B, int S, bool packed, hia_segments** 
   for (int b = 0; b < B; ++b) {
     const auto& t = g->samples[b];
     for (int qt = 0; qt < g->nQT; ++qt) {
-      int q0 = qt * kFwdBM, q1 = std::min(q0 + kFwdBM, int(t.rows)) - 1;
-      if (q0 >= t.rows) {  // packed: no rows here
-        nskip += g->nKT;
-        continue;
+      const int q0 = qt * kFwdBM, q1 = std::min(q0 + kFwdBM, int(t.rows)) - 1;
+      g->fwd_tiles[(size_t(b) * g->nQT + qt) * 2 + 0] = int32_t(g->fwd_list.size());
+      int count = 0;
+      for (int kt = 0; q0 <= q1 && kt < g->nKT; ++kt) {
+        const int k0 = kt * kFwdBN, k1 = std::min(k0 + kFwdBN, S) - 1;
+        int64_t vis = 0;
+        for (int q = q0; q <= q1; ++q) vis += visible_in(imgs(b), t.n_img, t.L, q, k0, k1);
+        if (vis == 0) continue;
+        const bool full = k1 - k0 + 1 == kFwdBN && vis == int64_t(q1 - q0 + 1) * kFwdBN;
+        g->fwd_list.push_back(kt | (full ? (1 << 16) : 0));
+        ++count;
+        (full ? nfull : npart) += 1;
       }
-      int e0 = row_bound(t.I0, t.I1, t.L, q0), e1 = row_bound(t.I0, t.I1, t.L, q1);
-      int n_vis = e1 < 0 ? 0 : ceil_div(e1 + 1, kFwdBN);
-      int n_full = e0 < 0 ? 0 : (e0 + 1) / kFwdBN;
-      n_full = std::min(n_full, n_vis);
-      g->fwd_tiles[(size_t(b) * g->nQT + qt) * 2 + 0] = n_full;
-      g->fwd_tiles[(size_t(b) * g->nQT + qt) * 2 + 1] = n_vis;
-      nfull += n_full;
-      npart += n_vis - n_full;
-      nskip += g->nKT - n_vis;
+      g->fwd_tiles[(size_t(b) * g->nQT + qt) * 2 + 1] = count;
+      nskip += g->nKT - count;
     }
   }
   std::vector<int> order(size_t(B) * g->nQT);
@@ -101,28 +133,42 @@ static int build(const hia_sample* s, int B, int S, bool packed, hia_segments** 
     g->fwd_work[i * 2 + 1] = order[i] % g->nQT;
   }
 
-  // backward tiles: 128 keys x 64 query rows.  For kv tile kt the visited
-  // query tiles are [qt_first, ceil(rows / 64)) (a suffix, by monotone e);
-  // those from qt_full on are FULL (all rows < rows and e(first row) >= last
-  // key).
+  // backward tiles: 128 keys x 64 query rows.  The query tiles that see a kv
+  // tile form a range (keys in a context image are seen only by its own
+  // rows, other keys by every later row); the FULL ones (every pair visible,
+  // a whole 64-row tile) are taken as their first contiguous run, the rest of
+  // the range is PARTIAL (the mask is evaluated there).
   using hia::kBwdBK;
   using hia::kBwdBQ;
   g->bQT = ceil_div(S, kBwdBQ);
   g->bKT = ceil_div(S, kBwdBK);
-  g->bwd_tiles.assign(size_t(B) * g->bKT * 2, 0);
+  g->bwd_tiles.assign(size_t(B) * g->bKT * 4, 0);
   std::vector<int64_t> bwd_cost(size_t(B) * g->bKT, 0);
   for (int b = 0; b < B; ++b) {
     const auto& t = g->samples[b];
-    const int R = t.rows, nq = ceil_div(R, kBwdBQ);
-    int first = 0, full = 0;  // non-decreasing in kt: two pointers
+    const int nq = ceil_div(t.rows, kBwdBQ);
     for (int kt = 0; kt < g->bKT; ++kt) {
-      int k0 = kt * kBwdBK, k1 = k0 + kBwdBK - 1;
-      while (first < nq && row_bound(t.I0, t.I1, t.L, std::min((first + 1) * kBwdBQ, R) - 1) < k0) ++first;
-      while (full < nq && !((full + 1) * kBwdBQ <= R && row_bound(t.I0, t.I1, t.L, full * kBwdBQ) >= k1)) ++full;
-      int f = std::max(full, first);
-      g->bwd_tiles[(size_t(b) * g->bKT + kt) * 2 + 0] = first;
-      g->bwd_tiles[(size_t(b) * g->bKT + kt) * 2 + 1] = f;
-      bwd_cost[size_t(b) * g->bKT + kt] = nq - first;
+      const int k0 = kt * kBwdBK, k1 = std::min(k0 + kBwdBK, S) - 1;
+      int first = -1, last = -1, f0 = -1, f1 = -1;
+      for (int qt = 0; qt < nq; ++qt) {
+        const int q0 = qt * kBwdBQ, q1 = std::min(q0 + kBwdBQ, int(t.rows)) - 1;
+        int64_t vis = 0;
+        for (int q = q0; q <= q1; ++q) vis += visible_in(imgs(b), t.n_img, t.L, q, k0, k1);
+        if (vis == 0) continue;
+        if (first < 0) first = qt;
+        last = qt;
+        const bool full = q1 - q0 + 1 == kBwdBQ && k1 - k0 + 1 == kBwdBK && vis == int64_t(kBwdBQ) * kBwdBK;
+        if (full && (f0 < 0 || f1 == qt)) {
+          if (f0 < 0) f0 = qt;
+          f1 = qt + 1;
+        }
+      }
+      int32_t* e = &g->bwd_tiles[(size_t(b) * g->bKT + kt) * 4];
+      e[0] = first < 0 ? 0 : first;
+      e[1] = first < 0 ? 0 : last + 1;
+      e[2] = f0 < 0 ? 0 : f0;
+      e[3] = f0 < 0 ? 0 : f1;
+      bwd_cost[size_t(b) * g->bKT + kt] = e[1] - e[0];
     }
   }
   order.assign(size_t(B) * g->bKT, 0);
@@ -151,31 +197,80 @@ static int build(const hia_sample* s, int B, int S, bool packed, hia_segments** 
   return HIA_OK;
 }
 
-static int check_args(const hia_sample* s, int B, hia_segments** out) {
-  if (!out || B < 0 || (B > 0 && !s)) return HIA_ERR_INVALID_ARG;
-  *out = nullptr;
-  if (B >= (1 << 20)) return HIA_ERR_INVALID_ARG;
+// The one-image form: prefix, one image (none when h = w = 0), suffix.
+int from_samples(const hia_sample* s, int B, std::vector<SampleSpec>* spec) {
+  spec->resize(B);
+  for (int b = 0; b < B; ++b) {
+    const hia_sample& x = s[b];
+    if (x.prefix_len < 0 || x.img_h < 0 || x.img_w < 0 || x.suffix_len < 0 || ((x.img_h == 0) != (x.img_w == 0)))
+      return HIA_ERR_INVALID_ARG;
+    SampleSpec& o = (*spec)[b];
+    if (x.img_h > 0) {
+      o.images.push_back({x.prefix_len, x.img_h, x.img_w});
+      o.suffix = x.suffix_len;
+    } else {
+      const int64_t t = int64_t(x.prefix_len) + x.suffix_len;
+      if (t >= (int64_t(1) << 31)) return HIA_ERR_INVALID_ARG;
+      o.suffix = int32_t(t);
+    }
+  }
   return HIA_OK;
 }
 
+int64_t max_length(const std::vector<SampleSpec>& spec) {
+  int64_t S = 0;
+  for (const SampleSpec& x : spec) {
+    int64_t L = x.suffix;
+    for (const hia_image& im : x.images) L += int64_t(im.text_before) + int64_t(im.img_h) * im.img_w;
+    S = std::max(S, L);
+  }
+  return S;
+}
+
+}  // namespace
+
 extern "C" int hia_segments_build(const hia_sample* s, int B, int S, hia_segments** out) {
-  int rc = check_args(s, B, out);
-  if (rc) return rc;
+  if (!out || B < 0 || (B > 0 && !s) || B >= (1 << 20)) return HIA_ERR_INVALID_ARG;
+  *out = nullptr;
   if (S < 0 || S >= (1 << 24)) return HIA_ERR_INVALID_ARG;
-  return build(s, B, S, false, out);
+  std::vector<SampleSpec> spec;
+  int rc = from_samples(s, B, &spec);
+  return rc ? rc : build(spec, S, false, out);
 }
 
 extern "C" int hia_segments_build_packed(const hia_sample* s, int B, hia_segments** out) {
-  int rc = check_args(s, B, out);
+  if (!out || B < 0 || (B > 0 && !s) || B >= (1 << 20)) return HIA_ERR_INVALID_ARG;
+  *out = nullptr;
+  std::vector<SampleSpec> spec;
+  int rc = from_samples(s, B, &spec);
   if (rc) return rc;
-  int64_t S = 0;
-  for (int b = 0; b < B; ++b) {
-    const hia_sample& x = s[b];
-    if (x.prefix_len < 0 || x.img_h < 0 || x.img_w < 0 || x.suffix_len < 0) return HIA_ERR_INVALID_ARG;
-    S = std::max(S, int64_t(x.prefix_len) + int64_t(x.img_h) * x.img_w + x.suffix_len);
-  }
+  const int64_t S = max_length(spec);
   if (S >= (1 << 24)) return HIA_ERR_INVALID_ARG;
-  return build(s, B, int(S), true, out);
+  return build(spec, int(S), true, out);
+}
+
+extern "C" int hia_segments_build_multi(const hia_image* images, const int32_t* n_images,
+                                        const int32_t* suffix_len, int B, int S, int packed,
+                                        hia_segments** out) {
+  if (!out || B < 0 || (B > 0 && (!n_images || !suffix_len)) || B >= (1 << 20)) return HIA_ERR_INVALID_ARG;
+  *out = nullptr;
+  std::vector<SampleSpec> spec(B);
+  int64_t k = 0;
+  for (int b = 0; b < B; ++b) {
+    if (n_images[b] < 0 || n_images[b] > (1 << 16) || suffix_len[b] < 0) return HIA_ERR_INVALID_ARG;
+    if (n_images[b] > 0 && !images) return HIA_ERR_INVALID_ARG;
+    spec[b].images.assign(images + k, images + k + n_images[b]);
+    spec[b].suffix = suffix_len[b];
+    k += n_images[b];
+  }
+  if (packed) {
+    const int64_t L = max_length(spec);
+    if (L >= (1 << 24)) return HIA_ERR_INVALID_ARG;
+    S = int(L);
+  } else if (S < 0 || S >= (1 << 24)) {
+    return HIA_ERR_INVALID_ARG;
+  }
+  return build(spec, S, packed != 0, out);
 }
 
 extern "C" int hia_segments_info(const hia_segments* g, hia_segments_info_t* info) {
@@ -197,7 +292,8 @@ extern "C" int hia_segments_row_bound(const hia_segments* g, int32_t* e) {
   if (!g || (!e && g->B * int64_t(g->S) > 0)) return HIA_ERR_INVALID_ARG;
   for (int b = 0; b < g->B; ++b) {
     const auto& t = g->samples[b];
-    for (int q = 0; q < g->S; ++q) e[int64_t(b) * g->S + q] = row_bound(t.I0, t.I1, t.L, q);
+    const ImageDev* im = g->images.data() + t.img0;
+    for (int q = 0; q < g->S; ++q) e[int64_t(b) * g->S + q] = row_bound(im, t.n_img, t.L, q);
   }
   return HIA_OK;
 }
@@ -207,11 +303,14 @@ extern "C" int hia_segments_mask(const hia_segments* g, uint8_t* m) {
   const int64_t S = g->S;
   for (int b = 0; b < g->B; ++b) {
     const auto& t = g->samples[b];
+    const ImageDev* im = g->images.data() + t.img0;
     for (int64_t q = 0; q < S; ++q) {
       uint8_t* row = m + (int64_t(b) * S + q) * S;
-      int64_t e = row_bound(t.I0, t.I1, t.L, int32_t(q));
+      int64_t e = row_bound(im, t.n_img, t.L, int32_t(q));
       std::memset(row, 0, size_t(S));
       if (e >= 0) std::memset(row, 1, size_t(e + 1));
+      for (int i = 0; i < t.n_img; ++i)  // context images ended before this row
+        if (im[i].hidden && im[i].I1 <= q) std::memset(row + im[i].I0, 0, size_t(im[i].I1 - im[i].I0));
     }
   }
   return HIA_OK;
@@ -222,15 +321,13 @@ extern "C" int hia_segments_tile_classes(const hia_segments* g, uint8_t* cls) {
   for (int b = 0; b < g->B; ++b) {
     const auto& t = g->samples[b];
     for (int qt = 0; qt < g->nQT; ++qt) {
-      int n_full = g->fwd_tiles[(size_t(b) * g->nQT + qt) * 2 + 0];
-      int n_vis = g->fwd_tiles[(size_t(b) * g->nQT + qt) * 2 + 1];
-      for (int kt = 0; kt < g->nKT; ++kt) {
-        uint8_t c;
-        if (kt < n_full) c = HIA_TILE_FULL;
-        else if (kt < n_vis) c = HIA_TILE_PARTIAL;
-        else if (kt * hia::kFwdBN >= t.L) c = HIA_TILE_PADDED;
-        else c = HIA_TILE_SKIP;
-        cls[(size_t(b) * g->nQT + qt) * g->nKT + kt] = c;
+      uint8_t* row = cls + (size_t(b) * g->nQT + qt) * g->nKT;
+      for (int kt = 0; kt < g->nKT; ++kt) row[kt] = kt * hia::kFwdBN >= t.L ? HIA_TILE_PADDED : HIA_TILE_SKIP;
+      const int first = g->fwd_tiles[(size_t(b) * g->nQT + qt) * 2 + 0];
+      const int count = g->fwd_tiles[(size_t(b) * g->nQT + qt) * 2 + 1];
+      for (int j = 0; j < count; ++j) {
+        const int32_t x = g->fwd_list[first + j];
+        row[x & 0xffff] = (x >> 16) ? HIA_TILE_FULL : HIA_TILE_PARTIAL;
       }
     }
   }

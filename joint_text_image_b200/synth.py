@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for the five attention workloads.
+"""Seeded synthetic inputs for the attention workloads.
 
 This module holds no attention, mask or RoPE arithmetic: it only draws
 sequence lengths and bf16 normal tensors from a seeded torch CPU generator.
@@ -21,7 +21,7 @@ import torch
 @dataclass
 class Workload:
     name: str
-    samples: list            # [(prefix, img_h, img_w, suffix)] per batch row
+    samples: list            # per batch row: (prefix, img_h, img_w, suffix) or (images, suffix)
     Hq: int
     Hkv: int
     D: int
@@ -44,13 +44,22 @@ def _draw(gen, lo, hi, n):
     return [int(x) for x in torch.randint(lo, hi + 1, (n,), generator=gen)]
 
 
+def _length(x):
+    """Valid length of a sample: (prefix, h, w, suffix), or (images, suffix)
+    with images a list of (text_before, h, w)."""
+    if len(x) == 2:
+        return sum(t + h * w for (t, h, w) in x[0]) + x[1]
+    p, h, w, s = x
+    return p + h * w + s
+
+
 def _finish(name, samples, Hq, Hkv, D, **kw):
-    S = max(p + h * w + s for (p, h, w, s) in samples) if samples else 0
+    S = max(_length(x) for x in samples) if samples else 0
     return Workload(name=name, samples=samples, Hq=Hq, Hkv=Hkv, D=D, S=S, **kw)
 
 
 def workload(name: str, seed: int = 0) -> Workload:
-    """The five synthetic workloads; lengths drawn from torch.Generator(seed)."""
+    """The synthetic workloads; lengths drawn from torch.Generator(seed)."""
     gen = torch.Generator().manual_seed(seed)
     if name == "tiny":
         # 15 text + <timestep> = prefix 16; 8x8 image; suffix 2; no padding.
@@ -72,10 +81,17 @@ def workload(name: str, seed: int = 0) -> Workload:
         return _finish(name, samples, 32, 8, 128)
     if name == "1024px_bwd":
         return _finish(name, [(1024, 64, 64, 2)], 32, 8, 128, backward=True)
+    if name == "multi_image":
+        # two generated images per sample: prefix U[256,768], a 512px image
+        # (32x32 tokens, in context for what follows), a 64-token caption,
+        # a 1024px image (64x64), suffix 2.
+        pre = _draw(gen, 256, 768, 2)
+        samples = [([(p, 32, 32), (64, 64, 64)], 2) for p in pre]
+        return _finish(name, samples, 32, 8, 128, backward=True)
     raise KeyError(name)
 
 
-WORKLOADS = ("tiny", "256px", "1024px", "mixed", "1024px_bwd")
+WORKLOADS = ("tiny", "256px", "1024px", "mixed", "1024px_bwd", "multi_image")
 
 
 def tensors(wl: Workload, seed: int = 0, grad: bool = False):

@@ -1,0 +1,112 @@
+"""GPU parity for samples with several images (hia_segments_build_multi):
+the forward and backward against the fp64 oracle, the one-image form against
+the canonical builder, and the packed layout against the padded one."""
+import numpy as np
+import pytest
+import torch
+
+import joint_text_image_b200 as jt
+from helpers import GRAD_REL, LSE_MAX, O_MAX, O_MEAN
+
+pytestmark = pytest.mark.gpu
+
+# Two context images and a last one, text in between; a sample whose only
+# image is followed by a second; a text-only sample; image at position 0.
+SAMPLES = [
+    ([(33, 8, 16), (20, 16, 8), (7, 12, 12)], 2),
+    ([(150, 16, 16), (1, 4, 32)], 40),
+    ([], 300),
+    ([(0, 10, 10), (64, 6, 6)], 3),
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    assert torch.cuda.is_available(), "needs a GPU"
+    jt.lib()
+
+
+def length(x):
+    return sum(t + h * w for t, h, w in x[0]) + x[1]
+
+
+def inputs(S, Hq, Hkv, D, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    B = len(SAMPLES)
+    q = torch.randn(B, S, Hq, D, generator=g).bfloat16()
+    k = torch.randn(B, S, Hkv, D, generator=g).bfloat16()
+    v = torch.randn(B, S, Hkv, D, generator=g).bfloat16()
+    do = torch.randn(B, S, Hq, D, generator=g).bfloat16()
+    return q, k, v, do
+
+
+def run(seg, q, k, v, do, scale):
+    D = q.shape[-1]
+    c, s = jt.hia_rope2d_tables(seg, D)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = jt.hia_attn_fwd(seg, qd, kd, vd, c, s, scale)
+    dq, dk, dv = jt.hia_attn_bwd(seg, qd, kd, vd, c, s, o, lse, dod, scale)
+    torch.cuda.synchronize()
+    assert jt.hia_get_device_status() == 0
+    return [t.cpu() for t in (o, lse, dq, dk, dv)], (c.cpu(), s.cpu())
+
+
+@pytest.mark.parametrize("D", [128, 64])
+def test_multi_image_parity_with_oracle(oracle_mod, D):
+    S = max(length(x) for x in SAMPLES) + 17
+    Hq, Hkv = 4, 2
+    q, k, v, do = inputs(S, Hq, Hkv, D)
+    seg = jt.hia_segments_build_multi(SAMPLES, S)
+    (o, lse, dq, dk, dv), (c, s) = run(seg, q, k, v, do, D ** -0.5)
+    # tables: each image on its own grid, within one fp32 ulp of the oracle
+    cr, sr = oracle_mod.rope_tables(SAMPLES, S, D)
+    for got, ref in ((c, cr), (s, sr)):
+        ref32 = ref.astype(np.float32)
+        assert np.all(np.abs(got.numpy().astype(np.float64) - ref32) <= np.spacing(np.abs(ref32)))
+    f64 = lambda t: t.double().numpy()
+    o_ref, lse_ref, _ = oracle_mod.attn_fwd(SAMPLES, f64(q), f64(k), f64(v), D ** -0.5)
+    err = np.abs(o.float().numpy() - o_ref)
+    assert err.max() <= O_MAX and err.mean() <= O_MEAN
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lse.numpy()), fin)
+    assert np.abs(lse.numpy()[fin] - lse_ref[fin]).max() <= LSE_MAX
+    refs = oracle_mod.attn_bwd(SAMPLES, f64(q), f64(k), f64(v), f64(do), D ** -0.5)[:3]
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
+        rel = np.linalg.norm(got.float().numpy() - ref) / np.linalg.norm(ref)
+        assert rel <= GRAD_REL, (name, rel)
+
+
+def test_multi_packed_equals_padded():
+    S = max(length(x) for x in SAMPLES) + 9
+    q, k, v, do = inputs(S, 4, 2, 128, seed=1)
+    lens = [length(x) for x in SAMPLES]
+    for b, L in enumerate(lens):
+        do[b, L:] = 0  # padded rows then add nothing to dk, dv
+    pad, _ = run(jt.hia_segments_build_multi(SAMPLES, S), q, k, v, do, 128 ** -0.5)
+    seg = jt.hia_segments_build_multi(SAMPLES, packed=True)
+    pack = lambda x: torch.cat([x[b, :L] for b, L in enumerate(lens)], 0).contiguous()
+    c, s = jt.hia_rope2d_tables(seg, 128)
+    qp, kp, vp, dop = (pack(t).cuda() for t in (q, k, v, do))
+    o, lse = jt.hia_attn_fwd(seg, qp, kp, vp, c, s)
+    dq, dk, dv = jt.hia_attn_bwd(seg, qp, kp, vp, c, s, o, lse, dop)
+    torch.cuda.synchronize()
+    o, lse, dq, dk, dv = (t.cpu() for t in (o, lse, dq, dk, dv))
+    off = 0
+    for b, L in enumerate(lens):
+        assert torch.equal(o[off:off + L], pad[0][b, :L]) and torch.equal(lse[:, off:off + L], pad[1][b, :, :L])
+        assert torch.equal(dk[off:off + L], pad[3][b, :L]) and torch.equal(dv[off:off + L], pad[4][b, :L])
+        a, r = dq[off:off + L].float(), pad[2][b, :L].float()
+        assert (a - r).norm() <= 1e-3 * max(r.norm(), 1e-30)
+        off += L
+
+
+def test_one_image_multi_form_equals_canonical():
+    canon = [(40, 8, 8, 2), (0, 0, 0, 0), (90, 0, 0, 0), (0, 12, 12, 5)]
+    multi = [([(40, 8, 8)], 2), ([], 0), ([], 90), ([(0, 12, 12)], 5)]
+    S = 160
+    q, k, v, do = inputs(S, 4, 2, 128, seed=2)
+    a, _ = run(jt.hia_segments_build(canon, S), q, k, v, do, 128 ** -0.5)
+    b, _ = run(jt.hia_segments_build_multi(multi, S), q, k, v, do, 128 ** -0.5)
+    for i in (0, 1, 3, 4):  # o, lse, dk, dv bitwise; dq up to its reduction order
+        assert torch.equal(a[i], b[i])
+    assert (a[2].float() - b[2].float()).norm() <= 1e-3 * a[2].float().norm()

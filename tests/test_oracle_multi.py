@@ -1,5 +1,6 @@
 """Pins for the oracle's multi-image sequences (technical report summary
-3.1.2: images in context are masked from subsequent tokens): hand-written
+3.1.2: with several generated images, an image already in context is hidden
+from the tokens after it): hand-written
 masks, the reduction to the one-image layout, hand-derived positions, the
 row-bound-minus-hidden-spans form the kernels use, and a library attention
 routine on the multi-image mask."""
@@ -120,3 +121,30 @@ def test_bad_multi_geometry_refused(oracle_mod):
         oracle_mod.mask([([(1, 0, 2)], 1)], 8)   # an image needs h, w > 0
     with pytest.raises(ValueError):
         oracle_mod.mask([([(1, 2, 2)], 1)], 5)   # L = 6 > S
+
+
+def test_mask_columns_are_row_intervals(oracle_mod):
+    """The backward's form: key k is seen exactly by the rows
+    [first(k), end(k)), first(k) = its image's first token (or k itself for
+    text), end(k) = the end of its image when that is a context image (else S);
+    padded keys by no row."""
+    rng = np.random.default_rng(33)
+    for images, suffix in _random_layouts(rng, 60):
+        spans, pos = [], 0
+        for (t, h, w) in images:
+            spans.append((pos + t, pos + t + h * w))
+            pos += t + h * w
+        L = pos + suffix
+        S = L + int(rng.integers(0, 3))
+        m = oracle_mod.mask([(images, suffix)], S)[0].astype(bool)
+        for k in range(S):
+            want = np.zeros(S, dtype=bool)
+            if k < L:
+                first, end = k, S
+                for i, (a, b) in enumerate(spans):
+                    if a <= k < b:
+                        first = a
+                        if i < len(spans) - 1:
+                            end = b
+                want[first:end] = True
+            assert np.array_equal(m[:, k], want), (images, suffix, k)
