@@ -191,6 +191,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-inflight", type=int, default=2,
+                    help="host-buffer steps in flight (each on its own stream and hia_step) in the e2e timing")
     ap.add_argument("--ref-row-stride", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
@@ -327,27 +329,30 @@ def main():
     # would run it.
     e2e = None
     if args.e2e_steps > 0 and not args.packed:  # the host-buffer step uses the padded layout
-        hin = [tuple(t.pin_memory() for t in (q, k, v, do)) for _ in range(2)]
+        nf = max(1, args.e2e_inflight)
+        hin = [tuple(t.pin_memory() for t in (q, k, v, do)) for _ in range(nf)]
         mk = lambda t, dt=torch.bfloat16: torch.empty(t.shape, dtype=dt, pin_memory=True)
-        hout = [(mk(o), mk(lse, torch.float32), mk(dq), mk(dk), mk(dv)) for _ in range(2)]
+        hout = [(mk(o), mk(lse, torch.float32), mk(dq), mk(dk), mk(dv)) for _ in range(nf)]
         h2d = sum(t.numel() * t.element_size() for t in hin[0])
         d2h = sum(t.numel() * t.element_size() for t in hout[0])
-        hsteps = [jt.hia_step_create(seg, wl.Hq, wl.Hkv, wl.D, wl.base) for _ in range(2)]
-        hstreams = [torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)]
+        hsteps = [jt.hia_step_create(seg, wl.Hq, wl.Hkv, wl.D, wl.base) for _ in range(nf)]
+        hstreams = [torch.cuda.Stream(device=dev) for _ in range(nf)]
 
         def e2e_run(n):
             for i in range(n):
-                j = i % 2
+                j = i % nf
                 jt.hia_attn_step_host(hsteps[j], *hin[j], *hout[j], scale=wl.scale, stream=hstreams[j])
 
-        e2e_run(4)
+        e2e_run(2 * nf)
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(hstreams[0])
-        hstreams[1].wait_stream(hstreams[0])
+        for st in hstreams[1:]:
+            st.wait_stream(hstreams[0])
         e2e_run(args.e2e_steps)
-        hstreams[0].wait_stream(hstreams[1])
+        for st in hstreams[1:]:
+            hstreams[0].wait_stream(st)
         e1.record(hstreams[0])
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1) / args.e2e_steps
@@ -357,7 +362,7 @@ def main():
             ems = float(t.item())
         e2e = {"value": world * step_flops / (ems * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems,
-               "api": "hia_attn_step_host (C ABI, host buffers), two steps in flight on two streams"}
+               "api": f"hia_attn_step_host (C ABI, host buffers), {nf} steps in flight on {nf} streams"}
         del hsteps
 
     cpu = None
