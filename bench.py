@@ -89,6 +89,24 @@ SAMPLE_DESC = ("batch row 0, kv head 0 (its {g} query heads), query rows 0, {str
                "fp64 oracle forward + backward restricted to those rows")
 
 
+def max_over_ranks(x, world, device="cpu"):
+    """The largest of every rank's x (each rank's device-timed milliseconds):
+    an all-reduce MAX, on `device` (cuda for NCCL, cpu for gloo)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world, step_flops, ms):
+    """Whole-job throughput: every rank's step (the same work per rank) over
+    the slowest rank's step time."""
+    return world * step_flops / (ms * 1e-3) / 1e12
+
+
 def kernel_source_sha256(kernel):
     """sha256 over the sources the kernel is compiled from, in a fixed order."""
     h = hashlib.sha256()
@@ -295,11 +313,8 @@ def main():
     ms = ev0.elapsed_time(ev1) / args.steps
     if jt.hia_get_device_status() != 0:
         raise RuntimeError("device wait timed out during the timed region")
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * step_flops / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(ms, world, dev)
+    value = job_tflops(world, step_flops, ms)
     launches = sum(n for (n, _) in prof.values())
 
     # per-kernel times measured live in the timed region (events on the launch stream)
@@ -356,11 +371,8 @@ def main():
         e1.record(hstreams[0])
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * step_flops / (ems * 1e-3) / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+        ems = max_over_ranks(ems, world, dev)
+        e2e = {"value": job_tflops(world, step_flops, ems), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems,
                "api": f"hia_attn_step_host (C ABI, host buffers), {nf} steps in flight on {nf} streams"}
         del hsteps
