@@ -348,7 +348,8 @@ const char* hia_status_string(int status);
  * records, one per kernel name, with the launch count and the summed
  * event-to-event time; *n_out receives the number of records.  Kernel names:
  * "rope2d_tables", "rope_rotate", "attn_fwd", "bwd_pre", "attn_bwd",
- * "dq_finalize".  Not a library-wide profiler: no other state changes. */
+ * "grad_finalize", "dw_reduce".  Not a library-wide profiler: no other state
+ * changes. */
 typedef struct {
     char name[32];
     int32_t launches;
