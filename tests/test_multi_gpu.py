@@ -110,3 +110,48 @@ def test_one_image_multi_form_equals_canonical():
     for i in (0, 1, 3, 4):  # o, lse, dk, dv bitwise; dq up to its reduction order
         assert torch.equal(a[i], b[i])
     assert (a[2].float() - b[2].float()).norm() <= 1e-3 * a[2].float().norm()
+
+
+def test_multi_packed_with_qk_norm_against_oracle(oracle_mod):
+    """All three options at once: several images per sample, the packed
+    layout and the QK RMSNorm, against the oracle on the padded equivalent."""
+    S = max(length(x) for x in SAMPLES) + 5
+    Hq, Hkv, D, eps = 4, 2, 128, 1e-5
+    q, k, v, do = inputs(S, Hq, Hkv, D, seed=3)
+    lens = [length(x) for x in SAMPLES]
+    for b, L in enumerate(lens):
+        do[b, L:] = 0
+    g = torch.Generator().manual_seed(9)
+    wq = (torch.rand(D, generator=g, dtype=torch.float64) + 0.5).float()
+    wk = (torch.rand(D, generator=g, dtype=torch.float64) + 0.5).float()
+    seg = jt.hia_segments_build_multi(SAMPLES, packed=True)
+    pack = lambda x: torch.cat([x[b, :L] for b, L in enumerate(lens)], 0).contiguous()
+    c, s = jt.hia_rope2d_tables(seg, D)
+    qp, kp, vp, dop = (pack(t).cuda() for t in (q, k, v, do))
+    norm = (wq.cuda(), wk.cuda(), eps)
+    o, lse = jt.hia_attn_fwd(seg, qp, kp, vp, c, s, qk_norm=norm)
+    dq, dk, dv, dwq, dwk = jt.hia_attn_bwd(seg, qp, kp, vp, c, s, o, lse, dop, qk_norm=norm)
+    torch.cuda.synchronize()
+    assert jt.hia_get_device_status() == 0
+    ref_norm = (wq.double().numpy(), wk.double().numpy(), eps)
+    f64 = lambda t: t.double().numpy()
+    o_ref, lse_ref, _ = oracle_mod.attn_fwd(SAMPLES, f64(q), f64(k), f64(v), D ** -0.5, qk_norm=ref_norm)
+    rdq, rdk, rdv, rdwq, rdwk, _ = oracle_mod.attn_bwd_qknorm(SAMPLES, f64(q), f64(k), f64(v), f64(do), ref_norm,
+                                                              D ** -0.5)
+    off = 0
+    errs, grads = [], {"dq": ([], []), "dk": ([], []), "dv": ([], [])}
+    for b, L in enumerate(lens):
+        errs.append(np.abs(o[off:off + L].float().cpu().numpy() - o_ref[b, :L]).ravel())
+        lr = lse_ref[b, :, :L]
+        assert np.abs(lse[:, off:off + L].cpu().numpy() - lr).max() <= LSE_MAX
+        for name, got, ref in (("dq", dq, rdq), ("dk", dk, rdk), ("dv", dv, rdv)):
+            grads[name][0].append(got[off:off + L].float().cpu().numpy().ravel())
+            grads[name][1].append(ref[b, :L].ravel())
+        off += L
+    e = np.concatenate(errs)
+    assert e.max() <= O_MAX and e.mean() <= O_MEAN
+    for name, (a, r) in grads.items():
+        a, r = np.concatenate(a), np.concatenate(r)
+        assert np.linalg.norm(a - r) / np.linalg.norm(r) <= GRAD_REL, name
+    for got, ref in ((dwq, rdwq), (dwk, rdwk)):
+        assert np.linalg.norm(got.cpu().numpy() - ref) / np.linalg.norm(ref) <= GRAD_REL

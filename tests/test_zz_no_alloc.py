@@ -75,3 +75,26 @@ def test_noalloc_refuses_problems_beyond_the_scratch():
     rc = jt.lib().hia_attn_fwd_noalloc(seg.handle, 32, 8, 128, z, z, z, None, None, 0.088, z, None, None)
     assert rc == SCRATCH_LIMIT
     assert b"64 MiB" in jt.lib().hia_status_string(rc)
+
+
+def test_noalloc_packed_layout_matches_workspace_forward():
+    """The fixed-scratch forward on a packed descriptor (samples back to back)."""
+    import joint_text_image_b200 as jt
+    from joint_text_image_b200 import synth
+    wl = synth.workload("256px")
+    q, k, v = synth.tensors(wl, 4)
+    seg = jt.hia_segments_build_packed(wl.samples)
+    pack = lambda x: torch.cat([x[b, :L] for b, L in enumerate(seg.lengths)], 0).contiguous().cuda()
+    qp, kp, vp = pack(q), pack(k), pack(v)
+    c, s = jt.hia_rope2d_tables(seg, wl.D)
+    o_ref, lse_ref = jt.hia_attn_fwd(seg, qp, kp, vp, c, s)
+    o = torch.empty_like(o_ref)
+    lse = torch.empty_like(lse_ref)
+    g = wl.Hq // wl.Hkv
+    rc = jt.lib().hia_attn_fwd_noalloc(seg.handle, wl.Hq, wl.Hkv, wl.D, jt._t(qp.unsqueeze(0), True, g),
+                                       jt._t(kp.unsqueeze(0), False, 1), jt._t(vp.unsqueeze(0), False, 1),
+                                       c.data_ptr(), s.data_ptr(), wl.scale, jt._t(o.unsqueeze(0), True, g),
+                                       lse.data_ptr(), jt._stream())
+    torch.cuda.synchronize()
+    assert rc == 0
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
