@@ -108,9 +108,10 @@ static int image_of(const osample* s, int64_t n) {
 }
 
 /* The literal mask rule (build_joint_attention_mask; 3.1.2; 3.3), with the
- * multi-image rule of 3.1.2 (images in context are masked from subsequent
- * tokens; read here as: every image but the sample's last is hidden from all
- * tokens after its span, the last image follows the one-image rule):
+ * multi-image rule of 3.1.2 (in a training sequence with several generated
+ * images, an image already in context is masked from the tokens after it;
+ * read here as: every image but the sample's last is hidden from all tokens
+ * after its span, the last image follows the one-image rule):
  *   key k visible from query q  <=>  k < L  and  ( q, k in the same image  or
  *                                   ( k <= q  and  k not in a context image ) ),
  * a context image being one of images 0 .. n-2 (any k <= q outside q's own
