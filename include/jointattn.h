@@ -249,7 +249,12 @@ int hia_attn_fwd_ex(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor 
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current), which also loads the
  *     library module holding it; make that first call before any stream
- *     capture on the device.
+ *     capture on the device.  The address belongs to the device's context:
+ *     if the context is replaced (cudaDeviceReset, then new work), the next
+ *     call sees the new context and looks the address up again, so that call
+ *     too should come before any capture.
+ *   - Argument errors are checked first, exactly as hia_attn_fwd checks
+ *     them; only a problem with valid arguments can get the size error.
  *   - All calls share the one array and it keeps the last call's contents
  *     (nothing in it needs to start at zero: every element that is read is
  *     first rewritten by the same call).  Calls whose GPU work overlaps, e.g.
@@ -288,13 +293,33 @@ int hia_attn_bwd_ex(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor 
                     hia_tensor dq, hia_tensor dk, hia_tensor dv, float* dwq, float* dwk,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* hia_attn_bwd_ex that reuses the rotated (and, with a norm, normed) q and
+ * k which the forward left in its workspace, instead of computing them again
+ * (the rotation is the same arithmetic either way: R q and R k in fp32,
+ * rounded once to bf16).  fwd_workspace: the workspace of the
+ * hia_attn_fwd / hia_attn_fwd_ex call that produced o and lse, with the same
+ * seg, heads, D, q, k, cos, sin and norm, not written since;
+ * fwd_workspace_bytes >= hia_attn_fwd_workspace_bytes and 256-byte aligned.
+ * A caller that keeps the forward workspace alive until the backward trades
+ * that memory (B*S*(Hq+Hkv)*D*2 bytes) for one rotation pass per step.
+ * fwd_workspace == NULL: identical to hia_attn_bwd_ex.  The backward
+ * workspace is still required (its dQ accumulator and row statistics).
+ * Errors as hia_attn_bwd_ex, plus HIA_ERR_INVALID_ARG for a short or
+ * misaligned fwd_workspace. */
+int hia_attn_bwd_reuse_fwd(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                           hia_tensor v, const float* cos_t, const float* sin_t, float scale,
+                           const hia_qk_norm* norm, hia_tensor o, const float* lse, hia_tensor dout,
+                           hia_tensor dq, hia_tensor dk, hia_tensor dv, float* dwq, float* dwk,
+                           const void* fwd_workspace, size_t fwd_workspace_bytes, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
 /* ---- One training step from HOST buffers.  (No counterpart on the pages:
  * a convenience of the library for callers that hold their tensors in host
  * memory.)  A hia_step owns, on the device current at creation, the device
  * copies of one step's tensors in the plain contiguous layout (q, dout, o,
  * dq: [B,S,Hq,D] bf16; k, v, dk, dv: [B,S,Hkv,D] bf16; lse: [B,Hq,S] fp32),
  * the RoPE tables of `seg` (computed once, at creation, with `rope_base`) and
- * both workspaces.  `seg` must stay alive and uploaded while the step exists.
+ * both workspaces (the backward reuses the forward's rotated q and k).  `seg` must stay alive and uploaded while the step exists.
  * Returns HIA_ERR_INVALID_ARG for null pointers, non-positive head counts
  * or rope_base, HIA_ERR_UNSUPPORTED unless D is 64 or 128 and Hq a multiple
  * of Hkv, HIA_ERR_NOT_ON_DEVICE if `seg` was not uploaded, HIA_ERR_CUDA if

@@ -30,7 +30,8 @@ EXPORTED_SYMBOLS = (
     "hia_get_device_status", "hia_debug_wait_timeout", "hia_status_string", "hia_profile_begin",
     "hia_profile_end", "hia_attn_fwd_noalloc", "hia_debug_exp2", "hia_step_create", "hia_step_destroy",
     "hia_attn_step_host", "hia_attn_fwd_ex", "hia_attn_bwd_ex", "hia_segments_build_packed",
-    "hia_segments_layout", "hia_segments_build_multi",
+    "hia_segments_layout", "hia_segments_build_multi", "hia_attn_bwd_reuse_fwd",
+    "hia_moe_workspace_bytes", "hia_moe_fwd",
 )
 
 
@@ -67,6 +68,11 @@ class _Image(ctypes.Structure):
     _fields_ = [("text_before", ctypes.c_int32), ("img_h", ctypes.c_int32), ("img_w", ctypes.c_int32)]
 
 
+class _MoeDims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("topk", ctypes.c_int32)]
+
+
 class _KernelTime(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_double)]
 
@@ -101,6 +107,11 @@ def lib():
         L.hia_attn_bwd_workspace_bytes.restype = Z
         L.hia_attn_fwd.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, T, P, P, Z, P]
         L.hia_attn_bwd.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, T, P, T, T, T, T, P, Z, P]
+        L.hia_attn_bwd_reuse_fwd.argtypes = [P, I, I, I, T, T, T, P, P, ctypes.c_float, P, T, P, T, T, T, T, P, P,
+                                             P, Z, P, Z, P]
+        L.hia_moe_workspace_bytes.argtypes = [ctypes.POINTER(_MoeDims)]
+        L.hia_moe_workspace_bytes.restype = Z
+        L.hia_moe_fwd.argtypes = [ctypes.POINTER(_MoeDims), P, P, P, P, P, P, P, P, Z, P]
         L.hia_get_device_status.argtypes = [P]
         L.hia_debug_wait_timeout.argtypes = [ctypes.c_uint64, P]
         QN = ctypes.POINTER(_QkNorm)
@@ -345,10 +356,12 @@ def hia_attn_fwd(seg: Segments, q, k, v, cos, sin, scale=None, o=None, lse=None,
 
 
 def hia_attn_bwd(seg: Segments, q, k, v, cos, sin, o, lse, dout, scale=None, dq=None, dk=None, dv=None,
-                 workspace=None, qk_norm=None):
+                 workspace=None, qk_norm=None, fwd_workspace=None):
     """Recompute backward.  Returns (dq, dk, dv) bf16; with qk_norm (the
     forward's (wq, wk, eps)) returns (dq, dk, dv, dwq, dwk), dwq/dwk fp32 [D]
-    (hia_attn_bwd_ex)."""
+    (hia_attn_bwd_ex).  fwd_workspace: the workspace tensor of the forward
+    that produced o and lse, untouched since; its rotated q and k are reused
+    (hia_attn_bwd_reuse_fwd)."""
     import torch
     Hq, Hkv, D = _heads(_view(seg, q)), _heads(_view(seg, k)), q.shape[-1]
     g = Hq // Hkv
@@ -365,6 +378,21 @@ def hia_attn_bwd(seg: Segments, q, k, v, cos, sin, o, lse, dout, scale=None, dq=
     q, k, v, o, dout, dq, dk, dv = (_view(seg, x) for x in (q, k, v, o, dout, dq, dk, dv))
     nb = hia_attn_bwd_workspace_bytes(seg, Hq, Hkv, D)
     ws = _ws(nb, workspace)
+    if fwd_workspace is not None:
+        nf = hia_attn_fwd_workspace_bytes(seg, Hq, Hkv, D)
+        if fwd_workspace.numel() * fwd_workspace.element_size() < nf:
+            raise ValueError("forward workspace too small")
+        dwq = dwk = None
+        if qk_norm is not None:
+            dwq = torch.empty(D, device=q.device, dtype=torch.float32)
+            dwk = torch.empty(D, device=q.device, dtype=torch.float32)
+        _check(lib().hia_attn_bwd_reuse_fwd(
+            seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1), cos.data_ptr(),
+            sin.data_ptr(), float(scale), _norm(qk_norm, D), _t(o, True, g), lse.data_ptr(), _t(dout, True, g),
+            _t(dq, True, g), _t(dk, False, 1), _t(dv, False, 1), dwq.data_ptr() if dwq is not None else None,
+            dwk.data_ptr() if dwk is not None else None, fwd_workspace.data_ptr(), nf, ws.data_ptr(), nb,
+            _stream()), "hia_attn_bwd_reuse_fwd")
+        return ret if qk_norm is None else (*ret, dwq, dwk)
     if qk_norm is None:
         _check(lib().hia_attn_bwd(seg.handle, Hq, Hkv, D, _t(q, True, g), _t(k, False, 1), _t(v, False, 1),
                                   cos.data_ptr(), sin.data_ptr(), float(scale), _t(o, True, g), lse.data_ptr(),
@@ -444,3 +472,36 @@ def hia_profile_end():
     n = ctypes.c_int(0)
     _check(lib().hia_profile_end(arr, 16, ctypes.byref(n)), "hia_profile_end")
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(min(n.value, 16))}
+
+
+def hia_moe_workspace_bytes(T, H, I, E, topk):
+    return int(lib().hia_moe_workspace_bytes(ctypes.byref(_MoeDims(T, H, I, E, topk))))
+
+
+def hia_moe_fwd(x, wg, w13, w2, topk, out=None, workspace=None):
+    """MoE feed-forward of one block (jointmoe.h): x bf16 [T, H], wg fp32
+    [E, H], w13 bf16 [E + 1, 2I, H] ([up; gate], index E the shared expert),
+    w2 bf16 [E + 1, H, I], all contiguous CUDA tensors.  Returns (out bf16
+    [T, H], topk_ids int32 [T, topk], topk_weights fp32 [T, topk])."""
+    import torch
+    T, H = x.shape
+    E = wg.shape[0]
+    I = w13.shape[1] // 2
+    for t, dt in ((x, torch.bfloat16), (wg, torch.float32), (w13, torch.bfloat16), (w2, torch.bfloat16)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != dt:
+            raise ValueError("hia_moe_fwd takes contiguous CUDA tensors (x, w13, w2 bf16; wg fp32)")
+    if tuple(w13.shape) != (E + 1, 2 * I, H) or tuple(w2.shape) != (E + 1, H, I) or wg.shape[1] != H:
+        raise ValueError("inconsistent MoE weight shapes")
+    dims = _MoeDims(T, H, I, E, int(topk))
+    nb = int(lib().hia_moe_workspace_bytes(ctypes.byref(dims)))
+    if nb == 0:
+        raise HiaError(1, "hia_moe_workspace_bytes")
+    ws = _ws(nb, workspace)
+    if out is None:
+        out = torch.empty(T, H, device=x.device, dtype=torch.bfloat16)
+    ids = torch.empty(T, topk, device=x.device, dtype=torch.int32)
+    w = torch.empty(T, topk, device=x.device, dtype=torch.float32)
+    _check(lib().hia_moe_fwd(ctypes.byref(dims), x.data_ptr(), wg.data_ptr(), w13.data_ptr(), w2.data_ptr(),
+                             out.data_ptr(), ids.data_ptr(), w.data_ptr(), ws.data_ptr(), nb, _stream()),
+           "hia_moe_fwd")
+    return out, ids, w

@@ -11,8 +11,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libjointattn.so")
 BUILD = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "rope.cu", "attn_fwd.cu", "attn_bwd.cu", "probe.cu", "segments.cpp", "profile.cpp", "fwd_noalloc.cu", "host_step.cpp"]
-HEADERS = ["sm100.cuh", "internal.h", "kernels.h"]
+SOURCES = ["api.cu", "rope.cu", "attn_fwd.cu", "attn_bwd.cu", "probe.cu", "segments.cpp", "profile.cpp", "fwd_noalloc.cu", "host_step.cpp", "moe.cu"]
+HEADERS = ["sm100.cuh", "internal.h", "kernels.h", "devctx.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-Xptxas", "-warn-spills"]
@@ -28,7 +28,8 @@ def nvcc() -> str:
 def _inputs():
     srcs = [os.path.join(CSRC, s) for s in SOURCES if os.path.exists(os.path.join(CSRC, s))]
     deps = [os.path.join(CSRC, h) for h in HEADERS] + [
-        os.path.join(os.path.dirname(HERE), "include", "jointattn.h"), __file__]
+        os.path.join(os.path.dirname(HERE), "include", "jointattn.h"),
+        os.path.join(os.path.dirname(HERE), "include", "jointmoe.h"), __file__]
     return srcs, deps
 
 

@@ -8,7 +8,36 @@
 #include <cstring>
 #include <mutex>
 
+#include "devctx.h"
 #include "kernels.h"
+
+namespace hia {
+
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext c = nullptr;
+  if (get_current(&c) != CUDA_SUCCESS || !c) return 0;
+  unsigned long long id = 0;
+  return get_id(c, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+}  // namespace hia
 
 namespace {
 
@@ -18,19 +47,14 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per barrier wait
 
 __device__ int g_status;  // per-device status word (HIA_OK or HIA_ERR_DEVICE_TIMEOUT)
 
+// Device address of g_status in the current device's context.
 int* status_ptr() {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  static std::mutex mu;
-  static int* ptrs[64] = {};
-  std::lock_guard<std::mutex> lk(mu);
-  if (dev < 0 || dev >= 64) return nullptr;
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<int*>(p);
-  }
-  return ptrs[dev];
+  static hia::PerContext<int*> cache;
+  int* p = nullptr;
+  if (cache.get(&p, [](int** out) { return cudaGetSymbolAddress(reinterpret_cast<void**>(out), g_status); }) !=
+      cudaSuccess)
+    return nullptr;
+  return p;
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -67,6 +91,24 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+}  // namespace
+
+namespace hia {
+
+int* device_status_word() { return status_ptr(); }
+
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
+                 uint32_t box_cols, uint32_t box_rows) {
+  uint64_t dims[2] = {cols, rows};
+  uint64_t st[1] = {row_stride_bytes};
+  uint32_t box[2] = {box_cols, box_rows};
+  return make_map(m, base, 2, dims, st, box);
+}
+
+}  // namespace hia
+
+namespace {
 
 // [rows = S][D] per (b, head) slab of a [B*H][S][D] workspace tensor.
 bool make_ws_map(CUtensorMap* m, const void* base, int D, int S, int BH, uint32_t rows = 128) {
@@ -171,24 +213,33 @@ int check_norm(const hia_qk_norm* n) {
   return HIA_OK;
 }
 
-void rotate_into(const hia_tensor& src, int H, int g, const float* c, const float* s, __nv_bfloat16* dst,
-                 const hia_segments* seg, int D, cudaStream_t st, const float* w = nullptr, float eps = 0.f) {
+// q and k rotated (and, with the norm, normed) into the workspace by one launch.
+void rotate_qk(const hia_segments* seg, int Hq, int Hkv, int D, const hia_tensor& q, const hia_tensor& k,
+               const float* c, const float* s, const hia_qk_norm* norm, __nv_bfloat16* qr, __nv_bfloat16* kr,
+               cudaStream_t st) {
   hia::RotateArgs a{};
   a.samples = seg->d_samples;
-  a.w = w;
-  a.eps = eps;
-  a.src = src.ptr;
-  a.src_sb = src.stride_b;
-  a.src_ss = src.stride_s;
-  a.src_shkv = src.stride_hkv;
-  a.src_shq = src.stride_hq;
-  a.g = g;
   a.cos_t = c;
   a.sin_t = s;
-  a.dst = dst;
   a.B = seg->B;
   a.S = seg->S;
-  a.H = H;
+  a.n_parts = 2;
+  const hia_tensor* src[2] = {&q, &k};
+  const int heads[2] = {Hq, Hkv}, groups[2] = {Hq / Hkv, 1};
+  __nv_bfloat16* dst[2] = {qr, kr};
+  for (int i = 0; i < 2; ++i) {
+    hia::RotatePart& p = a.part[i];
+    p.src = src[i]->ptr;
+    p.src_sb = src[i]->stride_b;
+    p.src_ss = src[i]->stride_s;
+    p.src_shkv = src[i]->stride_hkv;
+    p.src_shq = src[i]->stride_hq;
+    p.g = groups[i];
+    p.H = heads[i];
+    p.w = norm ? (i == 0 ? norm->wq : norm->wk) : nullptr;
+    p.eps = norm ? norm->eps : 0.f;
+    p.dst = dst[i];
+  }
   hia::launch_rope_rotate(a, D, st);
 }
 
@@ -281,9 +332,11 @@ extern "C" int hia_attn_fwd(const hia_segments* g, int Hq, int Hkv, int D, hia_t
   return hia_attn_fwd_ex(g, Hq, Hkv, D, q, k, v, c, s, scale, nullptr, o, lse, ws, ws_bytes, stream);
 }
 
-extern "C" int hia_attn_fwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
-                               hia_tensor v, const float* c, const float* s, float scale, const hia_qk_norm* norm,
-                               hia_tensor o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+namespace hia {
+
+int fwd_check_args(const hia_segments* g, int Hq, int Hkv, int D, const hia_tensor& q, const hia_tensor& k,
+                   const hia_tensor& v, const float* c, const float* s, float scale, const hia_qk_norm* norm,
+                   const hia_tensor& o, const float* lse) {
   int rc = check_common(g, Hq, Hkv, D, c, s);
   if (rc) return rc;
   if ((rc = check_norm(norm))) return rc;
@@ -293,7 +346,20 @@ extern "C" int hia_attn_fwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
   if ((rc = check_tensor(q, true, g->B, g->S, gq)) || (rc = check_tensor(k, false, g->B, g->S, 1)) ||
       (rc = check_tensor(v, false, g->B, g->S, 1)) || (rc = check_tensor(o, true, g->B, g->S, gq)))
     return rc;
-  if (!q.ptr || !k.ptr || !v.ptr || !o.ptr || !lse || !ws) return HIA_ERR_INVALID_ARG;
+  if (!q.ptr || !k.ptr || !v.ptr || !o.ptr || !lse) return HIA_ERR_INVALID_ARG;
+  return HIA_OK;
+}
+
+}  // namespace hia
+
+extern "C" int hia_attn_fwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                               hia_tensor v, const float* c, const float* s, float scale, const hia_qk_norm* norm,
+                               hia_tensor o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  int rc = hia::fwd_check_args(g, Hq, Hkv, D, q, k, v, c, s, scale, norm, o, lse);
+  if (rc) return rc;
+  if (g->B == 0 || g->S == 0) return HIA_OK;
+  if (!ws) return HIA_ERR_INVALID_ARG;
+  const int gq = Hq / Hkv;
   packed_view(g, {&q, &k, &v, &o});
   const FwdWs w = fwd_ws(g, Hq, Hkv, D);
   if (ws_bytes < w.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return HIA_ERR_INVALID_ARG;
@@ -309,8 +375,7 @@ extern "C" int hia_attn_fwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
       !make_kv_map(&tv, v, D, Hkv, map_rows(g), map_batches(g), 128))
     return HIA_ERR_CUDA;
 
-  rotate_into(q, Hq, gq, c, s, qr, g, D, st, norm ? norm->wq : nullptr, norm ? norm->eps : 0.f);
-  rotate_into(k, Hkv, 1, c, s, kr, g, D, st, norm ? norm->wk : nullptr, norm ? norm->eps : 0.f);
+  rotate_qk(g, Hq, Hkv, D, q, k, c, s, norm, qr, kr, st);
 
   hia::FwdParams p{};
   p.samples = g->d_samples;
@@ -381,6 +446,16 @@ extern "C" int hia_attn_bwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
                                hia_tensor v, const float* c, const float* s, float scale, const hia_qk_norm* norm,
                                hia_tensor o, const float* lse, hia_tensor dout, hia_tensor dq, hia_tensor dk,
                                hia_tensor dv, float* dwq, float* dwk, void* ws, size_t ws_bytes, void* stream) {
+  return hia_attn_bwd_reuse_fwd(g, Hq, Hkv, D, q, k, v, c, s, scale, norm, o, lse, dout, dq, dk, dv, dwq, dwk,
+                                nullptr, 0, ws, ws_bytes, stream);
+}
+
+extern "C" int hia_attn_bwd_reuse_fwd(const hia_segments* g, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
+                                      hia_tensor v, const float* c, const float* s, float scale,
+                                      const hia_qk_norm* norm, hia_tensor o, const float* lse, hia_tensor dout,
+                                      hia_tensor dq, hia_tensor dk, hia_tensor dv, float* dwq, float* dwk,
+                                      const void* fws, size_t fws_bytes, void* ws, size_t ws_bytes,
+                                      void* stream) {
   int rc = check_common(g, Hq, Hkv, D, c, s);
   if (rc) return rc;
   if ((rc = check_norm(norm))) return rc;
@@ -398,12 +473,18 @@ extern "C" int hia_attn_bwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
   packed_view(g, {&q, &k, &v, &o, &dout, &dq, &dk, &dv});
   const BwdWs w = bwd_ws(g, Hq, Hkv, D);
   if (ws_bytes < w.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return HIA_ERR_INVALID_ARG;
+  const FwdWs fw = fwd_ws(g, Hq, Hkv, D);
+  if (fws && (fws_bytes < fw.total || (reinterpret_cast<uintptr_t>(fws) & 255)))
+    return HIA_ERR_INVALID_ARG;
   int* status = status_ptr();
   if (!status) return HIA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* wb = static_cast<char*>(ws);
-  __nv_bfloat16* qr = reinterpret_cast<__nv_bfloat16*>(wb + w.q_off);
-  __nv_bfloat16* kr = reinterpret_cast<__nv_bfloat16*>(wb + w.k_off);
+  // the rotated q and k: the forward's (reused as they are) or rotated here
+  __nv_bfloat16* qr = reinterpret_cast<__nv_bfloat16*>(
+      fws ? static_cast<char*>(const_cast<void*>(fws)) + fw.q_off : wb + w.q_off);
+  __nv_bfloat16* kr = reinterpret_cast<__nv_bfloat16*>(
+      fws ? static_cast<char*>(const_cast<void*>(fws)) + fw.k_off : wb + w.k_off);
   float* lse2 = reinterpret_cast<float*>(wb + w.lse_off);
   float* delta = reinterpret_cast<float*>(wb + w.delta_off);
   float* dq_acc = reinterpret_cast<float*>(wb + w.dq_off);
@@ -417,9 +498,7 @@ extern "C" int hia_attn_bwd_ex(const hia_segments* g, int Hq, int Hkv, int D, hi
       !make_q_map(&tdo, dout, D, gq, Hkv, map_rows(g), map_batches(g), 64))
     return HIA_ERR_CUDA;
 
-  rotate_into(q, Hq, gq, c, s, qr, g, D, st, norm ? norm->wq : nullptr, norm ? norm->eps : 0.f);
-  rotate_into(k, Hkv, 1, c, s, kr, g, D, st, norm ? norm->wk : nullptr, norm ? norm->eps : 0.f);
-  if (cudaMemsetAsync(dq_acc, 0, size_t(g->B) * Hq * S_pad * D * 4, st) != cudaSuccess) return HIA_ERR_CUDA;
+  if (!fws) rotate_qk(g, Hq, Hkv, D, q, k, c, s, norm, qr, kr, st);
 
   hia::BwdPreParams pp{};
   pp.o = static_cast<const __nv_bfloat16*>(o.ptr);

@@ -33,6 +33,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "devctx.h"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -455,49 +456,56 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // delta = rowsum(dO o O) and lse2 = lse * log2(e) for every (b, h, q < S_pad);
-// rows q >= S get delta 0 and lse2 +inf (so they contribute nothing).
+// rows q >= the sample's rows get delta 0 and lse2 +inf (so they contribute
+// nothing).  The same pass zeroes the fp32 dQ accumulator rows (b, h, q, :)
+// that the attention kernel reduce-adds into.  One warp per (b, q) row: a
+// lane group of D/8 lanes covers one head with 16-byte loads, so a warp
+// reads 256/D heads per step, several steps in flight.
+template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreParams p) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= p.B * p.S_pad) return;
+  constexpr int LPH = D / 8;        // lanes per head (16-byte chunks of 8 bf16)
+  constexpr int HPS = 32 / LPH;     // heads per step
+  const int lane = threadIdx.x & 31;
+  const int c = lane % LPH, hs = lane / LPH;
+  const unsigned gmask = (LPH == 32 ? 0xffffffffu : ((1u << LPH) - 1u)) << (hs * LPH);
+  // grid-stride over (b, q) rows: a fixed grid of resident warps
+  for (int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; warp < p.B * p.S_pad;
+       warp += (gridDim.x * blockDim.x) >> 5) {
   const int b = warp / p.S_pad, q = warp % p.S_pad;
-  const int per = p.D / 32;  // elements per lane: 4 (D=128) or 2 (D=64)
   const SampleDev t = p.samples[b];
-  for (int h = 0; h < p.Hq; ++h) {
+  const bool real = q < t.rows;  // beyond the sample's rows: padding past S, or past L when packed
+  const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int h = hs; h < p.Hq; h += HPS) {
     const int64_t orow = (int64_t(b) * p.Hq + h) * p.S_pad + q;
-    if (q >= t.rows) {  // beyond the sample's rows (padding past S, or past L when packed)
-      if (lane == 0) {
-        p.delta[orow] = 0.f;
-        p.lse2[orow] = INFINITY;
-      }
-      continue;
-    }
-    const __nv_bfloat16* o = p.o + int64_t(b) * p.o_sb + int64_t(t.off + q) * p.o_ss + int64_t(h / p.g) * p.o_shkv +
-                             int64_t(h % p.g) * p.o_shq;
-    const __nv_bfloat16* d = p.dout + int64_t(b) * p.d_sb + int64_t(t.off + q) * p.d_ss +
-                             int64_t(h / p.g) * p.d_shkv + int64_t(h % p.g) * p.d_shq;
-    float acc = 0.f;
-    if (per == 4) {
-      const uint2 ov = *reinterpret_cast<const uint2*>(o + lane * 4);
-      const uint2 dv = *reinterpret_cast<const uint2*>(d + lane * 4);
+    float4* acc = reinterpret_cast<float4*>(p.dq_acc + orow * D) + 2 * c;
+    acc[0] = z4;
+    acc[1] = z4;
+    float dot = 0.f;
+    if (real) {
+      const __nv_bfloat16* o = p.o + int64_t(b) * p.o_sb + int64_t(t.off + q) * p.o_ss +
+                               int64_t(h / p.g) * p.o_shkv + int64_t(h % p.g) * p.o_shq;
+      const __nv_bfloat16* d = p.dout + int64_t(b) * p.d_sb + int64_t(t.off + q) * p.d_ss +
+                               int64_t(h / p.g) * p.d_shkv + int64_t(h % p.g) * p.d_shq;
+      const uint4 ov = __ldg(reinterpret_cast<const uint4*>(o) + c);
+      const uint4 dv = __ldg(reinterpret_cast<const uint4*>(d) + c);
       const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
       const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const float2 a = __bfloat1622float2(o2[i]), c = __bfloat1622float2(d2[i]);
-        acc = fmaf(a.x, c.x, acc);
-        acc = fmaf(a.y, c.y, acc);
+      for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(o2[i]), y = __bfloat1622float2(d2[i]);
+        dot = fmaf(x.x, y.x, dot);
+        dot = fmaf(x.y, y.y, dot);
       }
-    } else {
-      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + lane * 2));
-      const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(d + lane * 2));
-      acc = fmaf(a.x, c.x, a.y * c.y);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      p.delta[orow] = acc;
-      p.lse2[orow] = p.lse[int64_t(b) * p.lse_sb + int64_t(h) * p.lse_sh + t.off + q] * 1.4426950408889634f;
+    for (int off = LPH / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(gmask, dot, off);
+    if (c == 0) {
+      p.delta[orow] = real ? dot : 0.f;
+      p.lse2[orow] = real ? p.lse[int64_t(b) * p.lse_sb + int64_t(h) * p.lse_sh + t.off + q] * 1.4426950408889634f
+                          : INFINITY;
     }
+  }
   }
 }
 
@@ -507,7 +515,11 @@ cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st) {
   const int64_t warps = int64_t(p.B) * p.S_pad;
   if (warps == 0) return cudaSuccess;
   prof_begin(kBwdPre, st);
-  bwd_pre_kernel<<<int((warps + 7) / 8), 256, 0, st>>>(p);
+  const int blocks = int(warps < 148 * 64 ? (warps + 7) / 8 : 148 * 8);  // grid-stride beyond 8 blocks per SM
+  if (p.D == 128)
+    bwd_pre_kernel<128><<<blocks, 256, 0, st>>>(p);
+  else
+    bwd_pre_kernel<64><<<blocks, 256, 0, st>>>(p);
   prof_end(kBwdPre, st);
   return cudaGetLastError();
 }
@@ -515,21 +527,29 @@ cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st) {
 cudaError_t launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const BwdParams& p, int n_blocks, int D, cudaStream_t st) {
   if (n_blocks == 0) return cudaSuccess;
-  cudaFuncAttributes fa{};
-  if (cudaFuncGetAttributes(&fa, D == 128 ? attn_bwd_kernel<128> : attn_bwd_kernel<64>) != cudaSuccess ||
-      fa.numRegs != kLaunchRegs)
-    return cudaErrorInvalidConfiguration;
+  static_assert(sizeof(BwdSmem<128>) + 1024 <= 232448, "shared memory budget");
+  const size_t smem = D == 128 ? sizeof(BwdSmem<128>) + 1024 : sizeof(BwdSmem<64>) + 1024;
+  const void* fn = D == 128 ? reinterpret_cast<const void*>(attn_bwd_kernel<128>)
+                            : reinterpret_cast<const void*>(attn_bwd_kernel<64>);
+  // once per device and context: the compiled register count (the setmaxnreg
+  // split assumes kLaunchRegs) and the dynamic shared-memory opt-in
+  static PerContext<int> ready[2];
+  int ok = 0;
+  const cudaError_t e = ready[D == 128].get(&ok, [&](int* out) {
+    cudaFuncAttributes fa{};
+    cudaError_t r = cudaFuncGetAttributes(&fa, fn);
+    if (r != cudaSuccess) return r;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    *out = 1;
+    return r;
+  });
+  if (e != cudaSuccess) return e;
   prof_begin(kAttnBwd, st);
-  if (D == 128) {
-    static_assert(sizeof(BwdSmem<128>) + 1024 <= 232448, "shared memory budget");
-    const size_t smem = sizeof(BwdSmem<128>) + 1024;
-    cudaFuncSetAttribute(attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (D == 128)
     attn_bwd_kernel<128><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, tdo, p);
-  } else {
-    const size_t smem = sizeof(BwdSmem<64>) + 1024;
-    cudaFuncSetAttribute(attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  else
     attn_bwd_kernel<64><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, tdo, p);
-  }
   prof_end(kAttnBwd, st);
   return cudaGetLastError();
 }

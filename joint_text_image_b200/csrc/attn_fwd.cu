@@ -26,6 +26,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "devctx.h"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -329,9 +330,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (have) have = __all_sync(0xffffffffu, mbar_wait(&sm.bar_o_final[t], 0, wc));
       if (have) tc_fence_after();
       const bool store = q < smp.rows;
-      __nv_bfloat16* orow = p.o + int64_t(b) * p.o_sb + int64_t(smp.off + q) * p.o_ss + int64_t(h / p.g) * p.o_shkv +
-                            int64_t(h % p.g) * p.o_shq;
       const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
+      // O / l -> bf16 rows staged in this tile's Q buffer (every MMA has
+      // finished, so Q is no longer read), 16-byte chunks XOR-swizzled by row
+      // so that a warp's 32 row writes hit distinct banks; then each warp
+      // writes its own 32 rows whole: CPR lanes per row, 16 bytes each, so a
+      // warp store covers 32 / CPR complete rows (coalesced 128-bit stores).
+      constexpr int CPR = D / 8;  // 16-byte chunks per row
+      uint8_t* tile = reinterpret_cast<uint8_t*>(sm.q[t]);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -342,14 +348,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = 0u;
         }
-        if (store) {
-          uint32_t pk[16];
+        uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        for (int i = 0; i < 4; ++i) {
+          const int ch = (c * 4 + i) ^ (r & (CPR - 1));
+          *reinterpret_cast<uint4*>(tile + r * (D * 2) + ch * 16) =
+              make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      __syncwarp();
+      {
+        constexpr int RPI = 32 / CPR;  // rows per warp store
+        const int ch = lane % CPR;
+        const int64_t head_off = int64_t(b) * p.o_sb + int64_t(h / p.g) * p.o_shkv + int64_t(h % p.g) * p.o_shq;
+#pragma unroll 4
+        for (int rr = 0; rr < 32; rr += RPI) {
+          const int row = quarter * 32 + rr + lane / CPR;
+          const int qrow = qt * 128 + row;
+          if (qrow < smp.rows) {
+            const uint4 v = *reinterpret_cast<const uint4*>(tile + row * (D * 2) + ((ch ^ (row & (CPR - 1))) * 16));
+            *reinterpret_cast<uint4*>(p.o + head_off + int64_t(smp.off + qrow) * p.o_ss + ch * 8) = v;
+          }
         }
       }
       if (store)
@@ -372,21 +394,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, int n_blocks, int D, cudaStream_t st) {
   if (n_blocks == 0) return cudaSuccess;
-  cudaFuncAttributes fa{};
-  if (cudaFuncGetAttributes(&fa, D == 128 ? attn_fwd_kernel<128> : attn_fwd_kernel<64>) != cudaSuccess ||
-      fa.numRegs != kLaunchRegs)
-    return cudaErrorInvalidConfiguration;  // the setmaxnreg split assumes kLaunchRegs
+  static_assert(sizeof(FwdSmem<128>) + 1024 <= 232448, "shared memory budget");
+  const size_t smem = D == 128 ? sizeof(FwdSmem<128>) + 1024 : sizeof(FwdSmem<64>) + 1024;
+  const void* fn = D == 128 ? reinterpret_cast<const void*>(attn_fwd_kernel<128>)
+                            : reinterpret_cast<const void*>(attn_fwd_kernel<64>);
+  // once per device and context: the compiled register count (the setmaxnreg
+  // split assumes kLaunchRegs) and the dynamic shared-memory opt-in
+  static PerContext<int> ready[2];
+  int ok = 0;
+  const cudaError_t e = ready[D == 128].get(&ok, [&](int* out) {
+    cudaFuncAttributes fa{};
+    cudaError_t r = cudaFuncGetAttributes(&fa, fn);
+    if (r != cudaSuccess) return r;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    *out = 1;
+    return r;
+  });
+  if (e != cudaSuccess) return e;
   prof_begin(kAttnFwd, st);
-  if (D == 128) {
-    static_assert(sizeof(FwdSmem<128>) + 1024 <= 232448, "shared memory budget");
-    const size_t smem = sizeof(FwdSmem<128>) + 1024;
-    cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (D == 128)
     attn_fwd_kernel<128><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, p);
-  } else {
-    const size_t smem = sizeof(FwdSmem<64>) + 1024;
-    cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  else
     attn_fwd_kernel<64><<<n_blocks, kThreads, smem, st>>>(tq, tk, tv, p);
-  }
   prof_end(kAttnFwd, st);
   return cudaGetLastError();
 }

@@ -12,12 +12,12 @@
 // The array is a file-scope __device__ variable of kScratchBytes (64 MiB).
 // Every GPU that loads this part of the library holds it until the process
 // exits.  In host code its name is only a host-side stand-in, so the device
-// address is looked up once per device with cudaGetSymbolAddress (with that
-// device current) and passed to the kernels.
+// address is looked up with cudaGetSymbolAddress (with the device current)
+// and passed to the kernels: once per device, and again if the device's
+// context has been replaced (after cudaDeviceReset the old address is stale).
 #include <cuda_runtime.h>
 
-#include <mutex>
-
+#include "devctx.h"
 #include "kernels.h"
 
 namespace {
@@ -26,25 +26,14 @@ constexpr size_t kScratchBytes = size_t(64) << 20;  // 64 MiB
 
 static __device__ __align__(256) unsigned char g_fwd_scratch[kScratchBytes];
 
-// Device address of g_fwd_scratch on the current device, looked up once per
-// device.  The first lookup on a device also loads the module that holds the
-// array, which is why the first call on each device should come before any
-// stream capture.
+// Device address of g_fwd_scratch in the current device's context.  The
+// first lookup in a context also loads the module that holds the array,
+// which is why the first call on each device should come before any stream
+// capture.
 int scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return HIA_ERR_CUDA;
-  static std::mutex mu;
-  static void* addr[64] = {};
-  if (dev >= 64) return HIA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_fwd_scratch);
-    if (e != cudaSuccess || !p) return HIA_ERR_CUDA;
-    addr[dev] = p;
-  }
-  *out = addr[dev];
-  return HIA_OK;
+  static hia::PerContext<void*> cache;
+  const cudaError_t e = cache.get(out, [](void** p) { return cudaGetSymbolAddress(p, g_fwd_scratch); });
+  return (e == cudaSuccess && *out) ? HIA_OK : HIA_ERR_CUDA;
 }
 
 }  // namespace
@@ -52,12 +41,15 @@ int scratch_address(void** out) {
 extern "C" int hia_attn_fwd_noalloc(const hia_segments* seg, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
                                     hia_tensor v, const float* cos_t, const float* sin_t, float scale,
                                     hia_tensor o, float* lse, void* stream) {
-  if (!seg || Hq <= 0 || Hkv <= 0 || D <= 0) return HIA_ERR_INVALID_ARG;
-  // The scratch holds the rotated q and k: B*S*(Hq+Hkv)*D bf16 values.
+  // The same argument checks as hia_attn_fwd, in the same order, before the
+  // size limit: a bad argument reports its own error.
+  int rc = hia::fwd_check_args(seg, Hq, Hkv, D, q, k, v, cos_t, sin_t, scale, nullptr, o, lse);
+  if (rc != HIA_OK) return rc;
+  if (seg->B == 0 || seg->S == 0) return HIA_OK;
+  // The scratch holds the rotated q and k (hia_attn_fwd's workspace).
   if (hia_attn_fwd_workspace_bytes(seg, Hq, Hkv, D) > kScratchBytes) return HIA_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
-  const int rc = scratch_address(&scratch);
-  if (rc != HIA_OK) return rc;
+  if ((rc = scratch_address(&scratch)) != HIA_OK) return rc;
   // Nothing in the scratch has to start at zero: the rotation pass rewrites
   // every element the attention kernel reads.  Calls share the array, so two
   // calls whose work overlaps on the GPU (different streams, or different

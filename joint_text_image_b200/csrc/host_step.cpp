@@ -149,8 +149,10 @@ extern "C" int hia_attn_step_host(hia_step* st, const void* q, const void* k, co
   if (rc == HIA_OK) rc = cuda_ok(cudaMemcpyAsync(lse, st->lse, st->lse_bytes, cudaMemcpyDeviceToHost, c));
   if (rc == HIA_OK) rc = cuda_ok(cudaStreamWaitEvent(s, st->ev_dout, 0));
   if (rc == HIA_OK)
-    rc = hia_attn_bwd(seg, Hq, Hkv, D, tq, tk, tv, st->cos_t, st->sin_t, scale, to, st->lse, tdo, tdq, tdk, tdv,
-                      st->ws_bwd, st->ws_bwd_bytes, s);
+    // the backward reads the rotated q and k the forward left in its workspace
+    rc = hia_attn_bwd_reuse_fwd(seg, Hq, Hkv, D, tq, tk, tv, st->cos_t, st->sin_t, scale, nullptr, to, st->lse,
+                                tdo, tdq, tdk, tdv, nullptr, nullptr, st->ws_fwd, st->ws_fwd_bytes, st->ws_bwd,
+                                st->ws_bwd_bytes, s);
   if (rc == HIA_OK) rc = cuda_ok(cudaMemcpyAsync(dq, st->dq, st->q_bytes, cudaMemcpyDeviceToHost, s));
   if (rc == HIA_OK) rc = cuda_ok(cudaMemcpyAsync(dk, st->dk, st->kv_bytes, cudaMemcpyDeviceToHost, s));
   if (rc == HIA_OK) rc = cuda_ok(cudaMemcpyAsync(dv, st->dv, st->kv_bytes, cudaMemcpyDeviceToHost, s));

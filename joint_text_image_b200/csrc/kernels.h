@@ -8,17 +8,25 @@
 
 namespace hia {
 
-struct RotateArgs {
-  const SampleDev* samples;  // rows / off of every sample (layout of src)
+// One tensor of the rotation pre-pass: src rows rotated (and optionally
+// RMS-normed) into dst.
+struct RotatePart {
   const void* src;  // bf16 [B,S,heads,D] with strides (elements)
   int64_t src_sb, src_ss, src_shkv, src_shq;
   int g;            // heads per stride_hkv group (1 for k)
-  const float* cos_t;
-  const float* sin_t;
+  int H;            // heads
   const float* w;   // QK RMSNorm weight [D], or nullptr: no norm
   float eps;
   __nv_bfloat16* dst;  // [B][H][S][D]
-  int B, S, H;
+};
+
+struct RotateArgs {
+  const SampleDev* samples;  // rows / off of every sample (layout of src)
+  const float* cos_t;
+  const float* sin_t;
+  RotatePart part[2];        // q and k, rotated by one launch
+  int n_parts;
+  int B, S;
 };
 
 struct GradFinalArgs {
@@ -66,7 +74,7 @@ struct BwdPreParams {
   int64_t lse_sb, lse_sh;
   float* lse2;          // [B][Hq][S_pad]: lse * log2(e); +inf beyond S
   float* delta;         // [B][Hq][S_pad]: rowsum(dout * o); 0 beyond S
-  float* dq_acc;        // [B][Hq][S_pad][D] zeroed
+  float* dq_acc;        // [B][Hq][S_pad][D]: zeroed by this pass
   int B, S, S_pad, Hq, g, D;
 };
 
@@ -93,8 +101,22 @@ struct BwdParams {
   uint64_t timeout_ns;
 };
 
+// 2D bf16 tensor map [rows][cols] (row stride in bytes, a multiple of 16),
+// 128-byte swizzle, box box_rows x box_cols (box_cols * 2 = 128 bytes).
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t row_stride_bytes,
+                 uint32_t box_cols, uint32_t box_rows);
+
+// Host-side argument checks of the forward (everything but the workspace):
+// HIA_OK, or the status hia_attn_fwd_ex would return for these arguments.
+int fwd_check_args(const hia_segments* g, int Hq, int Hkv, int D, const hia_tensor& q, const hia_tensor& k,
+                   const hia_tensor& v, const float* c, const float* s, float scale, const hia_qk_norm* norm,
+                   const hia_tensor& o, const float* lse);
+
 // Profiling brackets around one kernel launch (no-ops unless profiling is on).
-enum KernelId { kRopeTables = 0, kRopeRotate, kAttnFwd, kBwdPre, kAttnBwd, kGradFinalize, kDwReduce, kNumKernels };
+enum KernelId {
+  kRopeTables = 0, kRopeRotate, kAttnFwd, kBwdPre, kAttnBwd, kGradFinalize, kDwReduce,
+  kMoePrep, kMoeRouter, kMoeScan, kMoeGather, kMoeUpGate, kMoeDown, kMoeCombine, kNumKernels
+};
 void prof_begin(KernelId id, cudaStream_t st);
 void prof_end(KernelId id, cudaStream_t st);
 

@@ -10,8 +10,10 @@
 
 namespace {
 
-const char* kNames[hia::kNumKernels] = {"rope2d_tables", "rope_rotate", "attn_fwd",
-                                        "bwd_pre", "attn_bwd", "grad_finalize", "dw_reduce"};
+const char* kNames[hia::kNumKernels] = {"rope2d_tables", "rope_rotate", "attn_fwd",  "bwd_pre",
+                                        "attn_bwd",      "grad_finalize", "dw_reduce", "moe_prep",
+                                        "moe_router",    "moe_scan",    "moe_gather", "moe_up_gate",
+                                        "moe_down",      "moe_combine"};
 
 struct Rec {
   int id;

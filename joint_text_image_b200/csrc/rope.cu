@@ -11,17 +11,25 @@
 // [-v[D/2:], v[:D/2]].
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "kernels.h"
 
 namespace hia {
 
 // K1: one thread per (b, n, j < D/2).  Angle and cos/sin in fp64, rounded
-// once to fp32: a text-only sample reproduces the 1D tables exactly.
-__global__ void rope2d_tables_kernel(const SampleDev* __restrict__ samples, const ImageDev* __restrict__ images,
-                                     int B, int S, int D, double base, float* __restrict__ cos_out,
-                                     float* __restrict__ sin_out) {
+// once to fp32: a text-only sample reproduces the 1D tables exactly.  The
+// frequencies theta_j = base^(-2j/D) depend on j only: each block evaluates
+// them once into shared memory.
+__global__ void __launch_bounds__(256) rope2d_tables_kernel(const SampleDev* __restrict__ samples,
+                                                            const ImageDev* __restrict__ images, int B, int S, int D,
+                                                            double base, float* __restrict__ cos_out,
+                                                            float* __restrict__ sin_out) {
+  __shared__ double theta_s[128];
   const int half = D / 2;
+  for (int j = threadIdx.x; j < half; j += blockDim.x) theta_s[j] = pow(base, -2.0 * double(j) / double(D));
+  __syncthreads();
   const int64_t total = int64_t(B) * S * half;
   for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
        idx += int64_t(gridDim.x) * blockDim.x) {
@@ -38,8 +46,7 @@ __global__ void rope2d_tables_kernel(const SampleDev* __restrict__ samples, cons
       x = double(g.I0 + i % g.w);
       y = double(g.I0 + i / g.w);
     }
-    const double theta = pow(base, -2.0 * double(j) / double(D));
-    const double a = ((j & 1) ? y : x) * theta;
+    const double a = ((j & 1) ? y : x) * theta_s[j];
     double sn, cs;
     sincos(a, &sn, &cs);
     const int64_t o = bn * D + j;
@@ -96,34 +103,21 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8]) {
 }
 
 // Rotation pre-pass: dst[b][h][s][:] = R(b,s) src[b,s,h,:] in fp32, rounded
-// to bf16.  With QK RMSNorm weights (a.w != nullptr) the rotated row x is
-// replaced by w * x / sqrt(mean(x^2) + eps) before the rounding
-// (HunyuanImage3Attention applies RoPE, then the per-head QK RMSNorm).  The
-// cos/sin of the row are read once and reused for every head.
-template <int D>
-__global__ void __launch_bounds__(256) rope_rotate_kernel(RotateArgs a) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= a.B * a.S) return;
-  const int b = warp / a.S, s = warp % a.S;
-  const RowLanes<D> L(lane);
-  const SampleDev t = a.samples[b];
-  if (s >= t.rows) {  // packed layout: the sample has no row s; keep the slab finite
-    for (int h = L.hs; h < a.H; h += RowLanes<D>::HPI) {
-      __nv_bfloat16* dst = a.dst + ((int64_t(b) * a.H + h) * a.S + s) * D;
-      *reinterpret_cast<uint4*>(dst + L.c * 8) = make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(dst + D / 2 + L.c * 8) = make_uint4(0, 0, 0, 0);
-    }
-    return;
-  }
-  float cs[8], sn[8], wl[8], wh[8];
-  load8(a.cos_t + (int64_t(b) * a.S + s) * D + L.c * 8, cs);
-  load8(a.sin_t + (int64_t(b) * a.S + s) * D + L.c * 8, sn);
-  const bool norm = a.w != nullptr;
+// to bf16, for q and k in one launch.  With QK RMSNorm weights (w != nullptr)
+// the rotated row x is replaced by w * x / sqrt(mean(x^2) + eps) before the
+// rounding (HunyuanImage3Attention applies RoPE, then the per-head QK
+// RMSNorm).  A warp owns one (b, s) row: the cos/sin of the row are read once
+// and reused for every head of both tensors.
+template <int D, bool NORM>
+__device__ __forceinline__ void rotate_part(const RotatePart& a, const RowLanes<D>& L, int b, int s, int S,
+                                            const SampleDev& t, const float (&cs)[8], const float (&sn)[8]) {
+  constexpr bool norm = NORM;
+  float wl[8], wh[8];
   if (norm) {
     load8(a.w + L.c * 8, wl);
     load8(a.w + D / 2 + L.c * 8, wh);
   }
+#pragma unroll 2
   for (int h = L.hs; h < a.H; h += RowLanes<D>::HPI) {
     const int64_t so = int64_t(b) * a.src_sb + int64_t(t.off + s) * a.src_ss + int64_t(h / a.g) * a.src_shkv +
                        int64_t(h % a.g) * a.src_shq;
@@ -147,9 +141,38 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(RotateArgs a) {
         xu[k] = wh[k] * (xu[k] * r);
       }
     }
-    __nv_bfloat16* dst = a.dst + ((int64_t(b) * a.H + h) * a.S + s) * D;
+    __nv_bfloat16* dst = a.dst + ((int64_t(b) * a.H + h) * S + s) * D;
     *reinterpret_cast<uint4*>(dst + L.c * 8) = pack8_bf16(xl);
     *reinterpret_cast<uint4*>(dst + D / 2 + L.c * 8) = pack8_bf16(xu);
+  }
+}
+
+// NORM: the QK RMSNorm is applied (every part has weights); a separate
+// instantiation keeps the plain rotation's register budget small.
+template <int D, bool NORM>
+__global__ void __launch_bounds__(256, NORM ? 2 : 3) rope_rotate_kernel(RotateArgs a) {
+  const int lane = threadIdx.x & 31;
+  const RowLanes<D> L(lane);
+  const int n_rows = a.B * a.S;
+  // grid-stride over (b, s) rows: a fixed grid of resident warps, no partial last wave
+  for (int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; warp < n_rows; warp += (gridDim.x * blockDim.x) >> 5) {
+    const int b = warp / a.S, s = warp % a.S;
+    const SampleDev t = a.samples[b];
+    if (s >= t.rows) {  // packed layout: the sample has no row s; keep the slab finite
+      for (int p = 0; p < a.n_parts; ++p)
+        for (int h = L.hs; h < a.part[p].H; h += RowLanes<D>::HPI) {
+          __nv_bfloat16* dst = a.part[p].dst + ((int64_t(b) * a.part[p].H + h) * a.S + s) * D;
+          *reinterpret_cast<uint4*>(dst + L.c * 8) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(dst + D / 2 + L.c * 8) = make_uint4(0, 0, 0, 0);
+        }
+      continue;
+    }
+    float cs[8], sn[8];
+    load8(a.cos_t + (int64_t(b) * a.S + s) * D + L.c * 8, cs);
+    load8(a.sin_t + (int64_t(b) * a.S + s) * D + L.c * 8, sn);
+#pragma unroll
+    for (int p = 0; p < 2; ++p)
+      if (p < a.n_parts) rotate_part<D, NORM>(a.part[p], L, b, s, a.S, t, cs, sn);
   }
 }
 
@@ -160,19 +183,21 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(RotateArgs a) {
 // with respect to x is r (w v - xh <w v, xh> / D), then R^T; the weight
 // gradient w += v * xh is summed per block into dw_part[blockIdx.x][:] in a
 // fixed order (deterministic), and dw_reduce_kernel adds the blocks.
-template <int D>
-__global__ void __launch_bounds__(256) grad_finalize_kernel(GradFinalArgs a) {
+template <int D, bool NORM>
+__global__ void __launch_bounds__(256, NORM ? 2 : 4) grad_finalize_kernel(GradFinalArgs a) {
   constexpr int CPH = RowLanes<D>::CPH, HPI = RowLanes<D>::HPI;
   __shared__ float red[8][32][16];
   const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int warp = blockIdx.x * 8 + wib;
   const RowLanes<D> L(lane);
-  const bool norm = a.w != nullptr;
+  constexpr bool norm = NORM;
   float dwl[8], dwh[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) dwl[k] = dwh[k] = 0.f;
-  const int b = warp / max(a.S, 1), s = warp % max(a.S, 1);
-  if (warp < a.B * a.S && s < a.samples[b].rows) {
+  // grid-stride over (b, s) rows; which rows a block takes depends only on
+  // (B, S), so its weight-gradient partial is summed in a fixed order
+  for (int warp = blockIdx.x * 8 + wib; warp < a.B * a.S; warp += gridDim.x * 8) {
+  const int b = warp / a.S, s = warp % a.S;
+  if (s < a.samples[b].rows) {
     const int off = a.samples[b].off;
     float cs[8], sn[8], wl[8], wh[8];
     load8(a.cos_t + (int64_t(b) * a.S + s) * D + L.c * 8, cs);
@@ -239,6 +264,7 @@ __global__ void __launch_bounds__(256) grad_finalize_kernel(GradFinalArgs a) {
       *reinterpret_cast<uint4*>(dst + D / 2 + L.c * 8) = pack8_bf16(ou);
     }
   }
+  }
   if (!norm) return;  // uniform across the block
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -274,13 +300,18 @@ __global__ void __launch_bounds__(1024) dw_reduce_kernel(const float* __restrict
   if (ry == 0 && d < D) dw[d] = t[0][cx];
 }
 
+// Blocks of the row-per-warp kernels: 8 warps each, one warp per row (the
+// kernels' grid-stride loops then run once; the hardware block scheduler
+// balances the rows).
+int row_grid_blocks(int64_t rows) { return int((rows + 7) / 8); }
+
 void launch_rope2d_tables(const SampleDev* samples, const ImageDev* images, int B, int S, int D, double base,
                           float* cos_out, float* sin_out, cudaStream_t st) {
   const int64_t total = int64_t(B) * S * (D / 2);
   if (total == 0) return;
   const int threads = 256;
   int64_t blocks = (total + threads - 1) / threads;
-  if (blocks > 148 * 64) blocks = 148 * 64;
+  if (blocks > 148 * 8) blocks = 148 * 8;
   prof_begin(kRopeTables, st);
   rope2d_tables_kernel<<<int(blocks), threads, 0, st>>>(samples, images, B, S, D, base, cos_out, sin_out);
   prof_end(kRopeTables, st);
@@ -289,21 +320,33 @@ void launch_rope2d_tables(const SampleDev* samples, const ImageDev* images, int 
 void launch_rope_rotate(const RotateArgs& a, int D, cudaStream_t st) {
   const int64_t warps = int64_t(a.B) * a.S;
   if (warps == 0) return;
-  const int blocks = int((warps + 7) / 8);
+  const int blocks = row_grid_blocks(warps);
   prof_begin(kRopeRotate, st);
-  if (D == 128) rope_rotate_kernel<128><<<blocks, 256, 0, st>>>(a);
-  else rope_rotate_kernel<64><<<blocks, 256, 0, st>>>(a);
+  const bool norm = a.part[0].w != nullptr;
+  if (D == 128) {
+    if (norm) rope_rotate_kernel<128, true><<<blocks, 256, 0, st>>>(a);
+    else rope_rotate_kernel<128, false><<<blocks, 256, 0, st>>>(a);
+  } else {
+    if (norm) rope_rotate_kernel<64, true><<<blocks, 256, 0, st>>>(a);
+    else rope_rotate_kernel<64, false><<<blocks, 256, 0, st>>>(a);
+  }
   prof_end(kRopeRotate, st);
 }
 
-int grad_finalize_blocks(int B, int S) { return int((int64_t(B) * S + 7) / 8); }
+int grad_finalize_blocks(int B, int S) { return row_grid_blocks(int64_t(B) * S); }
 
 void launch_grad_finalize(const GradFinalArgs& a, int D, cudaStream_t st) {
   const int blocks = grad_finalize_blocks(a.B, a.S);
   if (blocks == 0) return;
   prof_begin(kGradFinalize, st);
-  if (D == 128) grad_finalize_kernel<128><<<blocks, 256, 0, st>>>(a);
-  else grad_finalize_kernel<64><<<blocks, 256, 0, st>>>(a);
+  const bool norm = a.w != nullptr;
+  if (D == 128) {
+    if (norm) grad_finalize_kernel<128, true><<<blocks, 256, 0, st>>>(a);
+    else grad_finalize_kernel<128, false><<<blocks, 256, 0, st>>>(a);
+  } else {
+    if (norm) grad_finalize_kernel<64, true><<<blocks, 256, 0, st>>>(a);
+    else grad_finalize_kernel<64, false><<<blocks, 256, 0, st>>>(a);
+  }
   prof_end(kGradFinalize, st);
 }
 

@@ -112,3 +112,59 @@ def custom(samples, Hq, Hkv, D, S=None, name="custom") -> Workload:
     if S is not None:
         wl.S = S
     return wl
+
+
+# ---------------------------------------------------------------- MoE feed-forward
+@dataclass
+class MoeWorkload:
+    """Sizes of one MoE feed-forward call: T tokens, hidden H, expert
+    intermediate I, E routed experts of which topk per token, plus the shared
+    expert.  The pages fix E = 64 and topk = 8 (technical report summary
+    3.1.1); they give neither H nor I: H = 4096 is the attention's 32 heads x
+    128, and I = 3072 is a reading (with 32 layers it matches both the 80B
+    total and the 13B active parameters the pages quote)."""
+    name: str
+    T: int
+    H: int
+    I: int
+    E: int
+    topk: int
+    note: str = ""
+
+
+def moe_workload(name: str, seed: int = 0) -> MoeWorkload:
+    if name == "moe_tiny":
+        return MoeWorkload(name, 300, 256, 128, 8, 2, note="every shape one or two tiles, ragged token count")
+    if name == "moe_mid":
+        return MoeWorkload(name, 1000, 512, 256, 64, 8, note="the pages' routing (64 experts, top-8), small dims")
+    if name == "moe_e16":
+        # the benchmark's H and I with 16 experts, top-4, 4096 tokens: 1.3 GB of
+        # weights (still well above L2), small enough for a full profiler capture
+        return MoeWorkload(name, 4096, 4096, 3072, 16, 4, note="profiling size: bench dims, fewer experts")
+    if name == "moe_1024px":
+        # the valid tokens of the 1024px attention workload's batch (two
+        # samples: prefix + 64x64 image + 2 suffix tokens each), packed
+        wl = workload("1024px", seed)
+        T = sum(p + h * w + s for (p, h, w, s) in wl.samples)
+        return MoeWorkload(name, T, 4096, 3072, 64, 8, note="tokens of the 1024px batch, packed")
+    raise KeyError(name)
+
+
+MOE_WORKLOADS = ("moe_tiny", "moe_mid", "moe_e16", "moe_1024px")
+
+
+def moe_tensors(mw: MoeWorkload, seed: int = 0):
+    """x bf16 [T, H] ~ N(0, 1) (the block's RMS-normed hidden states have unit
+    RMS); router weight fp32 [E, H] ~ N(0, 1/H), so logits ~ N(0, 1); w13 bf16
+    [E + 1, 2I, H] ~ N(0, 1/H) and w2 bf16 [E + 1, H, I] ~ N(0, 1/I) (index E:
+    the shared expert), so every projection keeps unit scale.  CPU tensors
+    from a seeded generator, one expert at a time."""
+    gen = torch.Generator().manual_seed(seed + 101)
+    x = torch.randn(mw.T, mw.H, generator=gen).to(torch.bfloat16)
+    wg = torch.randn(mw.E, mw.H, generator=gen) * mw.H ** -0.5
+    w13 = torch.empty(mw.E + 1, 2 * mw.I, mw.H, dtype=torch.bfloat16)
+    w2 = torch.empty(mw.E + 1, mw.H, mw.I, dtype=torch.bfloat16)
+    for e in range(mw.E + 1):
+        w13[e] = (torch.randn(2 * mw.I, mw.H, generator=gen) * mw.H ** -0.5).to(torch.bfloat16)
+        w2[e] = (torch.randn(mw.H, mw.I, generator=gen) * mw.I ** -0.5).to(torch.bfloat16)
+    return x, wg, w13, w2

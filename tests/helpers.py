@@ -15,6 +15,17 @@ from joint_text_image_b200 import synth
 # of the score errors, stays within max_k |ds_k|: ~4.5 std over the 10^6-10^7
 # rows checked gives 7e-3, so max-abs 1e-2 and mean-abs 1e-3.
 O_MAX, O_MEAN, LSE_MAX, LSE_MEAN, GRAD_REL = 2e-2, 2e-3, 1e-2, 1e-3, 1e-2
+# The relative Frobenius bound above is over whole tensors, where an error
+# confined to one tile (a tail tile, a partial image edge) adds only a small
+# share of the norm.  Every block is therefore also checked on its own: each
+# 128-row block of dq (per sample and kv-head group of g heads) and each
+# 128-key block of dk and dv (per sample and kv head), bound 2e-2.  The
+# measured whole-tensor error is ~3.6e-3 and the bf16 rounding of the
+# operands is uniform over blocks, so a block-local bug is what breaks it.
+# A block whose reference is exactly zero (padded keys; a one-token sample,
+# whose dq cancels exactly) takes the absolute form of the whole-tensor rule:
+# its norm must stay within the bound.
+GRAD_BLOCK_REL, GRAD_BLOCK = 2e-2, 128
 
 
 def gpu_tables(seg, D, base=10000.0):
@@ -121,12 +132,33 @@ def check_bwd(oracle_mod, wl, inputs, grads, groups=None, qk_norm=None, dw=None)
                 if gsel[b, hk]:
                     a.append(got[b, :, hk * per:(hk + 1) * per])
                     bref.append(r[b, :, hk * per:(hk + 1) * per])
+        worst = check_blocks(name, a, bref)
         a = np.concatenate([x.ravel() for x in a])
         bref = np.concatenate([x.ravel() for x in bref])
         assert np.all(np.isfinite(a)), f"{name} non-finite"
         nr = np.linalg.norm(bref)
         rel = np.linalg.norm(a - bref) / nr if nr > 0 else np.linalg.norm(a)
         out[name] = rel
+        out[name + "_worst_block"] = worst
         assert rel <= GRAD_REL, f"{name} relative Frobenius {rel:.3e}"
     print(f"[parity-bwd] {wl.name}: " + " ".join(f"{k} {v:.3e}" for k, v in out.items()))
     return out
+
+
+def check_blocks(name, got, ref, block=GRAD_BLOCK, bound=GRAD_BLOCK_REL):
+    """Relative Frobenius error of every `block`-row slice of each [S, heads, D]
+    array pair in got / ref (lists); returns the worst one."""
+    worst = 0.0
+    for i, (a, r) in enumerate(zip(got, ref)):
+        S = r.shape[0]
+        for r0 in range(0, S, block):
+            ab = np.asarray(a[r0:r0 + block], dtype=np.float64)
+            rb = r[r0:r0 + block]
+            nr = np.linalg.norm(rb)
+            if nr == 0:
+                assert np.linalg.norm(ab) <= bound, f"{name}: block {i}/{r0} should be zero"
+                continue
+            rel = np.linalg.norm(ab - rb) / nr
+            assert rel <= bound, f"{name}: block {i} rows [{r0}, {r0 + block}) relative Frobenius {rel:.3e}"
+            worst = max(worst, rel)
+    return worst

@@ -18,10 +18,16 @@ def built():
     jbuild.build()
 
 
+HEADERS = ("jointattn.h", "jointmoe.h")
+
+
 def declared_symbols():
-    txt = open(os.path.join(ROOT, "include", "jointattn.h")).read()
-    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    return sorted(set(re.findall(r"\b(hia_\w+)\s*\(", txt)))
+    names = set()
+    for h in HEADERS:
+        txt = open(os.path.join(ROOT, "include", h)).read()
+        txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+        names.update(re.findall(r"\b(hia_\w+)\s*\(", txt))
+    return sorted(names)
 
 
 def test_exports_every_declared_symbol():
@@ -119,3 +125,30 @@ def test_fwd_rejects_unsupported_without_launch():
     assert L.hia_attn_fwd(seg.handle, 4, 1, 64, z, z, z, p, p, 1.0, z, None, None, 0, None) == 5
     assert L.hia_rope2d_tables(seg.handle, 63, 10000.0, p, p, None) == 1
     assert L.hia_debug_wait_timeout(0, None) == 1
+
+
+@pytest.mark.parametrize("dims", [
+    (100, 300, 128, 8, 2),     # H not a multiple of 256
+    (100, 256, 100, 8, 2),     # I not a multiple of 128
+    (100, 256, 128, 81, 2),    # E above 80
+    (100, 256, 128, 8, 9),     # topk above E
+    (100, 256, 128, 64, 17),   # topk above 16
+    (-1, 256, 128, 8, 2),      # negative T
+    (100, 256, 128, 0, 1),     # no routed expert
+])
+def test_moe_bad_dims_rejected(dims):
+    """Host-side validation of the MoE sizes: no workspace size, and the
+    forward refuses before anything is launched (null pointers are never
+    reached)."""
+    import ctypes
+    assert jt.hia_moe_workspace_bytes(*dims) == 0
+    d = jt._MoeDims(*dims)
+    assert jt.lib().hia_moe_fwd(ctypes.byref(d), *([None] * 8), 0, None) == 1
+
+
+def test_moe_workspace_size_and_empty_batch():
+    import ctypes
+    assert jt.hia_moe_workspace_bytes(10803, 4096, 3072, 64, 8) > 0
+    # T = 0: nothing to do, no pointer needed
+    d = jt._MoeDims(0, 256, 128, 8, 2)
+    assert jt.lib().hia_moe_fwd(ctypes.byref(d), *([None] * 8), 0, None) == 0

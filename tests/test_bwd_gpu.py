@@ -36,6 +36,21 @@ def test_bwd_1024px_sampled_groups(oracle_mod):
         assert np.all(np.isfinite(gr))
 
 
+def test_bwd_bench_workload_groups_of_each_sample(oracle_mod):
+    """The workload the benchmark times (1024px: B=2, S=5554, right-padded;
+    sample 1 has 305 padded query rows whose dO is non-zero, and tail kv
+    tiles past its L): two complete (b, kv head) groups of each sample
+    against the oracle, whole-tensor and block by block."""
+    wl = synth.workload("1024px")
+    assert wl.B == 2 and wl.S > min(P + h * w + s for (P, h, w, s) in wl.samples)
+    inputs, grads = run_fwd_bwd(wl)
+    groups = np.zeros((wl.B, wl.Hkv), dtype=bool)
+    groups[0, 0] = groups[0, 5] = groups[1, 2] = groups[1, 7] = True
+    check_bwd(oracle_mod, wl, inputs, grads, groups=groups)
+    for gr in grads:
+        assert np.all(np.isfinite(gr))
+
+
 @pytest.mark.parametrize("samples,S,Hq,Hkv,D", [
     ([(5, 3, 3, 2)], 19, 4, 1, 64),
     ([(100, 10, 13, 7), (0, 0, 0, 0), (250, 0, 0, 0), (0, 16, 16, 2)], 261, 6, 2, 128),
@@ -78,3 +93,40 @@ def test_bwd_deterministic_dkdv():
     _, g1 = run_fwd_bwd(wl)
     _, g2 = run_fwd_bwd(wl)
     assert np.array_equal(g1[1], g2[1]) and np.array_equal(g1[2], g2[2])
+
+
+@pytest.mark.parametrize("norm", [False, True])
+def test_bwd_reusing_forward_workspace(oracle_mod, norm):
+    """hia_attn_bwd_reuse_fwd reads the rotated (and normed) q, k from the
+    forward's workspace: dk, dv equal the plain backward's bit for bit, dq
+    (unordered fp32 reduce-adds) to rounding, and all match the oracle.  The
+    backward workspace starts filled with NaN bytes and is used twice: its
+    dQ accumulator must be cleared by the library on every call."""
+    wl = synth.workload("256px")
+    q, k, v, do = synth.tensors(wl, 3, grad=True)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    seg = jt.hia_segments_build(wl.samples, wl.S)
+    c, s = jt.hia_rope2d_tables(seg, wl.D, wl.base)
+    qk = None
+    if norm:
+        gw = torch.Generator().manual_seed(11)
+        qk = (torch.rand(wl.D, generator=gw) + 0.5, torch.rand(wl.D, generator=gw) + 0.5, 1e-5)
+    qkd = None if qk is None else (qk[0].cuda(), qk[1].cuda(), qk[2])
+    wsf = torch.empty(jt.hia_attn_fwd_workspace_bytes(seg, wl.Hq, wl.Hkv, wl.D), dtype=torch.uint8, device="cuda")
+    wsb = torch.full((jt.hia_attn_bwd_workspace_bytes(seg, wl.Hq, wl.Hkv, wl.D),), 0xFF, dtype=torch.uint8,
+                     device="cuda")
+    o, lse = jt.hia_attn_fwd(seg, qd, kd, vd, c, s, wl.scale, workspace=wsf, qk_norm=qkd)
+    plain = jt.hia_attn_bwd(seg, qd, kd, vd, c, s, o, lse, dod, wl.scale, qk_norm=qkd)
+    reuse1 = jt.hia_attn_bwd(seg, qd, kd, vd, c, s, o, lse, dod, wl.scale, workspace=wsb, qk_norm=qkd,
+                             fwd_workspace=wsf)
+    reuse2 = jt.hia_attn_bwd(seg, qd, kd, vd, c, s, o, lse, dod, wl.scale, workspace=wsb, qk_norm=qkd,
+                             fwd_workspace=wsf)
+    torch.cuda.synchronize()
+    assert jt.hia_get_device_status() == 0
+    for r in (reuse1, reuse2):
+        assert torch.equal(r[1], plain[1]) and torch.equal(r[2], plain[2])
+        rel = float((r[0].float() - plain[0].float()).norm() / plain[0].float().norm())
+        assert rel <= 1e-5, rel
+    f = lambda t: t.float().cpu().numpy()
+    ref_norm = None if qk is None else (qk[0].numpy(), qk[1].numpy(), qk[2])
+    check_bwd(oracle_mod, wl, (q, k, v, do), (f(reuse2[0]), f(reuse2[1]), f(reuse2[2])), qk_norm=ref_norm)

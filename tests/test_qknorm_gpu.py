@@ -62,7 +62,7 @@ def test_qknorm_full_size_sampled(oracle_mod):
     (q, k, v, do), o, lse, (dq, dk, dv, dwq, dwk) = run(wl, wq, wk)
     check_fwd(oracle_mod, wl, q, k, v, o, lse, rows=sample_rows(wl, 4), qk_norm=ref_norm)
     groups = np.zeros((wl.B, wl.Hkv), dtype=bool)
-    groups[0, 2] = True
+    groups[0, 2] = groups[0, 7] = True
     f = lambda t: t.float().cpu().numpy()
     check_bwd(oracle_mod, wl, (q, k, v, do), (f(dq), f(dk), f(dv)), groups=groups, qk_norm=ref_norm)
     assert torch.isfinite(dwq).all() and torch.isfinite(dwk).all()
