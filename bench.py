@@ -34,8 +34,10 @@ METRIC = "joint-attn fwd+bwd masked TFLOPS & % bf16 peak, 1024px (4096 img tok)"
 WORKLOAD = "1024px"
 # committed ncu summaries holding dram traffic per launch at the 1024px workload
 PROFILE_FILES = {k: os.path.join(ROOT, "profiles", f"{k}_1024px.md") for k in ("attn_fwd", "attn_bwd")}
+PROFILE_FILES["moe_up_gate"] = os.path.join(ROOT, "profiles", "moe_up_gate_moe_1024px.md")
 # the files a kernel's machine code depends on (its translation unit and headers)
 KERNEL_SOURCES = {k: [f"{k}.cu", "sm100.cuh", "kernels.h", "internal.h"] for k in ("attn_fwd", "attn_bwd")}
+KERNEL_SOURCES["moe_up_gate"] = ["moe.cu", "sm100.cuh", "kernels.h", "internal.h"]
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # timed regions at least this long are compared with the sustained (power-capped) GEMM peak
 SUSTAINED_AFTER_S = 1.0
@@ -318,29 +320,53 @@ def run_moe(args, rank, world, local):
     dom = "moe_up_gate"
     achieved = up_flops / (kt[dom]["avg_ms"] * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": cached_traffic("moe_up_gate"),
                 "peak_kind": ("bf16_tflops_sustained" if long_run else "bf16_tflops burst") +
                              f" ({pk_kind}): timed region {timed_s:.2f} s",
                 "algorithmic_flops_per_launch": up_flops,
                 "down_proj_tflops": dn_flops / (kt["moe_down"]["avg_ms"] * 1e-3) / 1e12}
 
-    # end to end: x uploaded from pinned host memory and out downloaded every step
+    # End to end: every step uploads its x from pinned host memory and
+    # downloads its out, inside the timed region.  Several steps are in
+    # flight on their own streams (each with its own device buffers and
+    # workspace), so one step's PCIe copies run under another's kernels, as a
+    # pipeline feeding the layer from host memory would run it.
+    nf = max(1, args.e2e_inflight)
     hx = x.pin_memory()
-    hout = torch.empty(mw.T, mw.H, dtype=torch.bfloat16, pin_memory=True)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_e2e = max(1, args.e2e_steps)
-    for i in range(n_e2e + 2):
-        if i == 2:
-            e0.record(stream)
-        xd.copy_(hx, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
-    e1.record(stream)
+    slots = [(xd, out, ws, torch.empty(mw.T, mw.H, dtype=torch.bfloat16, pin_memory=True))]
+    for _ in range(nf - 1):
+        slots.append((torch.empty_like(xd), torch.empty_like(out), torch.empty_like(ws),
+                      torch.empty(mw.T, mw.H, dtype=torch.bfloat16, pin_memory=True)))
+    streams = [torch.cuda.Stream(device=dev) for _ in range(nf)]
+
+    def e2e_run(n):
+        for i in range(n):
+            sx, so, sw, sh = slots[i % nf]
+            with torch.cuda.stream(streams[i % nf]):
+                sx.copy_(hx, non_blocking=True)
+                jt.hia_moe_fwd(sx, wgd, w13d, w2d, mw.topk, out=so, workspace=sw)
+                sh.copy_(so, non_blocking=True)
+
     torch.cuda.synchronize()
+    e2e_run(2 * nf)
+    torch.cuda.synchronize()
+    n_e2e = max(1, args.e2e_steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(streams[0])
+    for st_ in streams[1:]:
+        st_.wait_stream(streams[0])
+    e2e_run(n_e2e)
+    for st_ in streams[1:]:
+        streams[0].wait_stream(st_)
+    e1.record(streams[0])
+    torch.cuda.synchronize()
+    if jt.hia_get_device_status() != 0:
+        raise RuntimeError("device wait timed out during the end-to-end steps")
     ems = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
     e2e = {"value": world * flops / (ems * 1e-3) / 1e12, "unit": "TFLOPS",
-           "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": hout.numel() * 2, "ms_per_step": ems,
-           "api": "hia_moe_fwd (C ABI) with x copied from pinned host memory and out copied back each step"}
+           "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": mw.T * mw.H * 2, "ms_per_step": ems,
+           "api": f"hia_moe_fwd (C ABI), x copied from pinned host memory and out copied back each step, "
+                  f"{nf} steps in flight on {nf} streams"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

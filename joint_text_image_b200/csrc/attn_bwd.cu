@@ -127,9 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.bar_s_full[i], 1);
       mbar_init(&sm.bar_dp_full[i], 1);
-      mbar_init(&sm.bar_ds_ready[i], 128);
+      mbar_init(&sm.bar_ds_ready[i], 4);   // one arrival per softmax warp
       mbar_init(&sm.bar_dq_full[i], 1);
-      mbar_init(&sm.bar_dq_empty[i], 128);
+      mbar_init(&sm.bar_dq_empty[i], 4);   // one arrival per dQ warp
       mbar_init(&sm.bar_s_free[i], 1);
     }
     mbar_init(&sm.bar_final, 1);
@@ -308,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&sm.bar_ds_ready[bf]);
+      __syncwarp();  // the warp's TMEM and shared-memory writes are done; one lane signals for it
+      if (lane == 0) mbar_arrive(&sm.bar_ds_ready[bf]);
     }
     // ---- epilogue: warpgroup 0 writes dK = R^T (scale dKr), warpgroup 1 dV
     bool have = n_it > 0 && ok;
@@ -423,7 +424,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
       }
       tc_fence_before();
-      mbar_arrive(&sm.bar_dq_empty[bf]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.bar_dq_empty[bf]);
       float* dst = p.dq_acc + ((int64_t(b) * p.Hq + h) * p.S_pad + int64_t(qt) * BQ) * D;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {

@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.bar_s_full[i], 1);
-      mbar_init(&sm.bar_p_ready[i], 128);
+      mbar_init(&sm.bar_p_ready[i], 4);  // one arrival per softmax warp
       mbar_init(&sm.bar_o_final[i], 1);
     }
     sm.abort_flag = 0;
@@ -322,7 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&sm.bar_p_ready[t]);
+      __syncwarp();  // the warp's P writes are done; one lane signals for it
+      if (lane == 0) mbar_arrive(&sm.bar_p_ready[t]);
     }
     // ---- epilogue: O / l -> bf16 rows, LSE
     if (active) {

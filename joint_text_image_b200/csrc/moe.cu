@@ -315,6 +315,21 @@ struct GemmSmem {
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z)); }
 
+// Tile t -> (group g, 128-row tile j of the group, column tile nt).  Tiles are
+// ordered group by group and, inside a group, column-tile-major: the CTAs that
+// run together (consecutive t) share each column tile of the group's weights,
+// which is then read from HBM once, and the group's few row tiles stay in L2.
+// Group g owns tiles [first_g * nt, first_g' * nt), first_g = offsets[g] / 128
+// its first row tile, so the row tile t / nt lies inside group g.
+__device__ __forceinline__ void decode_tile(const GemmParams& p, int t, int& g, int& j, int& nt) {
+  g = p.mtab[2 * (t / p.nt)];
+  const int first = p.meta->offsets[g] / kTileRows;
+  const int mtg = p.meta->offsets[g + 1] / kTileRows - first;  // row tiles of the group
+  const int local = t - first * p.nt;
+  nt = local / mtg;
+  j = local % mtg;
+}
+
 // tm_a: the sorted rows (x rows for UpGate, act rows for Down); tm_x: x itself
 // (the shared expert's A rows in UpGate); tm_b: W13 as [(E+1)*2I][H] or W2 as
 // [(E+1)*H][I].
@@ -360,8 +375,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
-        const int mt = tile / p.nt, nt = tile % p.nt;
-        const int g = p.mtab[2 * mt], j = p.mtab[2 * mt + 1];
+        int g, j, nt;
+        decode_tile(p, tile, g, j, nt);
         const bool shared_x = MODE == kUpGate && g == p.E;  // the shared expert reads x directly
         const CUtensorMap* ma = shared_x ? &tm_x : &tm_a;
         const int arow = shared_x ? j * kTileRows : p.meta->offsets[g] + j * kTileRows;
@@ -424,8 +439,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int buf = tl & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_acc_full[buf], (tl >> 1) & 1, wc))) break;
       tc_fence_after();
-      const int mt = tile / p.nt, nt = tile % p.nt;
-      const int g = p.mtab[2 * mt], j = p.mtab[2 * mt + 1];
+      int g, j, nt;
+      decode_tile(p, tile, g, j, nt);
       const int64_t row = p.meta->offsets[g] + j * kTileRows + r;
       const uint32_t acc = tmem + uint32_t(buf * 256) + lane_off;
       if (MODE == kUpGate) {
@@ -490,13 +505,27 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const __nv_bfloat16* _
   for (int64_t t = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5; t < T; t += n_warps) {
     const int my_row = lane < topk ? rowidx[t * topk + lane] : 0;
     const float my_w = lane < topk ? weights[t * topk + lane] : 0.f;
+    // the rows of every choice (then the shared row), fetched once per token
+    int rows[kMaxTopk + 1];
+    float ws[kMaxTopk + 1];
+#pragma unroll
+    for (int j = 0; j <= kMaxTopk; ++j) {
+      rows[j] = j < topk ? __shfl_sync(0xffffffffu, my_row, j) : shared0 + int(t);
+      ws[j] = j < topk ? __shfl_sync(0xffffffffu, my_w, j) : 1.f;
+    }
     for (int c = lane; c < nchunk; c += 32) {
+      // all k + 1 loads of this chunk in flight before the sum (in order:
+      // choices, then the shared expert)
+      uint4 u[kMaxTopk + 1];
+#pragma unroll
+      for (int j = 0; j <= kMaxTopk; ++j)
+        if (j <= topk) u[j] = __ldg(reinterpret_cast<const uint4*>(y + int64_t(rows[j]) * H) + c);
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int j = 0; j <= topk; ++j) {
-        const int row = j < topk ? __shfl_sync(0xffffffffu, my_row, j) : shared0 + int(t);
-        const float w = j < topk ? __shfl_sync(0xffffffffu, my_w, j) : 1.f;
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(y + int64_t(row) * H) + c);
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int j = 0; j <= kMaxTopk; ++j) {
+        if (j > topk) break;
+        const float w = j < topk ? ws[j] : 1.f;
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 f = __bfloat1622float2(h2[i]);

@@ -311,7 +311,7 @@ void launch_rope2d_tables(const SampleDev* samples, const ImageDev* images, int 
   if (total == 0) return;
   const int threads = 256;
   int64_t blocks = (total + threads - 1) / threads;
-  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks > 148 * 64) blocks = 148 * 64;  // one (b, n, j) per thread up to 2.4 M entries
   prof_begin(kRopeTables, st);
   rope2d_tables_kernel<<<int(blocks), threads, 0, st>>>(samples, images, B, S, D, base, cos_out, sin_out);
   prof_end(kRopeTables, st);
