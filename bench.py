@@ -411,6 +411,8 @@ def main():
                     help="synthetic workload (the metric is quoted on 1024px; the others are for profiling)")
     ap.add_argument("--packed", action="store_true",
                     help="packed (varlen) layout: no padded rows (no e2e line: the host step is padded-only)")
+    ap.add_argument("--bwd-split", choices=["auto", "never", "always"], default="auto",
+                    help="backward schedule: split the longest kv tiles in two (hia_segments_set_bwd_split)")
     ap.add_argument("--qk-norm", action="store_true",
                     help="enable the per-head QK RMSNorm after RoPE (weights seeded, eps 1e-5)")
     ap.add_argument("--source-hash", choices=sorted(KERNEL_SOURCES),
@@ -457,6 +459,7 @@ def main():
         q, k, v, do = (packf(t) for t in (q, k, v, do))
     else:
         seg = jt.hia_segments_build(wl.samples, wl.S)
+    seg.set_bwd_split({"auto": 0, "never": 1, "always": 2}[args.bwd_split])
     info = seg.info()
     pairs = info.visible_pairs
     fwd_flops = 4.0 * wl.D * wl.Hq * pairs

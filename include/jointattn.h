@@ -98,7 +98,7 @@ typedef struct {
     int32_t bwd_q_tiles;         /* ceil(S / 64) */
     int32_t bwd_kv_tiles;        /* ceil(S / 128) */
     int32_t packed;              /* 1: built by hia_segments_build_packed */
-    int32_t reserved;
+    int32_t bwd_split_units;     /* kv tiles whose backward work can be split in two (see hia_segments_set_bwd_split) */
     int64_t total_rows;          /* rows of a tensor in this layout: B*S, or the sum of L when packed */
 } hia_segments_info_t;
 
@@ -161,6 +161,23 @@ int hia_segments_upload(hia_segments* seg, void* stream);
 void hia_segments_destroy(hia_segments* seg);
 
 int hia_segments_info(const hia_segments* seg, hia_segments_info_t* info);
+
+/* Scheduling of the backward (a property of the library, not of the method:
+ * the result is the same either way, and deterministic).  One CTA of the
+ * backward handles one (sample, kv head, 128-key tile) over every query tile
+ * that sees it, so a few CTAs (keys seen by every later row) are far longer
+ * than the rest and can leave SMs idle at the end.  The descriptor also holds
+ * a second schedule in which those longest kv tiles (query range within 10%
+ * of the longest) are split into two halves, each writing an fp32 partial of
+ * dK and dV; the half that finishes second adds the two in a fixed order.
+ *   HIA_BWD_SPLIT_AUTO (default): each backward launch picks the schedule a
+ *     list-scheduling estimate (heaviest first, on the device's SM count, for
+ *     its number of kv heads) finishes sooner; it splits for one long sample,
+ *     not for batches where the balance is already good.
+ *   HIA_BWD_SPLIT_NEVER / HIA_BWD_SPLIT_ALWAYS: force one schedule.
+ * Errors: HIA_ERR_INVALID_ARG (null, unknown mode). */
+enum { HIA_BWD_SPLIT_AUTO = 0, HIA_BWD_SPLIT_NEVER = 1, HIA_BWD_SPLIT_ALWAYS = 2 };
+int hia_segments_set_bwd_split(hia_segments* seg, int mode);
 
 /* Host copies for tests and inspection.  row_bound: int32 [B, S] e_b(q)
  * (-1 for a sample with L = 0).  mask: uint8 [B, S, S] (1 = visible) rendered

@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = (
     "hia_profile_end", "hia_attn_fwd_noalloc", "hia_debug_exp2", "hia_step_create", "hia_step_destroy",
     "hia_attn_step_host", "hia_attn_fwd_ex", "hia_attn_bwd_ex", "hia_segments_build_packed",
     "hia_segments_layout", "hia_segments_build_multi", "hia_attn_bwd_reuse_fwd",
-    "hia_moe_workspace_bytes", "hia_moe_fwd",
+    "hia_moe_workspace_bytes", "hia_moe_fwd", "hia_segments_set_bwd_split",
 )
 
 
@@ -56,7 +56,7 @@ class SegmentsInfo(ctypes.Structure):
                 ("fwd_q_tiles", ctypes.c_int32), ("fwd_kv_tiles", ctypes.c_int32),
                 ("fwd_tiles_full", ctypes.c_int64), ("fwd_tiles_partial", ctypes.c_int64),
                 ("fwd_tiles_skipped", ctypes.c_int64), ("bwd_q_tiles", ctypes.c_int32),
-                ("bwd_kv_tiles", ctypes.c_int32), ("packed", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("bwd_kv_tiles", ctypes.c_int32), ("packed", ctypes.c_int32), ("bwd_split_units", ctypes.c_int32),
                 ("total_rows", ctypes.c_int64)]
 
 
@@ -96,6 +96,7 @@ def lib():
         L.hia_segments_destroy.argtypes = [P]
         L.hia_segments_destroy.restype = None
         L.hia_segments_info.argtypes = [P, ctypes.POINTER(SegmentsInfo)]
+        L.hia_segments_set_bwd_split.argtypes = [P, I]
         L.hia_segments_row_bound.argtypes = [P, P]
         L.hia_segments_layout.argtypes = [P, P, P]
         L.hia_segments_mask.argtypes = [P, P]
@@ -212,6 +213,12 @@ class Segments:
         e = np.zeros((self.B, self.S), dtype=np.int32)
         _check(lib().hia_segments_row_bound(self.handle, e.ctypes.data_as(ctypes.c_void_p)), "row_bound")
         return e
+
+    def set_bwd_split(self, mode):
+        """Backward schedule: 0 auto (default), 1 never split, 2 always split
+        the longest kv tiles (hia_segments_set_bwd_split)."""
+        _check(lib().hia_segments_set_bwd_split(self.handle, int(mode)), "hia_segments_set_bwd_split")
+        return self
 
     def mask(self):
         import numpy as np

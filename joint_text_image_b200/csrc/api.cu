@@ -4,7 +4,10 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <algorithm>
+#include <functional>
 #include <initializer_list>
+#include <queue>
 #include <cstring>
 #include <mutex>
 
@@ -185,7 +188,7 @@ FwdWs fwd_ws(const hia_segments* seg, int Hq, int Hkv, int D) {
 int S_pad64(int S) { return (S + 63) / 64 * 64; }
 
 struct BwdWs {
-  size_t q_off, k_off, lse_off, delta_off, dq_off, dk_off, dw_off, total;
+  size_t q_off, k_off, lse_off, delta_off, dq_off, dk_off, dw_off, part_off, cnt_off, total;
 };
 // The dK accumulator and the weight-gradient partials are used only with the
 // QK RMSNorm; the size always includes them so one workspace serves both.
@@ -200,11 +203,62 @@ BwdWs bwd_ws(const hia_segments* seg, int Hq, int Hkv, int D) {
   w.dq_off = w.delta_off + align256(BSp * Hq * 4);
   w.dk_off = w.dq_off + align256(BSp * Hq * D * 4);
   w.dw_off = w.dk_off + align256(BSp * Hkv * D * 4);
-  w.total = w.dw_off + align256(size_t(2) * hia::grad_finalize_blocks(seg->B, seg->S) * D * 4);
+  w.part_off = w.dw_off + align256(size_t(2) * hia::grad_finalize_blocks(seg->B, seg->S) * D * 4);
+  // split schedule: per (slot, kv head) two halves' fp32 dK and dV partials, and a ticket counter
+  w.cnt_off = w.part_off + align256(size_t(seg->n_split_slots) * Hkv * 2 * 2 * hia::kBwdBK * D * 4);
+  w.total = w.cnt_off + align256(size_t(seg->n_split_slots) * Hkv * 4);
   return w;
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? HIA_OK : HIA_ERR_CUDA; }
+
+// Finish time of a backward work list dispatched in order to the first free
+// SM (the block scheduler's policy), one CTA per (entry, kv head): a CTA
+// costs its query tiles times g plus a fixed part (K/V load, epilogue; about
+// four tile iterations), and a split half two more (its partial's write and
+// the combine).
+double bwd_makespan(const std::vector<int32_t>& work, int Hkv, int g, int n_sm) {
+  constexpr double kCtaCost = 4.0, kSplitCost = 2.0;
+  std::priority_queue<double, std::vector<double>, std::greater<double>> sms;
+  for (int i = 0; i < n_sm; ++i) sms.push(0.0);
+  double span = 0.0;
+  for (size_t e = 0; e + hia::kBwdWorkInts <= work.size(); e += hia::kBwdWorkInts) {
+    const double c = double(work[e + 3] - work[e + 2]) * g + kCtaCost + (work[e + 4] >= 0 ? kSplitCost : 0.0);
+    for (int h = 0; h < Hkv; ++h) {
+      const double t = sms.top() + c;
+      sms.pop();
+      sms.push(t);
+      span = std::max(span, t);
+    }
+  }
+  return span;
+}
+
+int device_sm_count() {
+  static hia::PerContext<int> cache;
+  int n = 0;
+  if (cache.get(&n, [](int* out) {
+        int dev = 0;
+        const cudaError_t e = cudaGetDevice(&dev);
+        return e != cudaSuccess ? e : cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev);
+      }) != cudaSuccess)
+    return 148;
+  return n;
+}
+
+// Whether a backward launch uses the split work list.
+bool use_bwd_split(hia_segments* g, int Hkv, int gq) {
+  if (g->n_split_slots == 0 || g->bwd_split_mode == HIA_BWD_SPLIT_NEVER) return false;
+  if (g->bwd_split_mode == HIA_BWD_SPLIT_ALWAYS) return true;
+  const int n_sm = device_sm_count();
+  std::lock_guard<std::mutex> lk(g->choice_mu);
+  const auto key = std::make_tuple(Hkv, gq, n_sm);
+  auto it = g->choice.find(key);
+  if (it != g->choice.end()) return it->second;
+  const bool split = bwd_makespan(g->bwd_work_split, Hkv, gq, n_sm) < bwd_makespan(g->bwd_work, Hkv, gq, n_sm);
+  g->choice[key] = split;
+  return split;
+}
 
 int check_norm(const hia_qk_norm* n) {
   if (!n) return HIA_OK;
@@ -264,10 +318,10 @@ extern "C" int hia_segments_upload(hia_segments* g, void* stream) {
   if (g->dbuf && g->device != dev) return HIA_ERR_INVALID_ARG;
   const size_t n_s = g->samples.size() * sizeof(SampleDev), n_i = g->images.size() * sizeof(hia::ImageDev);
   const size_t n_ft = g->fwd_tiles.size() * 4, n_fl = g->fwd_list.size() * 4, n_fw = g->fwd_work.size() * 4;
-  const size_t n_bt = g->bwd_tiles.size() * 4, n_bw = g->bwd_work.size() * 4;
+  const size_t n_bt = g->bwd_tiles.size() * 4, n_bw = g->bwd_work.size() * 4, n_bs = g->bwd_work_split.size() * 4;
   const size_t o_s = 0, o_i = align256(n_s), o_ft = o_i + align256(n_i), o_fl = o_ft + align256(n_ft),
                o_fw = o_fl + align256(n_fl), o_bt = o_fw + align256(n_fw), o_bw = o_bt + align256(n_bt),
-               total = o_bw + align256(n_bw) + 256;
+               o_bs = o_bw + align256(n_bw), total = o_bs + align256(n_bs) + 256;
   if (!g->dbuf) {
     if (cudaMalloc(&g->dbuf, total) != cudaSuccess) {
       g->dbuf = nullptr;
@@ -283,6 +337,8 @@ extern "C" int hia_segments_upload(hia_segments* g, void* stream) {
   if (e == cudaSuccess && n_fw) e = cudaMemcpyAsync(base + o_fw, g->fwd_work.data(), n_fw, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess && n_bt) e = cudaMemcpyAsync(base + o_bt, g->bwd_tiles.data(), n_bt, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess && n_bw) e = cudaMemcpyAsync(base + o_bw, g->bwd_work.data(), n_bw, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && n_bs)
+    e = cudaMemcpyAsync(base + o_bs, g->bwd_work_split.data(), n_bs, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return HIA_ERR_CUDA;
   g->device = dev;
   g->d_samples = reinterpret_cast<const SampleDev*>(base + o_s);
@@ -292,6 +348,7 @@ extern "C" int hia_segments_upload(hia_segments* g, void* stream) {
   g->d_fwd_work = reinterpret_cast<const int32_t*>(base + o_fw);
   g->d_bwd_tiles = reinterpret_cast<const int32_t*>(base + o_bt);
   g->d_bwd_work = reinterpret_cast<const int32_t*>(base + o_bw);
+  g->d_bwd_work_split = reinterpret_cast<const int32_t*>(base + o_bs);
   return HIA_OK;
 }
 
@@ -305,6 +362,13 @@ extern "C" void hia_segments_destroy(hia_segments* g) {
     if (cur != g->device) cudaSetDevice(cur);
   }
   delete g;
+}
+
+extern "C" int hia_segments_set_bwd_split(hia_segments* g, int mode) {
+  if (!g || mode < HIA_BWD_SPLIT_AUTO || mode > HIA_BWD_SPLIT_ALWAYS) return HIA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g->choice_mu);
+  g->bwd_split_mode = mode;
+  return HIA_OK;
 }
 
 extern "C" int hia_rope2d_tables(const hia_segments* g, int D, double base, float* c, float* s, void* stream) {
@@ -490,6 +554,9 @@ extern "C" int hia_attn_bwd_reuse_fwd(const hia_segments* g, int Hq, int Hkv, in
   float* dq_acc = reinterpret_cast<float*>(wb + w.dq_off);
   float* dk_acc = reinterpret_cast<float*>(wb + w.dk_off);
   float* dw_part = reinterpret_cast<float*>(wb + w.dw_off);
+  float* part = reinterpret_cast<float*>(wb + w.part_off);
+  int* part_cnt = reinterpret_cast<int*>(wb + w.cnt_off);
+  const bool split = use_bwd_split(const_cast<hia_segments*>(g), Hkv, gq);
   const int S_pad = S_pad64(g->S);
 
   CUtensorMap tq, tk, tv, tdo;
@@ -518,6 +585,8 @@ extern "C" int hia_attn_bwd_reuse_fwd(const hia_segments* g, int Hq, int Hkv, in
   pp.lse2 = lse2;
   pp.delta = delta;
   pp.dq_acc = dq_acc;
+  pp.part_cnt = part_cnt;
+  pp.n_cnt = g->n_split_slots * Hkv;
   pp.B = g->B;
   pp.S = g->S;
   pp.S_pad = S_pad;
@@ -530,7 +599,9 @@ extern "C" int hia_attn_bwd_reuse_fwd(const hia_segments* g, int Hq, int Hkv, in
   p.samples = g->d_samples;
   p.images = g->d_images;
   p.tiles = g->d_bwd_tiles;
-  p.work = g->d_bwd_work;
+  p.work = split ? g->d_bwd_work_split : g->d_bwd_work;
+  p.part = part;
+  p.part_cnt = part_cnt;
   p.B = g->B;
   p.S = g->S;
   p.S_pad = S_pad;
@@ -558,7 +629,8 @@ extern "C" int hia_attn_bwd_reuse_fwd(const hia_segments* g, int Hq, int Hkv, in
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = status;
   p.timeout_ns = kDefaultTimeoutNs;
-  const int64_t n_blocks = int64_t(g->B) * g->bKT * Hkv;
+  const int64_t n_entries = int64_t(split ? g->bwd_work_split.size() : g->bwd_work.size()) / hia::kBwdWorkInts;
+  const int64_t n_blocks = n_entries * Hkv;
   if (n_blocks > (1ll << 31) - 1) return HIA_ERR_UNSUPPORTED;
   if ((rc = cuda_status(hia::launch_attn_bwd(tq, tk, tv, tdo, p, int(n_blocks), D, st)))) return rc;
 

@@ -68,6 +68,7 @@ struct BwdSmem {
   uint64_t bar_final;
   uint32_t tmem_base;
   int abort_flag;
+  int split_ticket;  // split schedule: this half's ticket (0 first, 1 second to finish)
 };
 
 // S^T = Kr Qr^T and dP^T = V dO^T: A = 128-row tile (K-major, 64-wide D
@@ -110,10 +111,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   int bid = blockIdx.x;
   const int hkv = bid % p.Hkv;
   bid /= p.Hkv;
-  const int b = p.work[2 * bid], kt = p.work[2 * bid + 1];
-  // the query tiles [qt_first, qt_end) see this kv tile; [full_first, full_end) see all of it
+  // work entry: this CTA's query tiles [qt_first, qt_end) of kv tile kt (all
+  // that see it, or one half of them when split: slot >= 0)
+  const int32_t* we = p.work + kBwdWorkInts * bid;
+  const int b = we[0], kt = we[1], qt_first = we[2], qt_end = we[3], slot = we[4], part = we[5];
+  // [full_first, full_end): the query tiles that see all of the kv tile
   const int32_t* te = p.tiles + 4 * (b * p.bKT + kt);
-  const int qt_first = te[0], qt_end = te[1], full_first = te[2], full_end = te[3];
+  const int full_first = te[2], full_end = te[3];
   const SampleDev smp = p.samples[b];
   const int n_qt = max(qt_end - qt_first, 0);
   const int n_it = n_qt * p.g;  // iteration i: head hkv*g + i / n_qt, query tile qt_first + i % n_qt
@@ -315,7 +319,66 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool have = n_it > 0 && ok;
     if (have) have = __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, wc));
     if (have) tc_fence_after();
-    const bool store = key < smp.rows;
+    bool write_out = true;  // false: the other half of a split kv tile writes dK/dV
+    if (slot >= 0) {
+      // Split kv tile: this CTA saw half of its query tiles.  Each half writes
+      // its raw fp32 accumulator rows (dK in warpgroup 0, dV in warpgroup 1)
+      // to its own partial, fences, and takes a ticket; the half that
+      // finishes second adds the other half's partial into its TMEM (fp32
+      // a + b is commutative: the same bits whichever half is second) and
+      // runs the common epilogue below.  No thread waits on the other CTA.
+      const uint32_t tacc = (bf == 0 ? tdK : tdV) + lane_off;
+      const int64_t unit = (int64_t(slot) * p.Hkv + hkv) * 2;
+      float* mine = p.part + ((unit + part) * 2 + bf) * int64_t(BK * D) + int64_t(r) * D;
+      const float* other = p.part + ((unit + (part ^ 1)) * 2 + bf) * int64_t(BK * D) + int64_t(r) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        if (have) {
+          tmem_ld32(tacc + uint32_t(c * 32), v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        float4* d4 = reinterpret_cast<float4*>(mine + c * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
+                              __uint_as_float(v[4 * i + 3]));
+      }
+      __threadfence();
+      named_bar_sync(2, 256);  // both epilogue warpgroups' partial rows written and fenced
+      if (threadIdx.x == 128) sm.split_ticket = atomicAdd(&p.part_cnt[slot * p.Hkv + hkv], 1);
+      named_bar_sync(2, 256);
+      if (sm.split_ticket == 0) {
+        have = false;  // the other half finishes this kv tile
+        write_out = false;
+      } else {
+        __threadfence();
+      }
+      if (have) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tacc + uint32_t(c * 32), v);
+          tmem_ld_wait();
+          const float4* o4 = reinterpret_cast<const float4*>(other + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 a = __ldcg(o4 + i);
+            v[4 * i] = __float_as_uint(__uint_as_float(v[4 * i]) + a.x);
+            v[4 * i + 1] = __float_as_uint(__uint_as_float(v[4 * i + 1]) + a.y);
+            v[4 * i + 2] = __float_as_uint(__uint_as_float(v[4 * i + 2]) + a.z);
+            v[4 * i + 3] = __float_as_uint(__uint_as_float(v[4 * i + 3]) + a.w);
+          }
+          tmem_st32(tacc + uint32_t(c * 32), v);
+        }
+        tmem_st_wait();
+      }
+      if (write_out && threadIdx.x == 128) p.part_cnt[slot * p.Hkv + hkv] = 0;  // ready for the next launch
+    }
+    const bool store = write_out && key < smp.rows;
     if (bf == 0 && p.dk_acc) {
       // QK RMSNorm: the norm's backward needs the whole row, so write
       // scale * dK_n (gradient w.r.t. the normed rotated key row) in fp32 and
@@ -468,6 +531,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdPreParams p) {
   constexpr int LPH = D / 8;        // lanes per head (16-byte chunks of 8 bf16)
   constexpr int HPS = 32 / LPH;     // heads per step
   const int lane = threadIdx.x & 31;
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < p.n_cnt; i += blockDim.x) p.part_cnt[i] = 0;
   const int c = lane % LPH, hs = lane / LPH;
   const unsigned gmask = (LPH == 32 ? 0xffffffffu : ((1u << LPH) - 1u)) << (hs * LPH);
   // grid-stride over (b, q) rows: a fixed grid of resident warps

@@ -75,6 +75,8 @@ struct BwdPreParams {
   float* lse2;          // [B][Hq][S_pad]: lse * log2(e); +inf beyond S
   float* delta;         // [B][Hq][S_pad]: rowsum(dout * o); 0 beyond S
   float* dq_acc;        // [B][Hq][S_pad][D]: zeroed by this pass
+  int* part_cnt;        // [n_cnt] split-schedule tickets: zeroed by this pass
+  int n_cnt;
   int B, S, S_pad, Hq, g, D;
 };
 
@@ -82,7 +84,9 @@ struct BwdParams {
   const SampleDev* samples;
   const ImageDev* images;
   const int32_t* tiles;  // [B][bKT][4]: (qt_first, qt_end, full_first, full_end)
-  const int32_t* work;   // [n_work][2]
+  const int32_t* work;   // [n_work][kBwdWorkInts]: (b, kt, qt_lo, qt_hi, slot, part)
+  float* part;           // split halves' fp32 partials [slot][Hkv][part][dK, dV][128][D]
+  int* part_cnt;         // [slot][Hkv] tickets (zeroed by bwd_pre)
   int B, S, S_pad, Hq, Hkv, g, bQT, bKT;
   const float* lse2;
   const float* delta;

@@ -174,11 +174,36 @@ int build(const std::vector<SampleSpec>& spec, int S, bool packed, hia_segments*
   order.assign(size_t(B) * g->bKT, 0);
   for (size_t i = 0; i < order.size(); ++i) order[i] = int(i);
   std::stable_sort(order.begin(), order.end(), [&](int a, int c) { return bwd_cost[a] > bwd_cost[c]; });
-  g->bwd_work.resize(order.size() * 2);
-  for (size_t i = 0; i < order.size(); ++i) {
-    g->bwd_work[i * 2 + 0] = order[i] / g->bKT;
-    g->bwd_work[i * 2 + 1] = order[i] % g->bKT;
+  struct BwdJob {
+    int64_t cost;
+    int32_t b, kt, lo, hi, slot, part;
+  };
+  std::vector<BwdJob> whole, split;
+  int64_t max_cost = 0;
+  for (int u : order) max_cost = std::max(max_cost, bwd_cost[u]);
+  int n_slots = 0;
+  for (int u : order) {
+    const int b = u / g->bKT, kt = u % g->bKT;
+    const int32_t* e = &g->bwd_tiles[size_t(u) * 4];
+    const int64_t c = bwd_cost[u];
+    whole.push_back({c, b, kt, e[0], e[1], -1, 0});
+    if (c >= 4 && 10 * c > 9 * max_cost) {  // within 10% of the longest query range
+      const int mid = e[0] + int(c / 2);
+      split.push_back({mid - e[0], b, kt, e[0], mid, n_slots, 0});
+      split.push_back({e[1] - mid, b, kt, mid, e[1], n_slots, 1});
+      ++n_slots;
+    } else {
+      split.push_back({c, b, kt, e[0], e[1], -1, 0});
+    }
   }
+  std::stable_sort(split.begin(), split.end(), [](const BwdJob& a, const BwdJob& c) { return a.cost > c.cost; });
+  auto emit = [](const std::vector<BwdJob>& js, std::vector<int32_t>& out) {
+    out.clear();
+    for (const BwdJob& j : js) out.insert(out.end(), {j.b, j.kt, j.lo, j.hi, j.slot, j.part});
+  };
+  emit(whole, g->bwd_work);
+  emit(split, g->bwd_work_split);
+  g->n_split_slots = n_slots;
 
   hia_segments_info_t& in = g->info;
   in.B = B;
@@ -192,6 +217,7 @@ int build(const std::vector<SampleSpec>& spec, int S, bool packed, hia_segments*
   in.bwd_q_tiles = g->bQT;
   in.bwd_kv_tiles = g->bKT;
   in.packed = packed ? 1 : 0;
+  in.bwd_split_units = n_slots;
   in.total_rows = g->total_rows;
   *out = g;
   return HIA_OK;

@@ -152,3 +152,18 @@ def test_moe_workspace_size_and_empty_batch():
     # T = 0: nothing to do, no pointer needed
     d = jt._MoeDims(0, 256, 128, 8, 2)
     assert jt.lib().hia_moe_fwd(ctypes.byref(d), *([None] * 8), 0, None) == 0
+
+
+def test_bwd_split_units_and_mode():
+    """The descriptor's split schedule: kv tiles within 10% of the longest
+    query range; the mode setter refuses unknown modes."""
+    seg = jt.hia_segments_build(synth.workload("1024px_bwd").samples, synth.workload("1024px_bwd").S,
+                                upload=False)
+    assert seg.info().bwd_split_units > 0
+    assert seg.info().bwd_split_units < seg.info().bwd_kv_tiles
+    for mode in (0, 1, 2):
+        seg.set_bwd_split(mode)
+    with pytest.raises(jt.HiaError):
+        seg.set_bwd_split(3)
+    tiny = jt.hia_segments_build(synth.workload("tiny").samples, synth.workload("tiny").S, upload=False)
+    assert tiny.info().bwd_split_units == 0  # one query range of 2 tiles: nothing worth splitting

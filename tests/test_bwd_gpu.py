@@ -130,3 +130,44 @@ def test_bwd_reusing_forward_workspace(oracle_mod, norm):
     f = lambda t: t.float().cpu().numpy()
     ref_norm = None if qk is None else (qk[0].numpy(), qk[1].numpy(), qk[2])
     check_bwd(oracle_mod, wl, (q, k, v, do), (f(reuse2[0]), f(reuse2[1]), f(reuse2[2])), qk_norm=ref_norm)
+
+
+def _fwd_bwd_with_split(wl, mode, seed=0):
+    q, k, v, do = synth.tensors(wl, seed, grad=True)
+    seg = jt.hia_segments_build(wl.samples, wl.S).set_bwd_split(mode)
+    c, s = jt.hia_rope2d_tables(seg, wl.D, wl.base)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = jt.hia_attn_fwd(seg, qd, kd, vd, c, s, wl.scale)
+    dq, dk, dv = jt.hia_attn_bwd(seg, qd, kd, vd, c, s, o, lse, dod, wl.scale)
+    torch.cuda.synchronize()
+    assert jt.hia_get_device_status() == 0
+    f = lambda t: t.float().cpu().numpy()
+    return seg, (q, k, v, do), (f(dq), f(dk), f(dv))
+
+
+@pytest.mark.parametrize("name", ["256px", "mixed_small"])
+def test_bwd_split_schedule_parity(oracle_mod, name):
+    """The split schedule (the longest kv tiles' query ranges halved, the two
+    fp32 partials of dK/dV added by the half that finishes second), forced on:
+    against the oracle in full and block by block, dk/dv bitwise repeatable."""
+    if name == "mixed_small":
+        wl = synth.custom([(300, 12, 20, 5), (0, 0, 0, 0), (700, 0, 0, 0), (64, 16, 16, 2)], 8, 2, 128)
+    else:
+        wl = synth.workload(name)
+    seg, inputs, g1 = _fwd_bwd_with_split(wl, 2)
+    assert seg.info().bwd_split_units > 0
+    check_bwd(oracle_mod, wl, inputs, g1)
+    _, _, g2 = _fwd_bwd_with_split(wl, 2)
+    assert np.array_equal(g1[1], g2[1]) and np.array_equal(g1[2], g2[2])
+
+
+def test_bwd_split_schedule_full_size(oracle_mod):
+    """The single-sample training backward (1024px_bwd) with the split
+    schedule forced on: two complete (b, kv head) groups against the oracle,
+    one of them a kv head whose prefix tiles are split."""
+    wl = synth.workload("1024px_bwd")
+    seg, inputs, grads = _fwd_bwd_with_split(wl, 2)
+    assert seg.info().bwd_split_units > 0
+    groups = np.zeros((wl.B, wl.Hkv), dtype=bool)
+    groups[0, 1] = groups[0, 6] = True
+    check_bwd(oracle_mod, wl, inputs, grads, groups=groups)

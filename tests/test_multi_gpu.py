@@ -82,8 +82,9 @@ def test_multi_packed_equals_padded():
     lens = [length(x) for x in SAMPLES]
     for b, L in enumerate(lens):
         do[b, L:] = 0  # padded rows then add nothing to dk, dv
-    pad, _ = run(jt.hia_segments_build_multi(SAMPLES, S), q, k, v, do, 128 ** -0.5)
-    seg = jt.hia_segments_build_multi(SAMPLES, packed=True)
+    # one backward schedule for both layouts (bitwise dk, dv; see test_packed_gpu)
+    pad, _ = run(jt.hia_segments_build_multi(SAMPLES, S).set_bwd_split(1), q, k, v, do, 128 ** -0.5)
+    seg = jt.hia_segments_build_multi(SAMPLES, packed=True).set_bwd_split(1)
     pack = lambda x: torch.cat([x[b, :L] for b, L in enumerate(lens)], 0).contiguous()
     c, s = jt.hia_rope2d_tables(seg, 128)
     qp, kp, vp, dop = (pack(t).cuda() for t in (q, k, v, do))

@@ -64,3 +64,20 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_moe_reference_arm_under_torchrun_prints_once():
+    """The MoE workload's reference arm (the fp64 oracle on a token sample)
+    under torchrun: one line from rank 0, the other rank exits cleanly."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.join(ROOT, "bench.py"),
+           "--workload", "moe_tiny", "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
+           "--moe-ref-tokens", "4"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["metric"].startswith("MoE") and d["cpu_baseline"]["kind"] == "oracle"
