@@ -51,12 +51,12 @@ def run(seg, q, k, v, do, scale):
     return [t.cpu() for t in (o, lse, dq, dk, dv)], (c.cpu(), s.cpu())
 
 
-@pytest.mark.parametrize("D", [128, 64])
-def test_multi_image_parity_with_oracle(oracle_mod, D):
+@pytest.mark.parametrize("D,split", [(128, 0), (64, 0), (128, 2), (64, 2)])
+def test_multi_image_parity_with_oracle(oracle_mod, D, split):
     S = max(length(x) for x in SAMPLES) + 17
     Hq, Hkv = 4, 2
     q, k, v, do = inputs(S, Hq, Hkv, D)
-    seg = jt.hia_segments_build_multi(SAMPLES, S)
+    seg = jt.hia_segments_build_multi(SAMPLES, S).set_bwd_split(split)
     (o, lse, dq, dk, dv), (c, s) = run(seg, q, k, v, do, D ** -0.5)
     # tables: each image on its own grid, within one fp32 ulp of the oracle
     cr, sr = oracle_mod.rope_tables(SAMPLES, S, D)
@@ -113,9 +113,11 @@ def test_one_image_multi_form_equals_canonical():
     assert (a[2].float() - b[2].float()).norm() <= 1e-3 * a[2].float().norm()
 
 
-def test_multi_packed_with_qk_norm_against_oracle(oracle_mod):
+@pytest.mark.parametrize("split", [0, 2])
+def test_multi_packed_with_qk_norm_against_oracle(oracle_mod, split):
     """All three options at once: several images per sample, the packed
-    layout and the QK RMSNorm, against the oracle on the padded equivalent."""
+    layout and the QK RMSNorm, against the oracle on the padded equivalent;
+    with the automatic backward schedule and with the split one forced on."""
     S = max(length(x) for x in SAMPLES) + 5
     Hq, Hkv, D, eps = 4, 2, 128, 1e-5
     q, k, v, do = inputs(S, Hq, Hkv, D, seed=3)
@@ -125,7 +127,7 @@ def test_multi_packed_with_qk_norm_against_oracle(oracle_mod):
     g = torch.Generator().manual_seed(9)
     wq = (torch.rand(D, generator=g, dtype=torch.float64) + 0.5).float()
     wk = (torch.rand(D, generator=g, dtype=torch.float64) + 0.5).float()
-    seg = jt.hia_segments_build_multi(SAMPLES, packed=True)
+    seg = jt.hia_segments_build_multi(SAMPLES, packed=True).set_bwd_split(split)
     pack = lambda x: torch.cat([x[b, :L] for b, L in enumerate(lens)], 0).contiguous()
     c, s = jt.hia_rope2d_tables(seg, D)
     qp, kp, vp, dop = (pack(t).cuda() for t in (q, k, v, do))

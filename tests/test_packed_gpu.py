@@ -59,8 +59,8 @@ def run_padded(wl, q, k, v, do):
     return [t.cpu() for t in (o, lse, dq, dk, dv)]
 
 
-def run_packed(wl, q, k, v, do, lens):
-    seg = jt.hia_segments_build_packed(wl.samples).set_bwd_split(NEVER_SPLIT)
+def run_packed(wl, q, k, v, do, lens, split=NEVER_SPLIT):
+    seg = jt.hia_segments_build_packed(wl.samples).set_bwd_split(split)
     assert seg.S <= wl.S
     c, s = gpu_tables(seg, wl.D, wl.base)
     qp, kp, vp, dop = (pack(t, lens).cuda() for t in (q, k, v, do))
@@ -88,11 +88,12 @@ def test_packed_equals_padded_on_real_rows(name):
         off += L
 
 
-@pytest.mark.parametrize("name", ["tiny", "256px"])
-def test_packed_parity_with_oracle(oracle_mod, name):
+@pytest.mark.parametrize("name,split", [("tiny", 0), ("256px", 0), ("256px", 2)])
+def test_packed_parity_with_oracle(oracle_mod, name, split):
+    """split 2: the split backward schedule forced on, in the packed layout."""
     wl = synth.workload(name)
     q, k, v, do, lens = padded_inputs(wl, 1)
-    seg, (o, lse, dq, dk, dv) = run_packed(wl, q, k, v, do, lens)
+    seg, (o, lse, dq, dk, dv) = run_packed(wl, q, k, v, do, lens, split=split)
     S = wl.S
     # the oracle on the padded equivalent, compared on real rows only
     rows_ok = np.zeros((wl.B, S), dtype=bool)

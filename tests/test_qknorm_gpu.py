@@ -26,9 +26,9 @@ def weights(D, seed=0):
     return wq, wk  # fp32-representable, so the oracle sees the kernels' exact weights
 
 
-def run(wl, wq, wk, bwd=True):
+def run(wl, wq, wk, bwd=True, split=0):
     q, k, v, do = synth.tensors(wl, 0, grad=True)
-    seg = jt.hia_segments_build(wl.samples, wl.S)
+    seg = jt.hia_segments_build(wl.samples, wl.S).set_bwd_split(split)
     c, s = gpu_tables(seg, wl.D, wl.base)
     norm = (wq.float().cuda(), wk.float().cuda(), EPS)
     qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
@@ -41,12 +41,14 @@ def run(wl, wq, wk, bwd=True):
     return (q, k, v, do), o.float().cpu().numpy(), lse.cpu().numpy(), out
 
 
-@pytest.mark.parametrize("name", ["tiny", "256px"])
-def test_qknorm_fwd_bwd_parity(oracle_mod, name):
+@pytest.mark.parametrize("name,split", [("tiny", 0), ("256px", 0), ("256px", 2)])
+def test_qknorm_fwd_bwd_parity(oracle_mod, name, split):
+    """split 2: the split backward schedule forced on, whose combine feeds the
+    norm's fp32 dk accumulator."""
     wl = synth.workload(name)
     wq, wk = weights(wl.D)
     ref_norm = (wq.numpy(), wk.numpy(), EPS)
-    (q, k, v, do), o, lse, (dq, dk, dv, dwq, dwk) = run(wl, wq, wk)
+    (q, k, v, do), o, lse, (dq, dk, dv, dwq, dwk) = run(wl, wq, wk, split=split)
     check_fwd(oracle_mod, wl, q, k, v, o, lse, qk_norm=ref_norm)
     f = lambda t: t.float().cpu().numpy()
     check_bwd(oracle_mod, wl, (q, k, v, do), (f(dq), f(dk), f(dv)), qk_norm=ref_norm,
