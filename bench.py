@@ -399,7 +399,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--e2e-inflight", type=int, default=3,
+    ap.add_argument("--e2e-inflight", type=int, default=4,
                     help="host-buffer steps in flight (each on its own stream and hia_step) in the e2e timing")
     ap.add_argument("--ref-row-stride", type=int, default=64)
     ap.add_argument("--moe-ref-tokens", type=int, default=8,
