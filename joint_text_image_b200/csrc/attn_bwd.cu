@@ -7,11 +7,14 @@
 //   dKr = scale dS^T Qr,   dQr = scale dS Kr,
 // summed over the g query heads of each kv head; dK, dQ = R^T dKr, R^T dQr.
 //
-// bwd_pre: delta and LSE * log2(e) per row, padded to a multiple of 64 rows.
-// attn_bwd: one CTA per (b, kv head, 128-key tile).  It keeps Kr and V in
-// shared memory and dK, dV in TMEM, and walks the g heads x the 64-row query
-// tiles that see its keys (a suffix of query tiles, since the row bound e(q)
-// is non-decreasing).  Per query tile, with keys on the MMA M side:
+// bwd_pre: delta and LSE * log2(e) per row, padded to a multiple of 64 rows;
+// it also zeroes the dQ accumulator and the split schedule's tickets.
+// attn_bwd: one CTA per work-list entry and kv head: a (b, 128-key tile) over
+// the query tiles that see its keys (a range of query tiles, since the row
+// bound e(q) is non-decreasing), or one half of that range for the longest
+// tiles when the split schedule is chosen (the two halves' fp32 dK/dV are
+// added by the half that finishes second).  It keeps Kr and V in shared
+// memory and dK, dV in TMEM, and walks the g heads x its query tiles.  Per query tile, with keys on the MMA M side:
 //   S^T = Kr Qr^T, dP^T = V dO^T      (SS MMAs, M=128, N=64)
 //   P^T = exp2(S^T * scale*log2e - lse2), dS^T = P^T o (dP^T - delta)
 //   dV += P^T dO,  dK += dS^T Qr       (A = P^T / dS^T straight from TMEM)

@@ -255,28 +255,43 @@ __global__ void moe_scan_kernel(MoeMeta* meta, int E, int T, int32_t* mtab) {
 }
 
 // ---------------------------------------------------------------- gather
-// Row of (token t, choice j) = offsets[e] + slot; x[t] copied there; the
-// padding rows of every routed group zeroed.  One warp per row.
+// Row of (token t, choice j) = offsets[e] + slot; x[t] is read once and
+// written to its topk rows (one warp per token, the row in registers in
+// pieces of 16 chunks of 16 bytes per lane); the padding rows of every routed
+// group are zeroed.
 __global__ void __launch_bounds__(256) moe_gather_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int topk,
                                                          int E, const int32_t* __restrict__ ids,
                                                          const int32_t* __restrict__ slot, const MoeMeta* meta,
                                                          int32_t* __restrict__ rowidx, __nv_bfloat16* __restrict__ xp) {
+  constexpr int kPiece = 16;  // 16-byte chunks per lane per pass
   const int lane = threadIdx.x & 31;
   const int nchunk = H / 8;  // 16-byte chunks per row
-  const int64_t n_pairs = int64_t(T) * topk;
   const int64_t n_warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const int64_t w0 = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
-  for (int64_t pr = w0; pr < n_pairs + int64_t(E) * kTileRows; pr += n_warps) {
-    if (pr < n_pairs) {
-      const int t = int(pr / topk);
-      const int row = meta->offsets[ids[pr]] + slot[pr];
-      if (lane == 0) rowidx[pr] = row;
-      const uint4* src = reinterpret_cast<const uint4*>(x + int64_t(t) * H);
-      uint4* dst = reinterpret_cast<uint4*>(xp + int64_t(row) * H);
-#pragma unroll 4
-      for (int c = lane; c < nchunk; c += 32) dst[c] = __ldg(src + c);
+  for (int64_t t = w0; t < T + int64_t(E) * kTileRows; t += n_warps) {
+    if (t < T) {
+      // this token's rows in the sorted order (lane j holds choice j's)
+      const int my_row = lane < topk ? meta->offsets[ids[t * topk + lane]] + slot[t * topk + lane] : 0;
+      if (lane < topk) rowidx[t * topk + lane] = my_row;
+      const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
+      for (int c0 = 0; c0 < nchunk; c0 += 32 * kPiece) {
+        uint4 v[kPiece];
+#pragma unroll
+        for (int i = 0; i < kPiece; ++i) {
+          const int c = c0 + i * 32 + lane;
+          if (c < nchunk) v[i] = __ldg(src + c);
+        }
+        for (int j = 0; j < topk; ++j) {
+          uint4* dst = reinterpret_cast<uint4*>(xp + int64_t(__shfl_sync(0xffffffffu, my_row, j)) * H);
+#pragma unroll
+          for (int i = 0; i < kPiece; ++i) {
+            const int c = c0 + i * 32 + lane;
+            if (c < nchunk) dst[c] = v[i];
+          }
+        }
+      }
     } else {
-      const int g = int((pr - n_pairs) / kTileRows), r = int((pr - n_pairs) % kTileRows);
+      const int g = int((t - T) / kTileRows), r = int((t - T) % kTileRows);
       const int n = meta->counts[g];
       if (n + r < pad_rows(n)) {
         uint4* dst = reinterpret_cast<uint4*>(xp + int64_t(meta->offsets[g] + n + r) * H);
@@ -680,7 +695,7 @@ extern "C" int hia_moe_fwd(const hia_moe_dims* d, const void* x, const float* wg
   moe_scan_kernel<<<1, 128, 0, st>>>(meta, E, T, mtab);
   prof_end(kMoeScan, st);
 
-  const int64_t gather_warps = int64_t(T) * K + int64_t(E) * kTileRows;
+  const int64_t gather_warps = int64_t(T) + int64_t(E) * kTileRows;
   prof_begin(kMoeGather, st);
   moe_gather_kernel<<<int(std::min<int64_t>((gather_warps + 7) / 8, n_sm * 8)), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(x), T, H, K, E, ids, slot, meta, rowidx, xp);

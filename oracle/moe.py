@@ -24,8 +24,8 @@ Sources (page title, section / API item):
 Readings where the pages are silent (each is listed in the design notes):
   - SwiGLU: a = silu(gate) * up with silu(z) = z / (1 + exp(-z)), then the
     down projection; routed experts use the same fused [up; gate] layout as
-    the shared one (what the adapter's "fused [up; gate] expert projections"
-    name);
+    the shared one (the coverage page's adapter turns the release's fused
+    up/gate expert weights into grouped experts);
   - top-k ties: the lower expert index is taken first;
   - the routing weights multiply each selected expert's output and the
     shared expert's output is added with weight 1;
