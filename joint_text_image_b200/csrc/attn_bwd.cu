@@ -80,7 +80,7 @@ template <int D>
 __device__ __forceinline__ void issue_kq(uint32_t d, uint64_t adesc, uint64_t bdesc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, BQ, 0, 0);
   constexpr KMajorSteps<D / 16> sa(16384), sb(8192);
-  mma_chain_ss<D / 16>(d, adesc, sa.v, bdesc, sb.v, idesc, 0u);
+  mma_chain_ss_w<D / 16>(d, adesc, sa.v, bdesc, sb.v, idesc, 0u);
 }
 
 // dV += P^T dO or dK += dS^T Qr: A from TMEM (128 keys x 64 q, packed bf16),
@@ -89,7 +89,7 @@ template <int D>
 __device__ __forceinline__ void issue_acc(uint32_t d, uint32_t a_tmem, uint64_t bdesc, bool acc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
   constexpr MNMajorSteps<BQ / 16> st;
-  mma_chain_ts<BQ / 16>(d, a_tmem, 8u, bdesc, st.v, idesc, acc ? 1u : 0u);
+  mma_chain_ts_w<BQ / 16>(d, a_tmem, 8u, bdesc, st.v, idesc, acc ? 1u : 0u);
 }
 
 // dQ^T = Kr^T dS^T: M = 128 (head dims; for D = 64 the second 64-row block
@@ -98,7 +98,7 @@ __device__ __forceinline__ void issue_acc(uint32_t d, uint32_t a_tmem, uint64_t 
 __device__ __forceinline__ void issue_dq(uint32_t d, uint64_t kt_mn_desc, uint64_t ds_desc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, BQ, 1, 1);
   constexpr MNMajorSteps<BK / 16> st;
-  mma_chain_ss<BK / 16>(d, kt_mn_desc, st.v, ds_desc, st.v, idesc, 0u);
+  mma_chain_ss_w<BK / 16>(d, kt_mn_desc, st.v, ds_desc, st.v, idesc, 0u);
 }
 
 template <int D>
@@ -195,10 +195,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Two threads issue MMAs: a wait or fence in an issuing thread lets its
     // own short MMA queue drain, and the other thread's MMAs keep the tensor
     // core busy meanwhile.  Warp 1 issues S^T and dP^T (running up to two
-    // query tiles ahead), warp 2 the dV, dK and dQ^T MMAs of each tile.
-    if (lane == 0 && n_it > 0) {
+    // query tiles ahead), warp 2 the dV, dK and dQ^T MMAs of each tile.  Each
+    // issuing warp runs its loop converged (waits combined with __all_sync)
+    // and one elected lane issues, so the descriptors are warp-uniform.
+    if (n_it > 0) {
       constexpr uint32_t kQStep = (BQ * D * 2u) >> 4, kDsStep = (BK * BQ * 2u) >> 4;
-      bool ok = mbar_wait(&sm.bar_kv, 0, wc);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_kv, 0, wc));
       if (warp == 1) {
         const uint64_t k_km = sdesc_sw128(smem_u32(sm.k), 16, 1024);
         const uint64_t v_km = sdesc_sw128(smem_u32(sm.v), 16, 1024);
@@ -208,17 +210,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int b = i & 1, s = i % kStages;
           // S^T(i) reuses the buffer whose P^T(i-2) the dV MMA read; dP^T(i)
           // the buffer the dQ writers read dQ^T(i-2) from.
-          if (!mbar_wait(&sm.bar_full[s], (i / kStages) & 1, wc)) { ok = false; break; }
-          if (i >= 2 && !mbar_wait(&sm.bar_s_free[b], ((i >> 1) - 1) & 1, wc)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_full[s], (i / kStages) & 1, wc))) { ok = false; break; }
+          if (i >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_s_free[b], ((i >> 1) - 1) & 1, wc))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           issue_kq<D>(tS[b], k_km, q_km + uint32_t(s) * kQStep);
-          tc_commit(&sm.bar_s_full[b]);
+          tc_commit_w(&sm.bar_s_full[b]);
           if (i >= 2) {
-            if (!mbar_wait(&sm.bar_dq_empty[b], ((i >> 1) - 1) & 1, wc)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dq_empty[b], ((i >> 1) - 1) & 1, wc))) {
+              ok = false;
+              break;
+            }
             tc_fence_after();  // TMEM reuse after the dQ writers' loads
           }
           issue_kq<D>(tdP[b], v_km, o_km + uint32_t(s) * kQStep);
-          tc_commit(&sm.bar_dp_full[b]);
+          tc_commit_w(&sm.bar_dp_full[b]);
         }
       } else {
         const uint64_t k_mn = sdesc_sw128(smem_u32(sm.k), D == 128 ? 16384u : smem_u32(sm.v) - smem_u32(sm.k), 1024);
@@ -228,16 +236,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; ok && i < n_it; ++i) {
           const int b = i & 1, s = i % kStages;
           // P^T(i) and dS^T(i) are in TMEM and dS^T(i) in shared memory
-          if (!mbar_wait(&sm.bar_ds_ready[b], (i >> 1) & 1, wc)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_ds_ready[b], (i >> 1) & 1, wc))) { ok = false; break; }
           tc_fence_after();
           issue_acc<D>(tdV, tS[b], o_mn + uint32_t(s) * kQStep, i > 0);
-          tc_commit(&sm.bar_s_free[b]);
+          tc_commit_w(&sm.bar_s_free[b]);
           issue_acc<D>(tdK, tdP[b], q_mn + uint32_t(s) * kQStep, i > 0);
-          tc_commit(&sm.bar_empty[s]);  // the stage's Q and dO are no longer read
+          tc_commit_w(&sm.bar_empty[s]);  // the stage's Q and dO are no longer read
           issue_dq(tdP[b], k_mn, ds_mn + uint32_t(b) * kDsStep);  // over dS^T, after the dK MMA read it
-          tc_commit(&sm.bar_dq_full[b]);
+          tc_commit_w(&sm.bar_dq_full[b]);
         }
-        tc_commit(&sm.bar_final);
+        tc_commit_w(&sm.bar_final);
         mbar_wait_hw(&sm.bar_final, 0, wc);
       }
     }

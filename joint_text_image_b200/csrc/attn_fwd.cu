@@ -68,7 +68,7 @@ template <int D>
 __device__ __forceinline__ void issue_qk(uint32_t tS, uint64_t qdesc, uint64_t kdesc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
   constexpr KMajorSteps<D / 16> st(16384);
-  mma_chain_ss<D / 16>(tS, qdesc, st.v, kdesc, st.v, idesc, 0u);
+  mma_chain_ss_w<D / 16>(tS, qdesc, st.v, kdesc, st.v, idesc, 0u);
 }
 
 // O_t (+)= P_t V: A = P_t from TMEM (packed bf16, 8 columns per 16 keys),
@@ -77,7 +77,7 @@ template <int D>
 __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint64_t vdesc, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
   constexpr MNMajorSteps<8> st;
-  mma_chain_ts<8>(tO, tP, 8u, vdesc, st.v, idesc, accumulate ? 1u : 0u);
+  mma_chain_ts_w<8>(tO, tP, 8u, vdesc, st.v, idesc, accumulate ? 1u : 0u);
 }
 
 // P = exp2(S * scale*log2e - m) for one row of 128 scores, packed to bf16
@@ -186,47 +186,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // =============================== MMA issuer
-    if (lane == 0 && n_vis > 0) {
-      uint32_t tS[2] = {tmem, tmem + 128};
-      uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+    // The whole warp runs this loop (waits combined with __all_sync) and one
+    // elected lane issues each MMA chain and commit, so the descriptors are
+    // warp-uniform values.
+    if (n_vis > 0) {
+      const uint32_t tS[2] = {tmem, tmem + 128};
+      const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
       // descriptor bases (start address of each buffer); stages are adjacent
       const uint64_t qd[2] = {sdesc_sw128(smem_u32(sm.q[0]), 16, 1024), sdesc_sw128(smem_u32(sm.q[1]), 16, 1024)};
       const uint64_t kd0 = sdesc_sw128(smem_u32(sm.k[0]), 16, 1024);
       const uint64_t vd0 = sdesc_sw128(smem_u32(sm.v[0]), 16384, 1024);
       constexpr uint32_t kStageStep = (128u * D * 2u) >> 4;  // one K or V stage, 16-byte units
-      bool ok = mbar_wait(&sm.bar_q, 0, wc) && mbar_wait(&sm.bar_k_full[0], 0, wc);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_q, 0, wc) && mbar_wait(&sm.bar_k_full[0], 0, wc));
       if (ok) {
         for (int t = 0; t < n_tiles; ++t) {
           issue_qk<D>(tS[t], qd[t], kd0);
-          tc_commit(&sm.bar_s_full[t]);
+          tc_commit_w(&sm.bar_s_full[t]);
         }
-        tc_commit(&sm.bar_k_empty[0]);
+        tc_commit_w(&sm.bar_k_empty[0]);
       }
-      // Every wait/fence in this thread lets the short MMA queue drain, so each
-      // kv step has two synchronisation points, one per query tile: (1) V(j),
-      // K(j+1) loaded and P0(j) written; (2) P1(j) written.
+      // Every wait/fence in the issuing thread lets the short MMA queue drain,
+      // so each kv step has two synchronisation points, one per query tile:
+      // (1) V(j), K(j+1) loaded and P0(j) written; (2) P1(j) written.
       for (int j = 0; ok && j < n_vis; ++j) {
         const int vs = j % kVStages, ks1 = (j + 1) % kKStages;
         const bool more = j + 1 < n_vis;
         for (int t = 0; t < n_tiles; ++t) {
           if (t == 0) {
-            ok = mbar_wait(&sm.bar_v_full[vs], (j / kVStages) & 1, wc) &&
-                 (!more || mbar_wait(&sm.bar_k_full[ks1], ((j + 1) / kKStages) & 1, wc));
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_v_full[vs], (j / kVStages) & 1, wc) &&
+                                             (!more || mbar_wait(&sm.bar_k_full[ks1], ((j + 1) / kKStages) & 1, wc)));
             if (!ok) break;
           }
-          if (!mbar_wait(&sm.bar_p_ready[t], j & 1, wc)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_p_ready[t], j & 1, wc))) { ok = false; break; }
           tc_fence_after();
           issue_pv<D>(tO[t], tS[t], vd0 + uint32_t(vs) * kStageStep, j > 0);
           if (more) {
             issue_qk<D>(tS[t], qd[t], kd0 + uint32_t(ks1) * kStageStep);
-            tc_commit(&sm.bar_s_full[t]);
+            tc_commit_w(&sm.bar_s_full[t]);
           }
         }
         if (!ok) break;
-        tc_commit(&sm.bar_v_empty[vs]);
-        if (more) tc_commit(&sm.bar_k_empty[ks1]);
+        tc_commit_w(&sm.bar_v_empty[vs]);
+        if (more) tc_commit_w(&sm.bar_k_empty[ks1]);
       }
-      for (int t = 0; t < 2; ++t) tc_commit(&sm.bar_o_final[t]);
+      for (int t = 0; t < 2; ++t) tc_commit_w(&sm.bar_o_final[t]);
       // MMAs already issued must finish before TMEM can be released.
       mbar_wait_hw(&sm.bar_o_final[0], 0, wc);
     }
@@ -254,7 +257,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float cs = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = active;
+    // the tile-list entry of the next kv tile is loaded one step ahead, off
+    // the path from "S ready" to "P written"
+    int32_t ent_next = n_vis > 0 ? __ldg(tlist) : 0;
     for (int j = 0; ok && j < n_vis; ++j) {
+      const int32_t ent = ent_next;
+      if (j + 1 < n_vis) ent_next = __ldg(tlist + j + 1);
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_s_full[t], j & 1, wc));
       if (!ok) break;
       tc_fence_after();
@@ -262,7 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_ld_wait();
-      const int32_t ent = __ldg(tlist + j);
       const bool full = (ent >> 16) != 0;
       if (!full) {
         const int k0 = (ent & 0xffff) * 128;
@@ -288,23 +295,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < 8; ++k) mp[k] = fmax3(mp[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
       const float xmax = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                                fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * cs;
+      // Lazy O rescale: decided here, applied to O_t after P_t is stored (the
+      // 128 scores are dead by then, which keeps the warp within its register
+      // budget) and before the arrival that lets PV_t(j) accumulate into O_t.
+      float f = 1.f;
+      bool rescale = false;
       if (j == 0) {
         m = xmax;
       } else {
         const bool grow = xmax > m + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, grow)) {
-          const float f = grow ? ex2_approx(m - xmax) : 1.f;
-          l *= f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(tO + c * 32, ov);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
-            tmem_st32(tO + c * 32, ov);
-          }
-          if (grow) m = xmax;
+        rescale = __any_sync(0xffffffffu, grow);
+        if (grow) {
+          f = ex2_approx(m - xmax);
+          m = xmax;
         }
       }
       uint32_t pk[64];
@@ -317,9 +320,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         exp_pack<true>(sr, cs2, nm2, pk, ls);
       else
         exp_pack<false>(sr, cs2, nm2, pk, ls);
-      l += (ls[0].x + ls[1].x) + (ls[0].y + ls[1].y);
+      l = l * f + ((ls[0].x + ls[1].x) + (ls[0].y + ls[1].y));
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      if (rescale) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tO + c * 32, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+          tmem_st32(tO + c * 32, ov);
+        }
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();  // the warp's P writes are done; one lane signals for it

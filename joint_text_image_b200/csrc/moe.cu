@@ -155,18 +155,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_wait_hw(&sm.bar_full[kb % kRouterStages], (kb / kRouterStages) & 1, wc);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    // MMA issuer: the warp runs converged, one elected lane issues
+    {
       const uint32_t idesc = idesc_bf16_f32(kTileRows, N, 0, 0);
       constexpr KMajorSteps<4> st(0);
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % kRouterStages;
-        if (!mbar_wait(&sm.bar_full[s], (kb / kRouterStages) & 1, wc)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_full[s], (kb / kRouterStages) & 1, wc))) break;
         tc_fence_after();
-        mma_chain_ss<4>(tmem, sdesc_sw128(smem_u32(sm.a[s]), 16, 1024), st.v, sdesc_sw128(smem_u32(sm.b[s]), 16, 1024),
-                        st.v, idesc, kb > 0 ? 1u : 0u);
-        tc_commit(&sm.bar_empty[s]);
+        mma_chain_ss_w<4>(tmem, sdesc_sw128(smem_u32(sm.a[s]), 16, 1024), st.v,
+                          sdesc_sw128(smem_u32(sm.b[s]), 16, 1024), st.v, idesc, kb > 0 ? 1u : 0u);
+        tc_commit_w(&sm.bar_empty[s]);
       }
-      tc_commit(&sm.bar_acc);
+      tc_commit_w(&sm.bar_acc);
       mbar_wait_hw(&sm.bar_acc, 0, wc);
     }
   } else {
@@ -418,30 +419,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // =============================== MMA issuer
-    if (lane == 0) {
+    // The warp runs converged (waits combined with __all_sync) and one elected
+    // lane issues, so the descriptors are warp-uniform values.
+    {
       constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, 256, 0, 0);
       constexpr KMajorSteps<4> st(0);
       int it = 0, tl = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++tl) {
         const int buf = tl & 1;
-        if (tl >= 2 && !mbar_wait(&sm.bar_acc_empty[buf], ((tl >> 1) - 1) & 1, wc)) break;
+        if (tl >= 2 && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_acc_empty[buf], ((tl >> 1) - 1) & 1, wc))) break;
         tc_fence_after();
         const uint32_t acc = tmem + uint32_t(buf * 256);
         for (int kb = 0; kb < p.nk; ++kb, ++it) {
           const int s = it % kStages;
-          if (!mbar_wait(&sm.bar_full[s], (it / kStages) & 1, wc)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_full[s], (it / kStages) & 1, wc))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          mma_chain_ss<4>(acc, sdesc_sw128(smem_u32(sm.a[s]), 16, 1024), st.v,
-                          sdesc_sw128(smem_u32(sm.b[s]), 16, 1024), st.v, idesc, kb > 0 ? 1u : 0u);
-          tc_commit(&sm.bar_empty[s]);
+          mma_chain_ss_w<4>(acc, sdesc_sw128(smem_u32(sm.a[s]), 16, 1024), st.v,
+                            sdesc_sw128(smem_u32(sm.b[s]), 16, 1024), st.v, idesc, kb > 0 ? 1u : 0u);
+          tc_commit_w(&sm.bar_empty[s]);
         }
-        if (ok) tc_commit(&sm.bar_acc_full[buf]);
+        if (ok) tc_commit_w(&sm.bar_acc_full[buf]);
       }
-      tc_commit(&sm.bar_final);
+      tc_commit_w(&sm.bar_final);
       mbar_wait_hw(&sm.bar_final, 0, wc);
     }
   } else {

@@ -290,6 +290,52 @@ __device__ __forceinline__ void mma_chain_ts(uint32_t d, uint32_t a_tmem, uint32
 #pragma unroll
   for (int i = 0; i < NK; ++i) mma_ts(d, a[i], b[i], idesc, i == 0 ? acc_first : 1u);
 }
+// Warp-converged forms: the whole warp runs the surrounding code (so the
+// descriptors live in uniform registers) and one elected lane issues.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(r));
+  return r != 0;
+}
+template <int NK>
+__device__ __forceinline__ void mma_chain_ss_w(uint32_t d, uint64_t abase, const uint32_t (&aoff)[NK], uint64_t bbase,
+                                               const uint32_t (&boff)[NK], uint32_t idesc, uint32_t acc_first) {
+  uint64_t a[NK], b[NK];
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    a[i] = abase + aoff[i];
+    b[i] = bbase + boff[i];
+  }
+  if (elect_one()) {
+#pragma unroll
+    for (int i = 0; i < NK; ++i) mma_ss(d, a[i], b[i], idesc, i == 0 ? acc_first : 1u);
+  }
+  __syncwarp();
+}
+template <int NK>
+__device__ __forceinline__ void mma_chain_ts_w(uint32_t d, uint32_t a_tmem, uint32_t a_step, uint64_t bbase,
+                                               const uint32_t (&boff)[NK], uint32_t idesc, uint32_t acc_first) {
+  uint64_t b[NK];
+  uint32_t a[NK];
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
+    b[i] = bbase + boff[i];
+    a[i] = a_tmem + uint32_t(i) * a_step;
+  }
+  if (elect_one()) {
+#pragma unroll
+    for (int i = 0; i < NK; ++i) mma_ts(d, a[i], b[i], idesc, i == 0 ? acc_first : 1u);
+  }
+  __syncwarp();
+}
+__device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
+  if (elect_one()) tc_commit(bar);
+  __syncwarp();
+}
 // Offsets (16-byte units) of the K-steps of a K-major SW128 operand whose
 // 64-wide K blocks are `block_bytes` apart: 32 bytes per 16-element step.
 template <int NK>
