@@ -23,6 +23,9 @@
 //   PV0(j), QK0(j+1), PV1(j), QK1(j+1)
 // so the commit that publishes S_t(j+1) also proves PV_t(j) finished: the
 // softmax warps may then rescale O_t and overwrite P_t without extra barriers.
+// PV_t(j) is issued in two halves of 64 keys: the softmax warps signal once
+// the first half of P_t is stored (and O_t rescaled) and again at the end, so
+// the first half of the PV MMAs overlaps the second half of the exponentials.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -39,7 +42,7 @@ constexpr int kThreads = 384;
 // 128*88 + 256*208 = 64512 = 384*168.  The launcher checks the compiled count first.
 constexpr int kLaunchRegs = 168;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
-constexpr int kFmaExpPairs = 4;           // of every 16 column pairs, this many use exp2_fma2
+constexpr int kFmaExpPairs = 5;           // of every 16 column pairs, this many use exp2_fma2
 
 constexpr int kKStages = 3;  // K(j+1) is awaited together with V(j), so K runs one stage deeper
 constexpr int kVStages = 2;
@@ -56,6 +59,7 @@ struct FwdSmem {
   uint64_t bar_v_full[kVStages];
   uint64_t bar_v_empty[kVStages];
   uint64_t bar_s_full[2];
+  uint64_t bar_p_half[2];
   uint64_t bar_p_ready[2];
   uint64_t bar_o_final[2];
   uint32_t tmem_base;
@@ -71,23 +75,25 @@ __device__ __forceinline__ void issue_qk(uint32_t tS, uint64_t qdesc, uint64_t k
   mma_chain_ss_w<D / 16>(tS, qdesc, st.v, kdesc, st.v, idesc, 0u);
 }
 
-// O_t (+)= P_t V: A = P_t from TMEM (packed bf16, 8 columns per 16 keys),
-// B = V tile [128 keys][D] read MN-major (D blocks 16 KB apart, 2 KB per 16 keys).
+// O_t (+)= P_t V over one half of the kv tile (keys [64 half, 64 half + 64)):
+// A = P_t from TMEM (packed bf16, 8 columns per 16 keys), B = V tile [128
+// keys][D] read MN-major (D blocks 16 KB apart, 2 KB per 16 keys).
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint64_t vdesc, bool accumulate) {
+__device__ __forceinline__ void issue_pv_half(uint32_t tO, uint32_t tP, uint64_t vdesc, int half, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
-  constexpr MNMajorSteps<8> st;
-  mma_chain_ts_w<8>(tO, tP, 8u, vdesc, st.v, idesc, accumulate ? 1u : 0u);
+  constexpr MNMajorSteps<4> st;
+  mma_chain_ts_w<4>(tO, tP + uint32_t(half * 32), 8u, vdesc + uint64_t(half * (4 * 2048 >> 4)), st.v, idesc,
+                    accumulate ? 1u : 0u);
 }
 
-// P = exp2(S * scale*log2e - m) for one row of 128 scores, packed to bf16
-// pairs, with the row sum.  kFma: kFmaExpPairs of every 16 column pairs take
+// P = exp2(S * scale*log2e - m) for column pairs [C0, C1) of one row of 128
+// scores, packed to bf16 pairs, added to the row sum.  kFma: kFmaExpPairs of every 16 column pairs take
 // exp2 on the FMA pipe, the rest on MUFU.
-template <bool kFma>
+template <bool kFma, int C0, int C1>
 __device__ __forceinline__ void exp_pack(const uint32_t (&sr)[128], float2 cs2, float2 nm2, uint32_t (&pk)[64],
                                          float2 (&ls)[2]) {
 #pragma unroll
-  for (int c = 0; c < 64; ++c) {
+  for (int c = C0; c < C1; ++c) {
     const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), cs2, nm2);
     const float2 pv = (kFma && (c & 15) < kFmaExpPairs) ? exp2_fma2(x)
                                                         : make_float2(ex2_approx(x.x), ex2_approx(x.y));
@@ -131,7 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.bar_s_full[i], 1);
-      mbar_init(&sm.bar_p_ready[i], 4);  // one arrival per softmax warp
+      mbar_init(&sm.bar_p_half[i], 4);   // one arrival per softmax warp
+      mbar_init(&sm.bar_p_ready[i], 4);
       mbar_init(&sm.bar_o_final[i], 1);
     }
     sm.abort_flag = 0;
@@ -217,9 +224,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              (!more || mbar_wait(&sm.bar_k_full[ks1], ((j + 1) / kKStages) & 1, wc)));
             if (!ok) break;
           }
+          // PV_t(j) in two halves: the first as soon as P_t's first 64 keys are
+          // stored, the second once the whole P_t is
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_p_half[t], j & 1, wc))) { ok = false; break; }
+          tc_fence_after();
+          issue_pv_half<D>(tO[t], tS[t], vd0 + uint32_t(vs) * kStageStep, 0, j > 0);
           if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_p_ready[t], j & 1, wc))) { ok = false; break; }
           tc_fence_after();
-          issue_pv<D>(tO[t], tS[t], vd0 + uint32_t(vs) * kStageStep, j > 0);
+          issue_pv_half<D>(tO[t], tS[t], vd0 + uint32_t(vs) * kStageStep, 1, true);
           if (more) {
             issue_qk<D>(tS[t], qd[t], kd0 + uint32_t(ks1) * kStageStep);
             tc_commit_w(&sm.bar_s_full[t]);
@@ -316,13 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // FULL tiles have no masked entry: part of their exponentials run on the
       // FMA pipe.  PARTIAL tiles use MUFU only, whose ex2(-inf) is exactly 0,
       // so a masked key adds nothing (exp2_fma2 bottoms out at 2^-125).
+      // First half of P (keys 0-63): stored, O_t rescaled if needed, then
+      // signalled so that the first half of PV_t(j) runs while the second half
+      // of the exponentials is computed.
       if (full)
-        exp_pack<true>(sr, cs2, nm2, pk, ls);
+        exp_pack<true, 0, 32>(sr, cs2, nm2, pk, ls);
       else
-        exp_pack<false>(sr, cs2, nm2, pk, ls);
-      l = l * f + ((ls[0].x + ls[1].x) + (ls[0].y + ls[1].y));
+        exp_pack<false, 0, 32>(sr, cs2, nm2, pk, ls);
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       if (rescale) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -336,7 +349,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      __syncwarp();  // the warp's P writes are done; one lane signals for it
+      __syncwarp();  // the warp's writes are done; one lane signals for it
+      if (lane == 0) mbar_arrive(&sm.bar_p_half[t]);
+      if (full)
+        exp_pack<true, 32, 64>(sr, cs2, nm2, pk, ls);
+      else
+        exp_pack<false, 32, 64>(sr, cs2, nm2, pk, ls);
+      l = l * f + ((ls[0].x + ls[1].x) + (ls[0].y + ls[1].y));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
       if (lane == 0) mbar_arrive(&sm.bar_p_ready[t]);
     }
     // ---- epilogue: O / l -> bf16 rows, LSE
