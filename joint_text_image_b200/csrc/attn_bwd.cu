@@ -27,7 +27,7 @@
 // 8-11 two softmax warpgroups that take alternate query tiles (one key row
 // per thread; then the dK and dV epilogues), 12-15 dQ writers (one head-dim
 // lane per thread).  setmaxnreg moves registers from the producer/MMA and dQ
-// warpgroups to the softmax warpgroups: 128*80 + 256*168 + 128*96 = 65536 = 512*128.
+// warpgroups to the softmax warpgroups: 128*64 + 256*176 + 128*96 = 65536 = 512*128.
 // P^T and dS^T become visible to the second MMA thread together (one barrier
 // per tile).  TMEM: S^T[2] at 0/64, dP^T[2] at 128/192 (P^T, dS^T written over them as
 // packed bf16), dV at 256, dK at 256 + D; dQ^T of buffer i is written over
@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D;
 
   if (warp < 4) {
-   regs_dec<80>();
+   regs_dec<64>();
    if (warp == 0) {
     // =============================== TMA producer
     if (lane == 0 && n_it > 0) {
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
    }
   } else if (warp < 12) {
-    regs_inc<168>();
+    regs_inc<176>();
     // =============================== softmax: one key row per thread
     const int bf = (warp - 4) >> 2;  // this warpgroup's TMEM / dS buffer and iteration parity
     const int quarter = warp & 3;

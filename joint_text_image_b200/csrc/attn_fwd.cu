@@ -38,8 +38,8 @@ namespace {
 
 constexpr int kThreads = 384;
 // Register split (setmaxnreg): launch budget 384 x 168; warpgroup 0 (TMA, MMA)
-// drops to 88, the two softmax warpgroups rise to 208:
-// 128*88 + 256*208 = 64512 = 384*168.  The launcher checks the compiled count first.
+// drops to 72, the two softmax warpgroups rise to 216:
+// 128*72 + 256*216 = 64512 = 384*168.  The launcher checks the compiled count first.
 constexpr int kLaunchRegs = 168;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 constexpr int kFmaExpPairs = 5;           // of every 16 column pairs, this many use exp2_fma2
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wc{&sm.abort_flag, p.status, p.timeout_ns};
 
   if (warp < 4) {
-   regs_dec<88>();
+   regs_dec<72>();
    if (warp == 0) {
     // =============================== TMA producer
     if (lane == 0 && n_vis > 0) {
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
    }
   } else {
-    regs_inc<208>();
+    regs_inc<216>();
     // =============================== softmax / epilogue
     // tcgen05.ld/st are warp-collective: every branch around them below is
     // warp-uniform (waits are combined with __all_sync, the O rescale is
