@@ -152,8 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const WaitCtx wc{&sm.abort_flag, p.status, p.timeout_ns};
-  const uint32_t tS[2] = {tmem, tmem + 64};
-  const uint32_t tdP[2] = {tmem + 128, tmem + 192};
+  // buffer i of S^T / dP^T as arithmetic (a runtime-indexed array would live in local memory)
+  const auto tS = [tmem](int i) { return tmem + uint32_t(i) * 64u; };
+  const auto tdP = [tmem](int i) { return tmem + 128u + uint32_t(i) * 64u; };
   const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D;
 
   if (warp < 4) {
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          issue_kq<D>(tS[b], k_km, q_km + uint32_t(s) * kQStep);
+          issue_kq<D>(tS(b), k_km, q_km + uint32_t(s) * kQStep);
           tc_commit_w(&sm.bar_s_full[b]);
           if (i >= 2) {
             if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dq_empty[b], ((i >> 1) - 1) & 1, wc))) {
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();  // TMEM reuse after the dQ writers' loads
           }
-          issue_kq<D>(tdP[b], v_km, o_km + uint32_t(s) * kQStep);
+          issue_kq<D>(tdP(b), v_km, o_km + uint32_t(s) * kQStep);
           tc_commit_w(&sm.bar_dp_full[b]);
         }
       } else {
@@ -238,11 +239,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // P^T(i) and dS^T(i) are in TMEM and dS^T(i) in shared memory
           if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_ds_ready[b], (i >> 1) & 1, wc))) { ok = false; break; }
           tc_fence_after();
-          issue_acc<D>(tdV, tS[b], o_mn + uint32_t(s) * kQStep, i > 0);
+          issue_acc<D>(tdV, tS(b), o_mn + uint32_t(s) * kQStep, i > 0);
           tc_commit_w(&sm.bar_s_free[b]);
-          issue_acc<D>(tdK, tdP[b], q_mn + uint32_t(s) * kQStep, i > 0);
+          issue_acc<D>(tdK, tdP(b), q_mn + uint32_t(s) * kQStep, i > 0);
           tc_commit_w(&sm.bar_empty[s]);  // the stage's Q and dO are no longer read
-          issue_dq(tdP[b], k_mn, ds_mn + uint32_t(b) * kDsStep);  // over dS^T, after the dK MMA read it
+          issue_dq(tdP(b), k_mn, ds_mn + uint32_t(b) * kDsStep);  // over dS^T, after the dK MMA read it
           tc_commit_w(&sm.bar_dq_full[b]);
         }
         tc_commit_w(&sm.bar_final);
@@ -274,9 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[64];
-      tmem_ld32(tS[bf] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tS[bf] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld_wait();
+      tmem_ld32(tS(bf) + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS(bf) + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld_wait_regs(sr);
       float pv[64];
       const float4* l2 = reinterpret_cast<const float4*>(sm.lse2[s]);
 #pragma unroll
@@ -296,14 +297,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
-      tmem_st32(tS[bf] + lane_off, pk);
+      tmem_st32(tS(bf) + lane_off, pk);
 
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_dp_full[bf], (i >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      tmem_ld32(tdP[bf] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tdP[bf] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld_wait();
+      tmem_ld32(tdP(bf) + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tdP(bf) + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld_wait_regs(sr);
       const float4* dl = reinterpret_cast<const float4*>(sm.delta[s]);
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         pk[2 * c4 + 1] = pack_bf16x2(pv[4 * c4 + 2] * (__uint_as_float(sr[4 * c4 + 2]) - d.z),
                                      pv[4 * c4 + 3] * (__uint_as_float(sr[4 * c4 + 3]) - d.w));
       }
-      tmem_st32(tdP[bf] + lane_off, pk);
+      tmem_st32(tdP(bf) + lane_off, pk);
       // dS^T row -> shared memory, 128-byte swizzled rows of 64 query values
       uint8_t* dsrow = reinterpret_cast<uint8_t*>(sm.ds[bf]);
 #pragma unroll
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t v[32];
         if (have) {
           tmem_ld32(tacc + uint32_t(c * 32), v);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(v);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0u;
@@ -373,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(tacc + uint32_t(c * 32), v);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(v);
           const float4* o4 = reinterpret_cast<const float4*>(other + c * 32);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -400,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ov[32];
         if (have) {
           tmem_ld32(tdK + lane_off + c * 32, ov);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(ov);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = 0u;
@@ -424,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (have) {
           tmem_ld32(tdK + lane_off + c * 32, lo);
           tmem_ld32(tdK + lane_off + D / 2 + c * 32, hi);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(lo, hi);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) lo[i] = hi[i] = 0u;
@@ -461,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ov[32];
         if (have) {
           tmem_ld32(tdV + lane_off + c * 32, ov);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(ov);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = 0u;
@@ -493,9 +494,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t a[64];
       if (live) {
-        tmem_ld32(tdP[bf] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-        tmem_ld32(tdP[bf] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
-        tmem_ld_wait();
+        tmem_ld32(tdP(bf) + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+        tmem_ld32(tdP(bf) + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+        tmem_ld_wait_regs(a);
       }
       tc_fence_before();
       __syncwarp();

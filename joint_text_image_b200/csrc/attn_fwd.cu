@@ -266,6 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // context images this row no longer sees (only samples with several images)
     int n_hidden = 0;
     for (int i = 0; i < smp.n_img; ++i) n_hidden += (im[i].hidden && im[i].I1 <= q) ? 1 : 0;
+    // warp-uniform: the masking loop below must not leave the warp diverged
+    // before the warp-collective TMEM stores
+    const bool warp_hidden = __any_sync(0xffffffffu, n_hidden > 0);
     const float cs = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = active;
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sr[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-      tmem_ld_wait();
+      tmem_ld_wait_regs(sr);
       const bool full = (ent >> 16) != 0;
       if (!full) {
         const int k0 = (ent & 0xffff) * 128;
@@ -289,14 +292,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c > lim) sr[c] = __float_as_uint(-INFINITY);
-        for (int i = 0; n_hidden > 0 && i < smp.n_img; ++i) {
-          if (!im[i].hidden || im[i].I1 > q) continue;
+        for (int i = 0; warp_hidden && i < smp.n_img; ++i) {
+          const bool hide = im[i].hidden && im[i].I1 <= q;  // per row: applied by selects
           const int lo = im[i].I0 - k0, n = im[i].I1 - im[i].I0;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (unsigned(c - lo) < unsigned(n)) sr[c] = __float_as_uint(-INFINITY);
+            if (hide && unsigned(c - lo) < unsigned(n)) sr[c] = __float_as_uint(-INFINITY);
         }
       }
+      __syncwarp();
       // row max with 8 independent partial maxima (short dependency chains)
       float mp[8];
 #pragma unroll
@@ -322,6 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = xmax;
         }
       }
+      __syncwarp();  // converged again after the per-row rescale decision
       uint32_t pk[64];
       float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       const float2 cs2 = make_float2(cs, cs), nm2 = make_float2(-m, -m);
@@ -341,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
           tmem_ld32(tO + c * 32, ov);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(ov);
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
           tmem_st32(tO + c * 32, ov);
@@ -381,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ov[32];
         if (have) {
           tmem_ld32(tO + c * 32, ov);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(ov);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = 0u;

@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int c = 0; c < N; c += 16) {
         uint32_t v[16];
         tmem_ld16(tmem + lane_off + uint32_t(c), v);
-        tmem_ld_wait();
+        tmem_ld_wait_regs(v);
         const int part = c / p.Ep, e0 = c % p.Ep;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint32_t up[32], gt[32];
           tmem_ld32(acc + uint32_t(c), up);
           tmem_ld32(acc + uint32_t(128 + c), gt);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(up, gt);
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -487,7 +487,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int c = 0; c < 256; c += 32) {
           uint32_t v[32];
           tmem_ld32(acc + uint32_t(c), v);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(v);
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));

@@ -217,6 +217,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// tcgen05.ld writes its destination registers asynchronously: they hold the
+// loaded values only after tcgen05.wait::ld.  To the compiler they are defined
+// by the load statement itself, so it could schedule a use of them before the
+// wait.  reg_fence (an empty statement that reads and rewrites the registers,
+// ordered after the wait like every volatile asm) pins every later use after
+// the wait; tmem_ld_wait_regs is the wait followed by that fence.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
+  static_assert(N % 8 == 0, "whole groups of 8 registers");
+#pragma unroll
+  for (int i = 0; i < N; i += 8)
+    asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]),
+                 "+r"(r[i + 6]), "+r"(r[i + 7]));
+}
+template <class... R>
+__device__ __forceinline__ void tmem_ld_wait_regs(R&... regs) {
+  tmem_ld_wait();
+  (reg_fence(regs), ...);
+}
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
