@@ -294,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 64; ++c)
           if (q0 + c < vis_lo || q0 + c >= vis_hi) pv[c] = 0.f;
       }
+      __syncwarp();  // converged before the warp-collective TMEM store
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);

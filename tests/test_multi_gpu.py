@@ -158,3 +158,36 @@ def test_multi_packed_with_qk_norm_against_oracle(oracle_mod, split):
         assert np.linalg.norm(a - r) / np.linalg.norm(r) <= GRAD_REL, name
     for got, ref in ((dwq, rdwq), (dwk, rdwk)):
         assert np.linalg.norm(got.cpu().numpy() - ref) / np.linalg.norm(ref) <= GRAD_REL
+
+
+def test_multi_image_forward_repeated_with_held_allocations(oracle_mod):
+    """The several-images step (D = 128) repeated with differently sized
+    allocations held alive between calls, so that the inputs, tables,
+    workspaces and outputs land at other addresses each time, and with a
+    backward between forwards.  Warps that run the per-row hidden-image
+    masking once returned wrong forward rows on some boxes in exactly this
+    pattern (every row of such a warp, the same values every call: the warp
+    reached the warp-collective TMEM stores diverged); each forward must
+    match the oracle."""
+    S = max(length(x) for x in SAMPLES) + 17
+    Hq, Hkv, D = 4, 2, 128
+    q, k, v, do = inputs(S, Hq, Hkv, D)
+    f64 = lambda t: t.double().numpy()
+    o_ref = oracle_mod.attn_fwd(SAMPLES, f64(q), f64(k), f64(v), D ** -0.5)[0]
+    rng = np.random.default_rng(0)
+    held = []
+    for it in range(8):
+        held.append(torch.full((int(rng.integers(1, 3_000_000)),), float("nan"), device="cuda"))
+        if len(held) > 6:
+            held.pop(0)
+        seg = jt.hia_segments_build_multi(SAMPLES, S).set_bwd_split([0, 2, 1][it % 3])
+        c, s = jt.hia_rope2d_tables(seg, D)
+        qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+        o, lse = jt.hia_attn_fwd(seg, qd, kd, vd, c, s, D ** -0.5)
+        torch.cuda.synchronize()
+        assert jt.hia_get_device_status() == 0
+        err = np.abs(o.float().cpu().numpy() - o_ref)
+        assert err.max() <= O_MAX and err.mean() <= O_MEAN, (it, float(err.max()))
+        jt.hia_attn_bwd(seg, qd, kd, vd, c, s, o, lse, dod, D ** -0.5)
+        torch.cuda.synchronize()
+        assert jt.hia_get_device_status() == 0
