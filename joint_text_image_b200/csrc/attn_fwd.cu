@@ -321,12 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const bool grow = xmax > m + kRescaleThreshold;
         rescale = __any_sync(0xffffffffu, grow);
-        if (grow) {
-          f = ex2_approx(m - xmax);
-          m = xmax;
-        }
+        // selects, not a branch: the warp stays converged for the TMEM stores
+        const float fg = ex2_approx(m - xmax);
+        f = grow ? fg : 1.f;
+        m = grow ? xmax : m;
       }
-      __syncwarp();  // converged again after the per-row rescale decision
       uint32_t pk[64];
       float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       const float2 cs2 = make_float2(cs, cs), nm2 = make_float2(-m, -m);
