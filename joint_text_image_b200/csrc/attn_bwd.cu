@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 || warp == 2) {
     // =============================== MMA issuers
-    // Two threads issue MMAs: a wait or fence in an issuing thread lets its
+    // Two warps issue MMAs: a wait or fence in an issuing thread lets its
     // own short MMA queue drain, and the other thread's MMAs keep the tensor
     // core busy meanwhile.  Warp 1 issues S^T and dP^T (running up to two
     // query tiles ahead), warp 2 the dV, dK and dQ^T MMAs of each tile.  Each
@@ -392,6 +392,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (write_out && threadIdx.x == 128) p.part_cnt[slot * p.Hkv + hkv] = 0;  // ready for the next launch
     }
     const bool store = write_out && key < smp.rows;
+    // dK / dV rows leave through shared memory: each thread stages its key
+    // row's 16-byte chunks, XOR-swizzled by row so that a warp's 32 row writes
+    // spread over the banks, then each warp writes its own 32 rows whole
+    // (CPR lanes per row, 16 bytes each: coalesced 128-bit stores).
+    constexpr int CPR = D / 8;  // 16-byte chunks per bf16 row
+    const auto stage_chunk = [](uint8_t* tile, int row, int ch, uint4 v) {
+      *reinterpret_cast<uint4*>(tile + row * (D * 2) + ((ch ^ (row & (CPR - 1))) * 16)) = v;
+    };
+    const auto store_rows = [&](const uint8_t* tile, __nv_bfloat16* base, int64_t row_stride) {
+      constexpr int RPI = 32 / CPR;  // rows per warp store
+      const int ch = lane % CPR;
+#pragma unroll 4
+      for (int rr = 0; rr < 32; rr += RPI) {
+        const int row = quarter * 32 + rr + lane / CPR;
+        if (write_out && kt * BK + row < smp.rows) {
+          const uint4 v = *reinterpret_cast<const uint4*>(tile + row * (D * 2) + ((ch ^ (row & (CPR - 1))) * 16));
+          *reinterpret_cast<uint4*>(base + int64_t(smp.off + kt * BK + row) * row_stride + ch * 8) = v;
+        }
+      }
+    };
     if (bf == 0 && p.dk_acc) {
       // QK RMSNorm: the norm's backward needs the whole row, so write
       // scale * dK_n (gradient w.r.t. the normed rotated key row) in fp32 and
@@ -419,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kc = store ? key : 0;  // read only when storing
       const float* cp = p.cos_t + (int64_t(b) * p.S + kc) * D;
       const float* sp = p.sin_t + (int64_t(b) * p.S + kc) * D;
-      __nv_bfloat16* dkrow = p.dk + int64_t(b) * p.dk_sb + int64_t(smp.off + key) * p.dk_ss + int64_t(hkv) * p.dk_sh;
+      uint8_t* tile = reinterpret_cast<uint8_t*>(sm.k);  // K is no longer read: every MMA has finished
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t lo[32], hi[32];
@@ -447,17 +467,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             olo[i] = pack_bf16x2(a[0], a[1]);
             ohi[i] = pack_bf16x2(bb[0], bb[1]);
           }
-          uint4* d0 = reinterpret_cast<uint4*>(dkrow + c * 32);
-          uint4* d1 = reinterpret_cast<uint4*>(dkrow + D / 2 + c * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            d0[i] = make_uint4(olo[4 * i], olo[4 * i + 1], olo[4 * i + 2], olo[4 * i + 3]);
-            d1[i] = make_uint4(ohi[4 * i], ohi[4 * i + 1], ohi[4 * i + 2], ohi[4 * i + 3]);
+            stage_chunk(tile, r, c * 4 + i, make_uint4(olo[4 * i], olo[4 * i + 1], olo[4 * i + 2], olo[4 * i + 3]));
+            stage_chunk(tile, r, D / 16 + c * 4 + i,
+                        make_uint4(ohi[4 * i], ohi[4 * i + 1], ohi[4 * i + 2], ohi[4 * i + 3]));
           }
         }
       }
+      __syncwarp();
+      store_rows(tile, p.dk + int64_t(b) * p.dk_sb + int64_t(hkv) * p.dk_sh, p.dk_ss);
     } else {
-      __nv_bfloat16* dvrow = p.dv + int64_t(b) * p.dv_sb + int64_t(smp.off + key) * p.dv_ss + int64_t(hkv) * p.dv_sh;
+      uint8_t* tile = reinterpret_cast<uint8_t*>(sm.v);  // V is no longer read: every MMA has finished
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -469,15 +490,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) ov[i] = 0u;
         }
         if (store) {
-          uint4* d0 = reinterpret_cast<uint4*>(dvrow + c * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            d0[i] = make_uint4(pack_bf16x2(__uint_as_float(ov[8 * i]), __uint_as_float(ov[8 * i + 1])),
-                               pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3])),
-                               pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5])),
-                               pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7])));
+            stage_chunk(tile, r, c * 4 + i,
+                        make_uint4(pack_bf16x2(__uint_as_float(ov[8 * i]), __uint_as_float(ov[8 * i + 1])),
+                                   pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3])),
+                                   pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5])),
+                                   pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7]))));
         }
       }
+      __syncwarp();
+      store_rows(tile, p.dv + int64_t(b) * p.dv_sb + int64_t(hkv) * p.dv_sh, p.dv_ss);
     }
   } else {
     // =============================== dQ writers: one head-dim lane per thread

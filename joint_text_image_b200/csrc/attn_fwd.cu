@@ -14,7 +14,8 @@
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q tiles once, then K tiles (3-stage ring) and V
 //               tiles (2-stage ring)
-//   warp 1      TMEM owner and single-thread tcgen05.mma issuer
+//   warp 1      TMEM owner and tcgen05.mma issuer (the warp runs converged,
+//               one elected lane issues)
 //   warps 4-7   softmax / correction / epilogue of tile 0 (one row per thread)
 //   warps 8-11  the same for tile 1
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 after it;
