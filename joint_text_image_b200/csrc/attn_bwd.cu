@@ -400,7 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const auto stage_chunk = [](uint8_t* tile, int row, int ch, uint4 v) {
       *reinterpret_cast<uint4*>(tile + row * (D * 2) + ((ch ^ (row & (CPR - 1))) * 16)) = v;
     };
-    const auto store_rows = [&](const uint8_t* tile, __nv_bfloat16* base, int64_t row_stride) {
+    // rows of D * 2 bytes: a bf16 row, or half of an fp32 row; destination row
+    // row0 + r of `base` (row_bytes apart) gets tile row r
+    const auto store_rows = [&](const uint8_t* tile, uint8_t* base, int64_t row0, int64_t row_bytes) {
       constexpr int RPI = 32 / CPR;  // rows per warp store
       const int ch = lane % CPR;
 #pragma unroll 4
@@ -408,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = quarter * 32 + rr + lane / CPR;
         if (write_out && kt * BK + row < smp.rows) {
           const uint4 v = *reinterpret_cast<const uint4*>(tile + row * (D * 2) + ((ch ^ (row & (CPR - 1))) * 16));
-          *reinterpret_cast<uint4*>(base + int64_t(smp.off + kt * BK + row) * row_stride + ch * 8) = v;
+          *reinterpret_cast<uint4*>(base + (row0 + row) * row_bytes + ch * 16) = v;
         }
       }
     };
@@ -416,24 +418,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       // QK RMSNorm: the norm's backward needs the whole row, so write
       // scale * dK_n (gradient w.r.t. the normed rotated key row) in fp32 and
       // let the gradient epilogue kernel finish it
-      float* arow = p.dk_acc + ((int64_t(b) * p.Hkv + hkv) * p.S_pad + key) * D;
+      // fp32 rows of D * 4 bytes, staged half a row (D * 2 bytes) at a time
+      uint8_t* tile = reinterpret_cast<uint8_t*>(sm.k);  // K is no longer read: every MMA has finished
+      uint8_t* abase = reinterpret_cast<uint8_t*>(p.dk_acc + (int64_t(b) * p.Hkv + hkv) * p.S_pad * D);
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        if (have) {
-          tmem_ld32(tdK + lane_off + c * 32, ov);
-          tmem_ld_wait_regs(ov);
-        } else {
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t ov[32];
+          if (have) {
+            tmem_ld32(tdK + lane_off + half * (D / 2) + c * 32, ov);
+            tmem_ld_wait_regs(ov);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = 0u;
-        }
-        if (store) {
-          float4* d0 = reinterpret_cast<float4*>(arow + c * 32);
+            for (int i = 0; i < 32; ++i) ov[i] = 0u;
+          }
+          if (store) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d0[i] = make_float4(__uint_as_float(ov[4 * i]) * p.scale, __uint_as_float(ov[4 * i + 1]) * p.scale,
-                                __uint_as_float(ov[4 * i + 2]) * p.scale, __uint_as_float(ov[4 * i + 3]) * p.scale);
+            for (int i = 0; i < 8; ++i)
+              stage_chunk(tile, r, c * 8 + i,
+                          make_uint4(__float_as_uint(__uint_as_float(ov[4 * i]) * p.scale),
+                                     __float_as_uint(__uint_as_float(ov[4 * i + 1]) * p.scale),
+                                     __float_as_uint(__uint_as_float(ov[4 * i + 2]) * p.scale),
+                                     __float_as_uint(__uint_as_float(ov[4 * i + 3]) * p.scale)));
+          }
         }
+        __syncwarp();
+        store_rows(tile, abase + half * (D / 2) * 4, kt * BK, int64_t(D) * 4);
+        __syncwarp();  // the tile is staged again for the second half
       }
     } else if (bf == 0) {
       const int kc = store ? key : 0;  // read only when storing
@@ -476,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-      store_rows(tile, p.dk + int64_t(b) * p.dk_sb + int64_t(hkv) * p.dk_sh, p.dk_ss);
+      store_rows(tile, reinterpret_cast<uint8_t*>(p.dk + int64_t(b) * p.dk_sb + int64_t(hkv) * p.dk_sh),
+                 smp.off + kt * BK, p.dk_ss * 2);
     } else {
       uint8_t* tile = reinterpret_cast<uint8_t*>(sm.v);  // V is no longer read: every MMA has finished
 #pragma unroll 1
@@ -500,7 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-      store_rows(tile, p.dv + int64_t(b) * p.dv_sb + int64_t(hkv) * p.dv_sh, p.dv_ss);
+      store_rows(tile, reinterpret_cast<uint8_t*>(p.dv + int64_t(b) * p.dv_sb + int64_t(hkv) * p.dv_sh),
+                 smp.off + kt * BK, p.dv_ss * 2);
     }
   } else {
     // =============================== dQ writers: one head-dim lane per thread
