@@ -191,3 +191,51 @@ def test_multi_image_forward_repeated_with_held_allocations(oracle_mod):
         jt.hia_attn_bwd(seg, qd, kd, vd, c, s, o, lse, dod, D ** -0.5)
         torch.cuda.synchronize()
         assert jt.hia_get_device_status() == 0
+
+
+def _random_case(rng):
+    """A random batch of samples with up to three images each (text gaps,
+    image sizes and tails drawn at random; empty and text-only samples
+    included), a random GQA group size and head dim."""
+    B = int(rng.integers(1, 4))
+    samples = []
+    for _ in range(B):
+        segs = []
+        for _ in range(int(rng.integers(0, 4))):
+            segs.append((int(rng.integers(0, 81)), int(rng.integers(1, 17)), int(rng.integers(1, 17))))
+        samples.append((segs, int(rng.integers(0, 41))))
+    S = max(max(length(x) for x in samples), 1) + int(rng.integers(0, 41))
+    Hkv = int(rng.integers(1, 4))
+    g = int(rng.integers(1, 5))
+    D = int(rng.choice([64, 128]))
+    return samples, S, g * Hkv, Hkv, D
+
+
+@pytest.mark.parametrize("case", range(16))
+def test_multi_image_random_configs(oracle_mod, case):
+    """Seeded random several-images batches (ragged lengths, empty samples,
+    g from 1 to 4, D = 64 or 128, both backward schedules): forward and
+    backward against the oracle."""
+    rng = np.random.default_rng(1000 + case)
+    samples, S, Hq, Hkv, D = _random_case(rng)
+    g = torch.Generator().manual_seed(case)
+    B = len(samples)
+    q = torch.randn(B, S, Hq, D, generator=g).bfloat16()
+    k = torch.randn(B, S, Hkv, D, generator=g).bfloat16()
+    v = torch.randn(B, S, Hkv, D, generator=g).bfloat16()
+    do = torch.randn(B, S, Hq, D, generator=g).bfloat16()
+    seg = jt.hia_segments_build_multi(samples, S).set_bwd_split(2 * (case % 2))
+    (o, lse, dq, dk, dv), _ = run(seg, q, k, v, do, D ** -0.5)
+    f64 = lambda t: t.double().numpy()
+    o_ref, lse_ref, _ = oracle_mod.attn_fwd(samples, f64(q), f64(k), f64(v), D ** -0.5)
+    err = np.abs(o.float().numpy() - o_ref)
+    assert err.max() <= O_MAX and err.mean() <= O_MEAN, (samples, S, Hq, Hkv, D, float(err.max()))
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lse.numpy()), fin)
+    if fin.any():
+        assert np.abs(lse.numpy()[fin] - lse_ref[fin]).max() <= LSE_MAX
+    refs = oracle_mod.attn_bwd(samples, f64(q), f64(k), f64(v), f64(do), D ** -0.5)[:3]
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
+        nr = np.linalg.norm(ref)
+        diff = np.linalg.norm(got.float().numpy() - ref)
+        assert (diff <= GRAD_REL * nr) if nr > 0 else diff == 0, (name, samples, S, Hq, Hkv, D)
