@@ -283,10 +283,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
         const float4 l = l2[c4];
-        pv[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 0]), cs, -l.x));
-        pv[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), cs, -l.y));
-        pv[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), cs, -l.z));
-        pv[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), cs, -l.w));
+        // scale and subtract as packed f32x2 (two columns per instruction)
+        const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[4 * c4 + 0]), __uint_as_float(sr[4 * c4 + 1])),
+                                     make_float2(cs, cs), make_float2(-l.x, -l.y));
+        const float2 xb = __ffma2_rn(make_float2(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
+                                     make_float2(cs, cs), make_float2(-l.z, -l.w));
+        pv[4 * c4 + 0] = ex2_approx(xa.x);
+        pv[4 * c4 + 1] = ex2_approx(xa.y);
+        pv[4 * c4 + 2] = ex2_approx(xb.x);
+        pv[4 * c4 + 3] = ex2_approx(xb.y);
       }
       if (partial) {
         const int q0 = qt * BQ;
