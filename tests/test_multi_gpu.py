@@ -239,3 +239,65 @@ def test_multi_image_random_configs(oracle_mod, case):
         nr = np.linalg.norm(ref)
         diff = np.linalg.norm(got.float().numpy() - ref)
         assert (diff <= GRAD_REL * nr) if nr > 0 else diff == 0, (name, samples, S, Hq, Hkv, D)
+
+
+@pytest.mark.parametrize("case", range(8))
+def test_multi_image_random_packed_and_norm(oracle_mod, case):
+    """Seeded random several-images batches in the packed layout, half of them
+    with the QK RMSNorm, against the oracle on the padded equivalent (padded
+    rows get zero dO, so they add nothing to dk, dv)."""
+    rng = np.random.default_rng(2000 + case)
+    samples, S, Hq, Hkv, D = _random_case(rng)
+    lens = [length(x) for x in samples]
+    if sum(lens) == 0:
+        samples[0] = ([(3, 2, 2)], 1)
+        lens = [length(x) for x in samples]
+        S = max(S, lens[0])
+    g = torch.Generator().manual_seed(100 + case)
+    B = len(samples)
+    q = torch.randn(B, S, Hq, D, generator=g).bfloat16()
+    k = torch.randn(B, S, Hkv, D, generator=g).bfloat16()
+    v = torch.randn(B, S, Hkv, D, generator=g).bfloat16()
+    do = torch.randn(B, S, Hq, D, generator=g).bfloat16()
+    for b, L in enumerate(lens):
+        do[b, L:] = 0
+    norm = case % 2 == 1
+    eps = 1e-5
+    wq = (torch.rand(D, generator=g, dtype=torch.float64) + 0.5).float()
+    wk = (torch.rand(D, generator=g, dtype=torch.float64) + 0.5).float()
+    seg = jt.hia_segments_build_multi(samples, packed=True).set_bwd_split(2 * ((case // 2) % 2))
+    pack = lambda x: torch.cat([x[b, :L] for b, L in enumerate(lens)], 0).contiguous()
+    c, s = jt.hia_rope2d_tables(seg, D)
+    qp, kp, vp, dop = (pack(t).cuda() for t in (q, k, v, do))
+    qn = (wq.cuda(), wk.cuda(), eps) if norm else None
+    o, lse = jt.hia_attn_fwd(seg, qp, kp, vp, c, s, qk_norm=qn)
+    out = jt.hia_attn_bwd(seg, qp, kp, vp, c, s, o, lse, dop, qk_norm=qn)
+    torch.cuda.synchronize()
+    assert jt.hia_get_device_status() == 0
+    dq, dk, dv = out[:3]
+    f64 = lambda t: t.double().numpy()
+    ref_norm = (wq.double().numpy(), wk.double().numpy(), eps) if norm else None
+    o_ref, lse_ref, _ = oracle_mod.attn_fwd(samples, f64(q), f64(k), f64(v), D ** -0.5, qk_norm=ref_norm)
+    if norm:
+        rdq, rdk, rdv, rdwq, rdwk, _ = oracle_mod.attn_bwd_qknorm(samples, f64(q), f64(k), f64(v), f64(do), ref_norm,
+                                                                  D ** -0.5)
+    else:
+        rdq, rdk, rdv = oracle_mod.attn_bwd(samples, f64(q), f64(k), f64(v), f64(do), D ** -0.5)[:3]
+    off = 0
+    errs, grads = [], {"dq": ([], []), "dk": ([], []), "dv": ([], [])}
+    for b, L in enumerate(lens):
+        errs.append(np.abs(o[off:off + L].float().cpu().numpy() - o_ref[b, :L]).ravel())
+        lr = lse_ref[b, :, :L]
+        assert np.abs(lse[:, off:off + L].cpu().numpy() - lr).max() <= LSE_MAX
+        for name, got, ref in (("dq", dq, rdq), ("dk", dk, rdk), ("dv", dv, rdv)):
+            grads[name][0].append(got[off:off + L].float().cpu().numpy().ravel())
+            grads[name][1].append(ref[b, :L].ravel())
+        off += L
+    e = np.concatenate(errs)
+    assert e.max() <= O_MAX and e.mean() <= O_MEAN, (samples, Hq, Hkv, D, norm)
+    for name, (a, r) in grads.items():
+        a, r = np.concatenate(a), np.concatenate(r)
+        assert np.linalg.norm(a - r) <= GRAD_REL * np.linalg.norm(r), (name, samples, Hq, Hkv, D, norm)
+    if norm:
+        for got, ref in ((out[3], rdwq), (out[4], rdwk)):
+            assert np.linalg.norm(got.cpu().numpy() - ref) <= GRAD_REL * np.linalg.norm(ref)
