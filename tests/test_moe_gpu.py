@@ -121,6 +121,21 @@ def test_moe_edge_shapes(T, H, I, E, topk):
         assert np.all(w == 1.0)
 
 
+@pytest.mark.parametrize("case", range(6))
+def test_moe_random_shapes(case):
+    """Seeded random sizes inside the supported range (H a multiple of 256, I
+    of 128, 1 <= E <= 80, top-k up to min(E, 16), ragged token counts): routing,
+    weights and output against the oracle."""
+    rng = np.random.default_rng(300 + case)
+    E = int(rng.integers(1, 81))
+    topk = int(rng.integers(1, min(E, 16) + 1))
+    mw = synth.MoeWorkload("random", int(rng.integers(1, 700)), 256 * int(rng.integers(1, 4)),
+                           128 * int(rng.integers(1, 4)), E, topk)
+    x, wg, w13, w2 = synth.moe_tensors(mw, 10 + case)
+    out, ids, w = run(x, wg, w13, w2, mw.topk)
+    check(x, wg, w13, w2, mw.topk, out, ids, w)
+
+
 def test_moe_all_tokens_to_one_expert():
     """A router that sends every token to expert 3 (imbalance: one group of T
     rows, the others nearly empty)."""
