@@ -24,13 +24,13 @@
 // reduce-add into the dq accumulator (the reduction runs in L2).
 // Warps (512 threads): 0 TMA producer, 1 TMEM owner + S^T/dP^T MMA issuer,
 // 2 dV/dK/dQ^T MMA issuer, 4-7 and
-// 8-11 two softmax warpgroups that take alternate query tiles (one key row
-// per thread; then the dK and dV epilogues), 12-15 dQ writers (one head-dim
-// lane per thread).  setmaxnreg moves registers from the producer/MMA and dQ
+// 8-11 two softmax warpgroups that share every query tile, one half of its
+// 64 query columns each (one key row per thread; then the dK and dV
+// epilogues), 12-15 dQ writers (one head-dim lane per thread).  setmaxnreg moves registers from the producer/MMA and dQ
 // warpgroups to the softmax warpgroups: 128*64 + 256*176 + 128*96 = 65536 = 512*128.
-// P^T and dS^T become visible to the second MMA thread together (one barrier
+// P^T and dS^T become visible to the second MMA warp together (one barrier
 // per tile).  TMEM: S^T[2] at 0/64, dP^T[2] at 128/192 (P^T, dS^T written over them as
-// packed bf16), dV at 256, dK at 256 + D; dQ^T of buffer i is written over
+// packed bf16, each column half inside the columns it was computed from), dV at 256, dK at 256 + D; dQ^T of buffer i is written over
 // dP^T[i] after the dK MMA that read dS^T from there (MMAs run in issue
 // order), so the next S^T never waits for the dQ writers.
 #include <cuda.h>
@@ -83,13 +83,27 @@ __device__ __forceinline__ void issue_kq(uint32_t d, uint64_t adesc, uint64_t bd
   mma_chain_ss_w<D / 16>(d, adesc, sa.v, bdesc, sb.v, idesc, 0u);
 }
 
-// dV += P^T dO or dK += dS^T Qr: A from TMEM (128 keys x 64 q, packed bf16),
-// B = 64-row tile read MN-major (N = D contiguous, D blocks 8 KB apart).
+// dV += P^T dO or dK += dS^T Qr: A from TMEM (128 keys x 64 q, packed bf16:
+// query rows 0-31 in columns [0, 16) of the buffer, rows 32-63 in [48, 64),
+// each half where the softmax warpgroup of that half wrote it), B = 64-row
+// tile read MN-major (N = D contiguous, D blocks 8 KB apart).
 template <int D>
 __device__ __forceinline__ void issue_acc(uint32_t d, uint32_t a_tmem, uint64_t bdesc, bool acc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
   constexpr MNMajorSteps<BQ / 16> st;
-  mma_chain_ts_w<BQ / 16>(d, a_tmem, 8u, bdesc, st.v, idesc, acc ? 1u : 0u);
+  constexpr uint32_t aoff[4] = {0u, 8u, 48u, 56u};
+  uint64_t bd[4];
+  uint32_t ad[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    bd[i] = bdesc + st.v[i];
+    ad[i] = a_tmem + aoff[i];
+  }
+  if (elect_one()) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mma_ts(d, ad[i], bd[i], idesc, i == 0 ? (acc ? 1u : 0u) : 1u);
+  }
+  __syncwarp();
 }
 
 // dQ^T = Kr^T dS^T: M = 128 (head dims; for D = 64 the second 64-row block
@@ -134,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.bar_s_full[i], 1);
       mbar_init(&sm.bar_dp_full[i], 1);
-      mbar_init(&sm.bar_ds_ready[i], 4);   // one arrival per softmax warp
+      mbar_init(&sm.bar_ds_ready[i], 8);   // one arrival per softmax warp (both warpgroups)
       mbar_init(&sm.bar_dq_full[i], 1);
       mbar_init(&sm.bar_dq_empty[i], 4);   // one arrival per dQ warp
       mbar_init(&sm.bar_s_free[i], 1);
@@ -254,7 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 12) {
     regs_inc<176>();
     // =============================== softmax: one key row per thread
-    const int bf = (warp - 4) >> 2;  // this warpgroup's TMEM / dS buffer and iteration parity
+    // Both warpgroups work on every query tile, each on one half of its 64
+    // query columns (hq = 0: rows 0-31, hq = 1: rows 32-63), so a tile's P^T
+    // and dS^T are ready in half the time.  Each half writes its packed bf16
+    // P^T / dS^T inside the TMEM columns it has just read (columns [0, 16) or
+    // [48, 64) of the buffer), never over the other half's scores.
+    const int bf = (warp - 4) >> 2;  // warpgroup: query-column half here, dK / dV in the epilogue
+    const int hq = bf;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int key = kt * BK + r;
@@ -265,23 +285,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const float cs = p.scale_log2;
     bool ok = true;
-    for (int i = bf; i < n_it; i += 2) {
-      const int s = i % kStages;
+    for (int i = 0; i < n_it; ++i) {
+      const int b = i & 1, s = i % kStages;
       const int qt = qt_first + i % n_qt;
       const bool partial = qt < full_first || qt >= full_end || (qt + 1) * BQ > smp.rows;
       // the stage's lse2/delta were written by TMA: acquire them through its barrier
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_full[s], (i / kStages) & 1, wc) &&
-                                       mbar_wait(&sm.bar_s_full[bf], (i >> 1) & 1, wc));
+                                       mbar_wait(&sm.bar_s_full[b], (i >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(tS(bf) + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tS(bf) + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      uint32_t sr[32];
+      tmem_ld32(tS(b) + lane_off + uint32_t(hq * 32), sr);
       tmem_ld_wait_regs(sr);
-      float pv[64];
-      const float4* l2 = reinterpret_cast<const float4*>(sm.lse2[s]);
+      float pv[32];
+      const float4* l2 = reinterpret_cast<const float4*>(sm.lse2[s]) + hq * 8;
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
+      for (int c4 = 0; c4 < 8; ++c4) {
         const float4 l = l2[c4];
         // scale and subtract as packed f32x2 (two columns per instruction)
         const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[4 * c4 + 0]), __uint_as_float(sr[4 * c4 + 1])),
@@ -294,44 +313,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         pv[4 * c4 + 3] = ex2_approx(xb.y);
       }
       if (partial) {
-        const int q0 = qt * BQ;
+        const int q0 = qt * BQ + hq * 32;
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < 32; ++c)
           if (q0 + c < vis_lo || q0 + c >= vis_hi) pv[c] = 0.f;
       }
       __syncwarp();  // converged before the warp-collective TMEM store
-      uint32_t pk[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
-      tmem_st32(tS(bf) + lane_off, pk);
+      for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+      tmem_st16(tS(b) + lane_off + uint32_t(hq * 48), pk);
 
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_dp_full[bf], (i >> 1) & 1, wc));
+      ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar_dp_full[b], (i >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after();
-      tmem_ld32(tdP(bf) + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tdP(bf) + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tdP(b) + lane_off + uint32_t(hq * 32), sr);
       tmem_ld_wait_regs(sr);
-      const float4* dl = reinterpret_cast<const float4*>(sm.delta[s]);
+      const float4* dl = reinterpret_cast<const float4*>(sm.delta[s]) + hq * 8;
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
+      for (int c4 = 0; c4 < 8; ++c4) {
         const float4 d = dl[c4];
         pk[2 * c4] = pack_bf16x2(pv[4 * c4 + 0] * (__uint_as_float(sr[4 * c4 + 0]) - d.x),
                                  pv[4 * c4 + 1] * (__uint_as_float(sr[4 * c4 + 1]) - d.y));
         pk[2 * c4 + 1] = pack_bf16x2(pv[4 * c4 + 2] * (__uint_as_float(sr[4 * c4 + 2]) - d.z),
                                      pv[4 * c4 + 3] * (__uint_as_float(sr[4 * c4 + 3]) - d.w));
       }
-      tmem_st32(tdP(bf) + lane_off, pk);
-      // dS^T row -> shared memory, 128-byte swizzled rows of 64 query values
-      uint8_t* dsrow = reinterpret_cast<uint8_t*>(sm.ds[bf]);
+      tmem_st16(tdP(b) + lane_off + uint32_t(hq * 48), pk);
+      // dS^T row half -> shared memory: 16-byte chunks hq*4 .. hq*4+3 of the
+      // 128-byte swizzled row of 64 query values
+      uint8_t* dsrow = reinterpret_cast<uint8_t*>(sm.ds[b]);
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(dsrow + sw128_offset(uint32_t(r), uint32_t(c))) =
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(dsrow + sw128_offset(uint32_t(r), uint32_t(hq * 4 + c))) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();  // the warp's TMEM and shared-memory writes are done; one lane signals for it
-      if (lane == 0) mbar_arrive(&sm.bar_ds_ready[bf]);
+      if (lane == 0) mbar_arrive(&sm.bar_ds_ready[b]);
     }
     // ---- epilogue: warpgroup 0 writes dK = R^T (scale dKr), warpgroup 1 dV
     bool have = n_it > 0 && ok;
