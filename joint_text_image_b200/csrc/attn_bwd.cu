@@ -46,6 +46,7 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kLaunchRegs = 128;  // the setmaxnreg split below assumes 512 x 128 at launch
 constexpr int kStages = 3;
+constexpr int kFmaExpPairs = 4;  // of every 16 column pairs of P^T, this many use exp2_fma2
 constexpr int BK = kBwdBK;  // 128 keys
 constexpr int BQ = kBwdBQ;  // 64 query rows
 
@@ -91,6 +92,7 @@ template <int D>
 __device__ __forceinline__ void issue_acc(uint32_t d, uint32_t a_tmem, uint64_t bdesc, bool acc) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
   constexpr MNMajorSteps<BQ / 16> st;
+  static_assert(BQ == 64, "two 32-row query halves of two 16-row K-steps each");
   constexpr uint32_t aoff[4] = {0u, 8u, 48u, 56u};
   uint64_t bd[4];
   uint32_t ad[4];
@@ -307,10 +309,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      make_float2(cs, cs), make_float2(-l.x, -l.y));
         const float2 xb = __ffma2_rn(make_float2(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
                                      make_float2(cs, cs), make_float2(-l.z, -l.w));
-        pv[4 * c4 + 0] = ex2_approx(xa.x);
-        pv[4 * c4 + 1] = ex2_approx(xa.y);
-        pv[4 * c4 + 2] = ex2_approx(xb.x);
-        pv[4 * c4 + 3] = ex2_approx(xb.y);
+        // kFmaExpPairs of every 16 column pairs take exp2 on the FMA pipe (both
+        // warpgroups share the MUFU unit on the same tile); masked columns are
+        // zeroed below, whatever the emulation returned for them
+        const float2 pa = ((2 * c4) % 16 < kFmaExpPairs) ? exp2_fma2(xa)
+                                                         : make_float2(ex2_approx(xa.x), ex2_approx(xa.y));
+        const float2 pb = ((2 * c4 + 1) % 16 < kFmaExpPairs) ? exp2_fma2(xb)
+                                                             : make_float2(ex2_approx(xb.x), ex2_approx(xb.y));
+        pv[4 * c4 + 0] = pa.x;
+        pv[4 * c4 + 1] = pa.y;
+        pv[4 * c4 + 2] = pb.x;
+        pv[4 * c4 + 3] = pb.y;
       }
       if (partial) {
         const int q0 = qt * BQ + hq * 32;
