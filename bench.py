@@ -51,6 +51,16 @@ def peaks():
         return PEAKS_FALLBACK, "fallback"
 
 
+def bwd_schedule_desc(seg, wl):
+    """The backward schedule the launches take on this device: how many kv
+    tiles are cut into how many parts."""
+    import torch
+    n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    parts, ent = seg.bwd_schedules()[seg.bwd_choice(wl.Hkv, wl.Hq // wl.Hkv, n_sm)]
+    return {"parts": parts, "split_kv_tiles": int((ent[:, 4] >= 0).sum()) // parts if parts > 1 else 0,
+            "ctas": int(len(ent)) * wl.Hkv}
+
+
 def workload_desc(wl):
     if wl.name != "1024px":
         return (f"{wl.name} fwd+bwd: samples (prefix, h, w, suffix) {wl.samples}, S={wl.S}; Hq={wl.Hq}, "
@@ -411,8 +421,10 @@ def main():
                     help="synthetic workload (the metric is quoted on 1024px; the others are for profiling)")
     ap.add_argument("--packed", action="store_true",
                     help="packed (varlen) layout: no padded rows (no e2e line: the host step is padded-only)")
-    ap.add_argument("--bwd-split", choices=["auto", "never", "always"], default="auto",
-                    help="backward schedule: split the longest kv tiles in two (hia_segments_set_bwd_split)")
+    ap.add_argument("--bwd-split", choices=["auto", "never", "always", "parts2", "parts3", "parts4"],
+                    default="auto",
+                    help="backward schedule: cut the longest kv tiles' query ranges into parts "
+                         "(hia_segments_set_bwd_split)")
     ap.add_argument("--qk-norm", action="store_true",
                     help="enable the per-head QK RMSNorm after RoPE (weights seeded, eps 1e-5)")
     ap.add_argument("--source-hash", choices=sorted(KERNEL_SOURCES),
@@ -459,7 +471,7 @@ def main():
         q, k, v, do = (packf(t) for t in (q, k, v, do))
     else:
         seg = jt.hia_segments_build(wl.samples, wl.S)
-    seg.set_bwd_split({"auto": 0, "never": 1, "always": 2}[args.bwd_split])
+    seg.set_bwd_split({"auto": 0, "never": 1, "always": 2, "parts2": 3, "parts3": 4, "parts4": 5}[args.bwd_split])
     info = seg.info()
     pairs = info.visible_pairs
     fwd_flops = 4.0 * wl.D * wl.Hq * pairs
@@ -608,7 +620,8 @@ def main():
                        "l2": f"inputs larger than L2: {(q.numel() + k.numel() + v.numel() + do.numel()) * 2 / 1e6:.0f} MB read per step",
                        "visible_pairs": pairs, "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
                        "qk_norm": ({"eps": 1e-5, "weights": "seeded U[0.5,1.5)"} if args.qk_norm else None),
-                       "layout": f"packed ({seg.total_rows} rows)" if args.packed else "padded"},
+                       "layout": f"packed ({seg.total_rows} rows)" if args.packed else "padded",
+                       "bwd_schedule": bwd_schedule_desc(seg, wl)},
             "pct_of_bf16_peak": value / world / peak_burst * 100.0,
             "fwd_tflops": fwd_flops / (fwd_t * 1e-3) / 1e12 if fwd_t else None,
             "bwd_tflops": bwd_flops / (bwd_t * 1e-3) / 1e12 if bwd_t else None,

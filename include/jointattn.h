@@ -98,7 +98,7 @@ typedef struct {
     int32_t bwd_q_tiles;         /* ceil(S / 64) */
     int32_t bwd_kv_tiles;        /* ceil(S / 128) */
     int32_t packed;              /* 1: built by hia_segments_build_packed */
-    int32_t bwd_split_units;     /* kv tiles whose backward work can be split in two (see hia_segments_set_bwd_split) */
+    int32_t bwd_split_units;     /* kv tiles a split schedule can cut into parts (see hia_segments_set_bwd_split) */
     int64_t total_rows;          /* rows of a tensor in this layout: B*S, or the sum of L when packed */
 } hia_segments_info_t;
 
@@ -165,19 +165,49 @@ int hia_segments_info(const hia_segments* seg, hia_segments_info_t* info);
 /* Scheduling of the backward (a property of the library, not of the method:
  * the result is the same either way, and deterministic).  One CTA of the
  * backward handles one (sample, kv head, 128-key tile) over every query tile
- * that sees it, so a few CTAs (keys seen by every later row) are far longer
- * than the rest and can leave SMs idle at the end.  The descriptor also holds
- * a second schedule in which those longest kv tiles (query range within 10%
- * of the longest) are split into two halves, each writing an fp32 partial of
- * dK and dV; the half that finishes second adds the two in a fixed order.
- *   HIA_BWD_SPLIT_AUTO (default): each backward launch picks the schedule a
+ * that sees it, so CTAs differ in length by up to the whole query range and
+ * the last ones can leave SMs idle at the end.  Besides that whole schedule,
+ * the descriptor holds split schedules: for parts k in {2, 3, 4} and a
+ * threshold of 95, 90 or 85% of the longest query range, every kv tile at or
+ * above the threshold is cut into k consecutive query sub-ranges (of at least
+ * two 64-row tiles each), each run by its own CTA that writes fp32 partials
+ * of dK and dV; the part that finishes last adds the k partials in part
+ * order (bitwise the same whichever part is last) and writes dK and dV.
+ *   HIA_BWD_SPLIT_AUTO (default): each backward launch takes the schedule a
  *     list-scheduling estimate (heaviest first, on the device's SM count, for
- *     its number of kv heads) finishes sooner; it splits for one long sample,
- *     not for batches where the balance is already good.
- *   HIA_BWD_SPLIT_NEVER / HIA_BWD_SPLIT_ALWAYS: force one schedule.
+ *     its number of kv heads and g) finishes soonest.
+ *   HIA_BWD_SPLIT_NEVER: the whole schedule.
+ *   HIA_BWD_SPLIT_ALWAYS: the estimate's best split schedule.
+ *   HIA_BWD_SPLIT_PARTS_2 / _3 / _4: the estimate's best schedule cutting
+ *     tiles into exactly 2 / 3 / 4 parts.
+ * A mode that admits no schedule of the descriptor (nothing long enough to
+ * split) runs the whole one.  The choice is made per (mode, kv heads, g, SM
+ * count); hia_attn_bwd_workspace_bytes sizes the partials for the choice on
+ * the current device, and a workspace too small for a later choice (another
+ * device, or the mode changed after sizing) runs the whole schedule.
  * Errors: HIA_ERR_INVALID_ARG (null, unknown mode). */
-enum { HIA_BWD_SPLIT_AUTO = 0, HIA_BWD_SPLIT_NEVER = 1, HIA_BWD_SPLIT_ALWAYS = 2 };
+enum {
+  HIA_BWD_SPLIT_AUTO = 0,
+  HIA_BWD_SPLIT_NEVER = 1,
+  HIA_BWD_SPLIT_ALWAYS = 2,
+  HIA_BWD_SPLIT_PARTS_2 = 3,
+  HIA_BWD_SPLIT_PARTS_3 = 4,
+  HIA_BWD_SPLIT_PARTS_4 = 5
+};
 int hia_segments_set_bwd_split(hia_segments* seg, int mode);
+
+/* Inspection of the backward schedules (host only, no CUDA call).
+ * hia_segments_bwd_schedule: schedule `index` (0 = the whole one; the
+ * others in order of parts, then of decreasing threshold): *parts (1 for the
+ * whole schedule), *n_entries, and, if entries is not NULL, its work list,
+ * int32 [n_entries][8] = (b, kv tile, first query tile, end query tile,
+ * slot (-1 unless split), part, parts, 0), in launch order (one CTA per
+ * entry and kv head).  HIA_ERR_INVALID_ARG past the last schedule.
+ * hia_segments_bwd_choice: the schedule index a launch with Hkv kv heads, g
+ * query heads per kv head and n_sm SMs takes under the current mode. */
+int hia_segments_bwd_schedule(const hia_segments* seg, int index, int32_t* parts, int64_t* n_entries,
+                              int32_t* entries);
+int hia_segments_bwd_choice(const hia_segments* seg, int Hkv, int g, int n_sm, int* index);
 
 /* Host copies for tests and inspection.  row_bound: int32 [B, S] e_b(q)
  * (-1 for a sample with L = 0).  mask: uint8 [B, S, S] (1 = visible) rendered
@@ -201,7 +231,9 @@ int hia_segments_tile_classes(const hia_segments* seg, uint8_t* classes);
  * sin block layout of the [B, S, head_dim] tables taken by
  * HunyuanImage3Attention.forward).  Angles and cos/sin are evaluated in fp64
  * and rounded once to fp32, so a text-only sample gives exactly the 1D RoPE
- * tables.  D even, 2 <= D <= 256, base > 0. */
+ * tables.  D even, 2 <= D <= 256, base > 0.  Errors: HIA_ERR_INVALID_ARG
+ * (null seg or buffers, D or base out of range), HIA_ERR_UNSUPPORTED
+ * (B * S >= 2^31 table rows), HIA_ERR_NOT_ON_DEVICE, HIA_ERR_CUDA. */
 int hia_rope2d_tables(const hia_segments* seg, int D, double base, float* cos_out,
                       float* sin_out, void* stream);
 
@@ -282,7 +314,9 @@ int hia_attn_fwd_noalloc(const hia_segments* seg, int Hq, int Hkv, int D, hia_te
                          hia_tensor o, float* lse, void* stream);
 
 /* Bytes of device workspace hia_attn_bwd and hia_attn_bwd_ex need (the
- * size covers the QK RMSNorm's extra accumulators either way). */
+ * size covers the QK RMSNorm's extra accumulators either way, and the fp32
+ * partials of the backward schedule chosen for the current device and the
+ * descriptor's mode: see hia_segments_set_bwd_split). */
 size_t hia_attn_bwd_workspace_bytes(const hia_segments* seg, int Hq, int Hkv, int D);
 
 /* Recompute backward of hia_attn_fwd: given o and lse from the forward and

@@ -31,7 +31,8 @@ EXPORTED_SYMBOLS = (
     "hia_profile_end", "hia_attn_fwd_noalloc", "hia_debug_exp2", "hia_step_create", "hia_step_destroy",
     "hia_attn_step_host", "hia_attn_fwd_ex", "hia_attn_bwd_ex", "hia_segments_build_packed",
     "hia_segments_layout", "hia_segments_build_multi", "hia_attn_bwd_reuse_fwd",
-    "hia_moe_workspace_bytes", "hia_moe_fwd", "hia_segments_set_bwd_split",
+    "hia_moe_workspace_bytes", "hia_moe_fwd", "hia_segments_set_bwd_split", "hia_segments_bwd_schedule",
+    "hia_segments_bwd_choice",
 )
 
 
@@ -97,6 +98,8 @@ def lib():
         L.hia_segments_destroy.restype = None
         L.hia_segments_info.argtypes = [P, ctypes.POINTER(SegmentsInfo)]
         L.hia_segments_set_bwd_split.argtypes = [P, I]
+        L.hia_segments_bwd_schedule.argtypes = [P, I, P, P, P]
+        L.hia_segments_bwd_choice.argtypes = [P, I, I, I, P]
         L.hia_segments_row_bound.argtypes = [P, P]
         L.hia_segments_layout.argtypes = [P, P, P]
         L.hia_segments_mask.argtypes = [P, P]
@@ -215,10 +218,35 @@ class Segments:
         return e
 
     def set_bwd_split(self, mode):
-        """Backward schedule: 0 auto (default), 1 never split, 2 always split
-        the longest kv tiles (hia_segments_set_bwd_split)."""
+        """Backward schedule (hia_segments_set_bwd_split): 0 auto (default),
+        1 never split, 2 the best split schedule, 3 / 4 / 5 the best one
+        cutting the longest kv tiles into exactly 2 / 3 / 4 parts."""
         _check(lib().hia_segments_set_bwd_split(self.handle, int(mode)), "hia_segments_set_bwd_split")
         return self
+
+    def bwd_schedules(self):
+        """Every backward schedule of the descriptor as (parts, entries):
+        entries int32 [n, 8] = (b, kv tile, first query tile, end query tile,
+        slot, part, parts, 0) in launch order (hia_segments_bwd_schedule)."""
+        import numpy as np
+        out = []
+        while True:
+            parts, n = ctypes.c_int32(0), ctypes.c_int64(0)
+            rc = lib().hia_segments_bwd_schedule(self.handle, len(out), ctypes.byref(parts), ctypes.byref(n), None)
+            if rc != 0:
+                return out
+            e = np.zeros((max(n.value, 1), 8), dtype=np.int32)
+            _check(lib().hia_segments_bwd_schedule(self.handle, len(out), ctypes.byref(parts), ctypes.byref(n),
+                                                   e.ctypes.data_as(ctypes.c_void_p)), "hia_segments_bwd_schedule")
+            out.append((parts.value, e[:n.value]))
+
+    def bwd_choice(self, Hkv, g, n_sm):
+        """Index into bwd_schedules() of the schedule a backward launch takes
+        (hia_segments_bwd_choice)."""
+        i = ctypes.c_int(0)
+        _check(lib().hia_segments_bwd_choice(self.handle, int(Hkv), int(g), int(n_sm), ctypes.byref(i)),
+               "hia_segments_bwd_choice")
+        return i.value
 
     def mask(self):
         import numpy as np

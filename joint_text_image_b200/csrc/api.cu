@@ -192,7 +192,8 @@ struct BwdWs {
 };
 // The dK accumulator and the weight-gradient partials are used only with the
 // QK RMSNorm; the size always includes them so one workspace serves both.
-BwdWs bwd_ws(const hia_segments* seg, int Hq, int Hkv, int D) {
+// The partials of split kv tiles are sized for the schedule `sc`.
+BwdWs bwd_ws(const hia_segments* seg, int Hq, int Hkv, int D, const hia_segments::BwdSched& sc) {
   BwdWs w{};
   const size_t BS = size_t(seg->B) * seg->S;
   const size_t BSp = size_t(seg->B) * S_pad64(seg->S);
@@ -204,26 +205,34 @@ BwdWs bwd_ws(const hia_segments* seg, int Hq, int Hkv, int D) {
   w.dk_off = w.dq_off + align256(BSp * Hq * D * 4);
   w.dw_off = w.dk_off + align256(BSp * Hkv * D * 4);
   w.part_off = w.dw_off + align256(size_t(2) * hia::grad_finalize_blocks(seg->B, seg->S) * D * 4);
-  // split schedule: per (slot, kv head) two halves' fp32 dK and dV partials, and a ticket counter
-  w.cnt_off = w.part_off + align256(size_t(seg->n_split_slots) * Hkv * 2 * 2 * hia::kBwdBK * D * 4);
-  w.total = w.cnt_off + align256(size_t(seg->n_split_slots) * Hkv * 4);
+  // split kv tiles: per (slot, kv head) every part's fp32 dK and dV partials, and a ticket counter
+  w.cnt_off = w.part_off + align256(size_t(sc.n_slots) * Hkv * sc.parts * 2 * hia::kBwdBK * D * 4);
+  w.total = w.cnt_off + align256(size_t(sc.n_slots) * Hkv * 4);
   return w;
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? HIA_OK : HIA_ERR_CUDA; }
 
 // Finish time of a backward work list dispatched in order to the first free
-// SM (the block scheduler's policy), one CTA per (entry, kv head): a CTA
-// costs its query tiles times g plus a fixed part (K/V load, epilogue; about
-// four tile iterations), and a split half two more (its partial's write and
-// the combine).
+// SM (the block scheduler's policy), one CTA per (entry, kv head), in units of
+// one query-tile iteration of a whole kv tile.  A CTA costs its query tiles
+// times g plus a fixed part (K/V load, TMEM setup, dK/dV epilogue: about nine
+// iterations); a part of a split kv tile runs its iterations 20% slower and
+// the last part (the one that usually adds the partials) costs 22.5 more.  The
+// constants are fitted to per-CTA timings (globaltimer stamps) and backward
+// times of the 1024px, 1024px_bwd, mixed and multi_image workloads under every
+// schedule: the estimate's pick was within 1% of the fastest measured one on
+// each.
 double bwd_makespan(const std::vector<int32_t>& work, int Hkv, int g, int n_sm) {
-  constexpr double kCtaCost = 4.0, kSplitCost = 2.0;
+  constexpr double kCtaCost = 9.0, kPartSlowdown = 1.2, kMergeCost = 22.5;
   std::priority_queue<double, std::vector<double>, std::greater<double>> sms;
   for (int i = 0; i < n_sm; ++i) sms.push(0.0);
   double span = 0.0;
   for (size_t e = 0; e + hia::kBwdWorkInts <= work.size(); e += hia::kBwdWorkInts) {
-    const double c = double(work[e + 3] - work[e + 2]) * g + kCtaCost + (work[e + 4] >= 0 ? kSplitCost : 0.0);
+    const double it = double(work[e + 3] - work[e + 2]) * g;
+    const bool split = work[e + 4] >= 0;
+    const double c = split ? it * kPartSlowdown + kCtaCost + (work[e + 5] == work[e + 6] - 1 ? kMergeCost : 0.0)
+                           : it + kCtaCost;
     for (int h = 0; h < Hkv; ++h) {
       const double t = sms.top() + c;
       sms.pop();
@@ -246,18 +255,33 @@ int device_sm_count() {
   return n;
 }
 
-// Whether a backward launch uses the split work list.
-bool use_bwd_split(hia_segments* g, int Hkv, int gq) {
-  if (g->n_split_slots == 0 || g->bwd_split_mode == HIA_BWD_SPLIT_NEVER) return false;
-  if (g->bwd_split_mode == HIA_BWD_SPLIT_ALWAYS) return true;
-  const int n_sm = device_sm_count();
+// The backward schedule a launch uses (an index into bwd_sched): the one the
+// estimate finishes soonest among those the mode admits (all of them for
+// AUTO, the split ones for ALWAYS, those cutting tiles into k parts for
+// PARTS_k), the whole list for NEVER or when the mode admits none.
+int choose_bwd_sched(const hia_segments* gc, int Hkv, int gq, int n_sm) {
+  hia_segments* g = const_cast<hia_segments*>(gc);
   std::lock_guard<std::mutex> lk(g->choice_mu);
-  const auto key = std::make_tuple(Hkv, gq, n_sm);
+  const int mode = g->bwd_split_mode;
+  if (mode == HIA_BWD_SPLIT_NEVER || g->bwd_sched.size() <= 1) return 0;
+  const auto key = std::make_tuple(mode, Hkv, gq, n_sm);
   auto it = g->choice.find(key);
   if (it != g->choice.end()) return it->second;
-  const bool split = bwd_makespan(g->bwd_work_split, Hkv, gq, n_sm) < bwd_makespan(g->bwd_work, Hkv, gq, n_sm);
-  g->choice[key] = split;
-  return split;
+  int best = 0;  // the whole list when the mode admits none
+  double best_span = -1.0;
+  for (int i = 0; i < int(g->bwd_sched.size()); ++i) {
+    const int parts = g->bwd_sched[i].parts;
+    const bool admitted = mode == HIA_BWD_SPLIT_AUTO || (mode == HIA_BWD_SPLIT_ALWAYS && parts > 1) ||
+                          (mode >= HIA_BWD_SPLIT_PARTS_2 && parts == mode - HIA_BWD_SPLIT_PARTS_2 + 2);
+    if (!admitted) continue;
+    const double span = bwd_makespan(g->bwd_sched[i].work, Hkv, gq, n_sm);
+    if (best_span < 0.0 || span < best_span) {  // ties: the earlier (less split) schedule
+      best = i;
+      best_span = span;
+    }
+  }
+  g->choice[key] = best;
+  return best;
 }
 
 int check_norm(const hia_qk_norm* n) {
@@ -308,6 +332,7 @@ void packed_view(const hia_segments* g, std::initializer_list<hia_tensor*> ts) {
 int map_rows(const hia_segments* g) { return g->packed ? int(g->total_rows) : g->S; }
 int map_batches(const hia_segments* g) { return g->packed ? 1 : g->B; }
 
+
 }  // namespace
 
 extern "C" int hia_segments_upload(hia_segments* g, void* stream) {
@@ -318,10 +343,16 @@ extern "C" int hia_segments_upload(hia_segments* g, void* stream) {
   if (g->dbuf && g->device != dev) return HIA_ERR_INVALID_ARG;
   const size_t n_s = g->samples.size() * sizeof(SampleDev), n_i = g->images.size() * sizeof(hia::ImageDev);
   const size_t n_ft = g->fwd_tiles.size() * 4, n_fl = g->fwd_list.size() * 4, n_fw = g->fwd_work.size() * 4;
-  const size_t n_bt = g->bwd_tiles.size() * 4, n_bw = g->bwd_work.size() * 4, n_bs = g->bwd_work_split.size() * 4;
+  const size_t n_bt = g->bwd_tiles.size() * 4;
   const size_t o_s = 0, o_i = align256(n_s), o_ft = o_i + align256(n_i), o_fl = o_ft + align256(n_ft),
-               o_fw = o_fl + align256(n_fl), o_bt = o_fw + align256(n_fw), o_bw = o_bt + align256(n_bt),
-               o_bs = o_bw + align256(n_bw), total = o_bs + align256(n_bs) + 256;
+               o_fw = o_fl + align256(n_fl), o_bt = o_fw + align256(n_fw), o_bw = o_bt + align256(n_bt);
+  std::vector<size_t> o_sched(g->bwd_sched.size());
+  size_t total = o_bw;
+  for (size_t i = 0; i < g->bwd_sched.size(); ++i) {
+    o_sched[i] = total;
+    total += align256(g->bwd_sched[i].work.size() * 4);
+  }
+  total += 256;
   if (!g->dbuf) {
     if (cudaMalloc(&g->dbuf, total) != cudaSuccess) {
       g->dbuf = nullptr;
@@ -336,9 +367,11 @@ extern "C" int hia_segments_upload(hia_segments* g, void* stream) {
   if (e == cudaSuccess && n_fl) e = cudaMemcpyAsync(base + o_fl, g->fwd_list.data(), n_fl, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess && n_fw) e = cudaMemcpyAsync(base + o_fw, g->fwd_work.data(), n_fw, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess && n_bt) e = cudaMemcpyAsync(base + o_bt, g->bwd_tiles.data(), n_bt, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess && n_bw) e = cudaMemcpyAsync(base + o_bw, g->bwd_work.data(), n_bw, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess && n_bs)
-    e = cudaMemcpyAsync(base + o_bs, g->bwd_work_split.data(), n_bs, cudaMemcpyHostToDevice, st);
+  for (size_t i = 0; i < g->bwd_sched.size(); ++i) {
+    const std::vector<int32_t>& w = g->bwd_sched[i].work;
+    if (e == cudaSuccess && !w.empty())
+      e = cudaMemcpyAsync(base + o_sched[i], w.data(), w.size() * 4, cudaMemcpyHostToDevice, st);
+  }
   if (e != cudaSuccess) return HIA_ERR_CUDA;
   g->device = dev;
   g->d_samples = reinterpret_cast<const SampleDev*>(base + o_s);
@@ -347,8 +380,8 @@ extern "C" int hia_segments_upload(hia_segments* g, void* stream) {
   g->d_fwd_list = reinterpret_cast<const int32_t*>(base + o_fl);
   g->d_fwd_work = reinterpret_cast<const int32_t*>(base + o_fw);
   g->d_bwd_tiles = reinterpret_cast<const int32_t*>(base + o_bt);
-  g->d_bwd_work = reinterpret_cast<const int32_t*>(base + o_bw);
-  g->d_bwd_work_split = reinterpret_cast<const int32_t*>(base + o_bs);
+  for (size_t i = 0; i < g->bwd_sched.size(); ++i)
+    g->bwd_sched[i].d_work = reinterpret_cast<const int32_t*>(base + o_sched[i]);
   return HIA_OK;
 }
 
@@ -364,8 +397,14 @@ extern "C" void hia_segments_destroy(hia_segments* g) {
   delete g;
 }
 
+extern "C" int hia_segments_bwd_choice(const hia_segments* g, int Hkv, int gq, int n_sm, int* index) {
+  if (!g || Hkv <= 0 || gq <= 0 || n_sm <= 0 || !index) return HIA_ERR_INVALID_ARG;
+  *index = choose_bwd_sched(g, Hkv, gq, n_sm);
+  return HIA_OK;
+}
+
 extern "C" int hia_segments_set_bwd_split(hia_segments* g, int mode) {
-  if (!g || mode < HIA_BWD_SPLIT_AUTO || mode > HIA_BWD_SPLIT_ALWAYS) return HIA_ERR_INVALID_ARG;
+  if (!g || mode < HIA_BWD_SPLIT_AUTO || mode > HIA_BWD_SPLIT_PARTS_4) return HIA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lk(g->choice_mu);
   g->bwd_split_mode = mode;
   return HIA_OK;
@@ -375,6 +414,7 @@ extern "C" int hia_rope2d_tables(const hia_segments* g, int D, double base, floa
   if (!g || D < 2 || D > 256 || (D & 1) || !(base > 0.0) || !std::isfinite(base)) return HIA_ERR_INVALID_ARG;
   if (g->B == 0 || g->S == 0) return HIA_OK;
   if (!c || !s) return HIA_ERR_INVALID_ARG;
+  if (int64_t(g->B) * g->S >= (int64_t(1) << 31)) return HIA_ERR_UNSUPPORTED;  // one warp per row: grid size
   if (g->device < 0) return HIA_ERR_NOT_ON_DEVICE;
   hia::launch_rope2d_tables(g->d_samples, g->d_images, g->B, g->S, D, base, c, s, static_cast<cudaStream_t>(stream));
   return cuda_status(cudaGetLastError());
@@ -387,7 +427,8 @@ extern "C" size_t hia_attn_fwd_workspace_bytes(const hia_segments* g, int Hq, in
 
 extern "C" size_t hia_attn_bwd_workspace_bytes(const hia_segments* g, int Hq, int Hkv, int D) {
   if (!g || Hq <= 0 || Hkv <= 0 || D <= 0) return 0;
-  return bwd_ws(g, Hq, Hkv, D).total;
+  const int si = choose_bwd_sched(g, Hkv, std::max(1, Hq / Hkv), device_sm_count());
+  return bwd_ws(g, Hq, Hkv, D, g->bwd_sched[si]).total;
 }
 
 extern "C" int hia_attn_fwd(const hia_segments* g, int Hq, int Hkv, int D, hia_tensor q, hia_tensor k,
@@ -535,7 +576,13 @@ extern "C" int hia_attn_bwd_reuse_fwd(const hia_segments* g, int Hq, int Hkv, in
   if (!q.ptr || !k.ptr || !v.ptr || !o.ptr || !lse || !dout.ptr || !dq.ptr || !dk.ptr || !dv.ptr || !ws)
     return HIA_ERR_INVALID_ARG;
   packed_view(g, {&q, &k, &v, &o, &dout, &dq, &dk, &dv});
-  const BwdWs w = bwd_ws(g, Hq, Hkv, D);
+  // the schedule; a workspace sized for another choice (another device's SM
+  // count, or before the mode changed) that does not hold its partials runs
+  // the whole list, which needs none
+  int si = choose_bwd_sched(g, Hkv, gq, device_sm_count());
+  if (ws_bytes < bwd_ws(g, Hq, Hkv, D, g->bwd_sched[si]).total) si = 0;
+  const hia_segments::BwdSched& sched = g->bwd_sched[si];
+  const BwdWs w = bwd_ws(g, Hq, Hkv, D, sched);
   if (ws_bytes < w.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return HIA_ERR_INVALID_ARG;
   const FwdWs fw = fwd_ws(g, Hq, Hkv, D);
   if (fws && (fws_bytes < fw.total || (reinterpret_cast<uintptr_t>(fws) & 255)))
@@ -556,7 +603,6 @@ extern "C" int hia_attn_bwd_reuse_fwd(const hia_segments* g, int Hq, int Hkv, in
   float* dw_part = reinterpret_cast<float*>(wb + w.dw_off);
   float* part = reinterpret_cast<float*>(wb + w.part_off);
   int* part_cnt = reinterpret_cast<int*>(wb + w.cnt_off);
-  const bool split = use_bwd_split(const_cast<hia_segments*>(g), Hkv, gq);
   const int S_pad = S_pad64(g->S);
 
   CUtensorMap tq, tk, tv, tdo;
@@ -586,7 +632,7 @@ extern "C" int hia_attn_bwd_reuse_fwd(const hia_segments* g, int Hq, int Hkv, in
   pp.delta = delta;
   pp.dq_acc = dq_acc;
   pp.part_cnt = part_cnt;
-  pp.n_cnt = g->n_split_slots * Hkv;
+  pp.n_cnt = sched.n_slots * Hkv;
   pp.B = g->B;
   pp.S = g->S;
   pp.S_pad = S_pad;
@@ -599,7 +645,7 @@ extern "C" int hia_attn_bwd_reuse_fwd(const hia_segments* g, int Hq, int Hkv, in
   p.samples = g->d_samples;
   p.images = g->d_images;
   p.tiles = g->d_bwd_tiles;
-  p.work = split ? g->d_bwd_work_split : g->d_bwd_work;
+  p.work = sched.d_work;
   p.part = part;
   p.part_cnt = part_cnt;
   p.B = g->B;
@@ -629,7 +675,7 @@ extern "C" int hia_attn_bwd_reuse_fwd(const hia_segments* g, int Hq, int Hkv, in
   p.scale_log2 = scale * 1.4426950408889634f;
   p.status = status;
   p.timeout_ns = kDefaultTimeoutNs;
-  const int64_t n_entries = int64_t(split ? g->bwd_work_split.size() : g->bwd_work.size()) / hia::kBwdWorkInts;
+  const int64_t n_entries = int64_t(sched.work.size()) / hia::kBwdWorkInts;
   const int64_t n_blocks = n_entries * Hkv;
   if (n_blocks > (1ll << 31) - 1) return HIA_ERR_UNSUPPORTED;
   if ((rc = cuda_status(hia::launch_attn_bwd(tq, tk, tv, tdo, p, int(n_blocks), D, st)))) return rc;

@@ -11,10 +11,11 @@
 // it also zeroes the dQ accumulator and the split schedule's tickets.
 // attn_bwd: one CTA per work-list entry and kv head: a (b, 128-key tile) over
 // the query tiles that see its keys (a range of query tiles, since the row
-// bound e(q) is non-decreasing), or one half of that range for the longest
-// tiles when the split schedule is chosen (the two halves' fp32 dK/dV are
-// added by the half that finishes second).  It keeps Kr and V in shared
-// memory and dK, dV in TMEM, and walks the g heads x its query tiles.  Per query tile, with keys on the MMA M side:
+// bound e(q) is non-decreasing), or, in a split schedule, one of the 2-4
+// consecutive parts of that range for the longest tiles (the parts' fp32
+// dK/dV are added in part order by the part that finishes last).  It keeps
+// Kr and V in shared memory and dK, dV in TMEM, and walks the g heads x its
+// query tiles.  Per query tile, with keys on the MMA M side:
 //   S^T = Kr Qr^T, dP^T = V dO^T      (SS MMAs, M=128, N=64)
 //   P^T = exp2(S^T * scale*log2e - lse2), dS^T = P^T o (dP^T - delta)
 //   dV += P^T dO,  dK += dS^T Qr       (A = P^T / dS^T straight from TMEM)
@@ -131,9 +132,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hkv = bid % p.Hkv;
   bid /= p.Hkv;
   // work entry: this CTA's query tiles [qt_first, qt_end) of kv tile kt (all
-  // that see it, or one half of them when split: slot >= 0)
+  // that see it, or part `part` of `parts` consecutive sub-ranges when split:
+  // slot >= 0)
   const int32_t* we = p.work + kBwdWorkInts * bid;
-  const int b = we[0], kt = we[1], qt_first = we[2], qt_end = we[3], slot = we[4], part = we[5];
+  const int b = we[0], kt = we[1], qt_first = we[2], qt_end = we[3], slot = we[4], part = we[5], parts = we[6];
   // [full_first, full_end): the query tiles that see all of the kv tile
   const int32_t* te = p.tiles + 4 * (b * p.bKT + kt);
   const int full_first = te[2], full_end = te[3];
@@ -365,18 +367,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool have = n_it > 0 && ok;
     if (have) have = __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, wc));
     if (have) tc_fence_after();
-    bool write_out = true;  // false: the other half of a split kv tile writes dK/dV
+    bool write_out = true;  // false: another part of a split kv tile writes dK/dV
     if (slot >= 0) {
-      // Split kv tile: this CTA saw half of its query tiles.  Each half writes
-      // its raw fp32 accumulator rows (dK in warpgroup 0, dV in warpgroup 1)
-      // to its own partial, fences, and takes a ticket; the half that
-      // finishes second adds the other half's partial into its TMEM (fp32
-      // a + b is commutative: the same bits whichever half is second) and
-      // runs the common epilogue below.  No thread waits on the other CTA.
+      // Split kv tile: this CTA saw one of its `parts` query sub-ranges.
+      // Every part writes its raw fp32 accumulator rows (dK in warpgroup 0,
+      // dV in warpgroup 1) to its own partial, fences, and takes a ticket;
+      // the part that finishes last adds all the partials in part order
+      // (P_0 + P_1 + ..., its own from TMEM: the same bits whichever part is
+      // last) into its TMEM and runs the common epilogue below.  No thread
+      // waits on another CTA.
       const uint32_t tacc = (bf == 0 ? tdK : tdV) + lane_off;
-      const int64_t unit = (int64_t(slot) * p.Hkv + hkv) * 2;
-      float* mine = p.part + ((unit + part) * 2 + bf) * int64_t(BK * D) + int64_t(r) * D;
-      const float* other = p.part + ((unit + (part ^ 1)) * 2 + bf) * int64_t(BK * D) + int64_t(r) * D;
+      const int64_t unit = int64_t(slot) * p.Hkv + hkv;
+      const auto partial = [&](int j) {
+        return p.part + ((unit * parts + j) * 2 + bf) * int64_t(BK * D) + int64_t(r) * D;
+      };
+      float* mine = partial(part);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
@@ -395,10 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __threadfence();
       named_bar_sync(2, 256);  // both epilogue warpgroups' partial rows written and fenced
-      if (threadIdx.x == 128) sm.split_ticket = atomicAdd(&p.part_cnt[slot * p.Hkv + hkv], 1);
+      if (threadIdx.x == 128) sm.split_ticket = atomicAdd(&p.part_cnt[unit], 1);
       named_bar_sync(2, 256);
-      if (sm.split_ticket == 0) {
-        have = false;  // the other half finishes this kv tile
+      if (sm.split_ticket < parts - 1) {
+        have = false;  // a later part finishes this kv tile
         write_out = false;
       } else {
         __threadfence();
@@ -409,20 +414,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t v[32];
           tmem_ld32(tacc + uint32_t(c * 32), v);
           tmem_ld_wait_regs(v);
-          const float4* o4 = reinterpret_cast<const float4*>(other + c * 32);
+          float sum[32];
+#pragma unroll 1
+          for (int j = 0; j < parts; ++j) {
+            float x[32];
+            if (j == part) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 a = __ldcg(o4 + i);
-            v[4 * i] = __float_as_uint(__uint_as_float(v[4 * i]) + a.x);
-            v[4 * i + 1] = __float_as_uint(__uint_as_float(v[4 * i + 1]) + a.y);
-            v[4 * i + 2] = __float_as_uint(__uint_as_float(v[4 * i + 2]) + a.z);
-            v[4 * i + 3] = __float_as_uint(__uint_as_float(v[4 * i + 3]) + a.w);
+              for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(v[i]);
+            } else {
+              const float4* o4 = reinterpret_cast<const float4*>(partial(j) + c * 32);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 a = __ldcg(o4 + i);
+                x[4 * i] = a.x;
+                x[4 * i + 1] = a.y;
+                x[4 * i + 2] = a.z;
+                x[4 * i + 3] = a.w;
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum[i] = j == 0 ? x[i] : sum[i] + x[i];
           }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(sum[i]);
           tmem_st32(tacc + uint32_t(c * 32), v);
         }
         tmem_st_wait();
       }
-      if (write_out && threadIdx.x == 128) p.part_cnt[slot * p.Hkv + hkv] = 0;  // ready for the next launch
+      if (write_out && threadIdx.x == 128) p.part_cnt[unit] = 0;  // ready for the next launch
     }
     const bool store = write_out && key < smp.rows;
     // dK / dV rows leave through shared memory: each thread stages its key

@@ -22,7 +22,8 @@ constexpr int kFwdBM = 128;
 constexpr int kFwdBN = 128;
 constexpr int kBwdBK = 128;
 constexpr int kBwdBQ = 64;
-constexpr int kBwdWorkInts = 6;  // ints per backward work-list entry
+constexpr int kBwdWorkInts = 8;  // ints per backward work-list entry
+constexpr int kBwdMaxParts = 4;  // a split kv tile's query range is cut into at most this many parts
 
 // One image of a sample: tokens [I0, I1) on a grid of width w (row-major).
 // hidden = 1 for a context image: every image of a sample but its last is
@@ -100,19 +101,24 @@ struct hia_segments {
   // tile, those in [full_first, full_end) see all of it.
   int bQT = 0, bKT = 0;
   std::vector<int32_t> bwd_tiles;   // 4 per entry
-  // backward work lists, kBwdWorkInts per entry: (b, kt, qt_lo, qt_hi, slot,
-  // part), heaviest first.  bwd_work: every (b, kv tile) over its whole query
-  // range, slot -1.  bwd_work_split: the same, except that the kv tiles whose
-  // query range is within 10% of the longest are split into two halves (part
-  // 0 and 1) that share a slot: each half writes its fp32 dK/dV partial, and
-  // the half that finishes second adds part 0 + part 1 and writes dK/dV.
-  std::vector<int32_t> bwd_work;
-  std::vector<int32_t> bwd_work_split;
-  int n_split_slots = 0;
-  int bwd_split_mode = 0;           // HIA_BWD_SPLIT_AUTO / _NEVER / _ALWAYS
-  // launch-time choice between the two lists, per (Hkv, g, SM count)
+  // backward schedules: work lists of kBwdWorkInts per entry, (b, kt, qt_lo,
+  // qt_hi, slot, part, parts, 0), heaviest first.  bwd_sched[0]: every (b, kv
+  // tile) over its whole query range (slot -1, parts 1).  bwd_sched[i > 0]:
+  // the same, except that the kv tiles whose query range is at least a given
+  // fraction of the longest are cut into `parts` consecutive sub-ranges (part
+  // 0 .. parts-1) sharing a slot: each writes its fp32 dK/dV partial, and the
+  // one that finishes last adds the partials in part order and writes dK/dV.
+  struct BwdSched {
+    std::vector<int32_t> work;
+    int parts = 1;
+    int n_slots = 0;                  // kv tiles split
+    const int32_t* d_work = nullptr;  // device copy
+  };
+  std::vector<BwdSched> bwd_sched;
+  int bwd_split_mode = 0;           // HIA_BWD_SPLIT_*
+  // launch-time choice of a schedule, per (mode, Hkv, g, SM count)
   std::mutex choice_mu;
-  std::map<std::tuple<int, int, int>, bool> choice;
+  std::map<std::tuple<int, int, int, int>, int> choice;
   int64_t pairs = 0;
   hia_segments_info_t info{};
   // device copies (one allocation)
@@ -124,6 +130,4 @@ struct hia_segments {
   const int32_t* d_fwd_list = nullptr;
   const int32_t* d_fwd_work = nullptr;
   const int32_t* d_bwd_tiles = nullptr;
-  const int32_t* d_bwd_work = nullptr;
-  const int32_t* d_bwd_work_split = nullptr;
 };

@@ -18,10 +18,11 @@
 
 namespace hia {
 
-// K1: one thread per (b, n, j < D/2).  Angle and cos/sin in fp64, rounded
-// once to fp32: a text-only sample reproduces the 1D tables exactly.  The
-// frequencies theta_j = base^(-2j/D) depend on j only: each block evaluates
-// them once into shared memory.
+// K1: one warp per (b, n) row, lane l owns the angles j = l, l + 32, ... <
+// D/2.  The row's position (and its image grid cell) is found once per row.
+// Angle and cos/sin in fp64, rounded once to fp32: a text-only sample
+// reproduces the 1D tables exactly.  The frequencies theta_j = base^(-2j/D)
+// depend on j only: each block evaluates them once into shared memory.
 __global__ void __launch_bounds__(256) rope2d_tables_kernel(const SampleDev* __restrict__ samples,
                                                             const ImageDev* __restrict__ images, int B, int S, int D,
                                                             double base, float* __restrict__ cos_out,
@@ -30,30 +31,29 @@ __global__ void __launch_bounds__(256) rope2d_tables_kernel(const SampleDev* __r
   const int half = D / 2;
   for (int j = threadIdx.x; j < half; j += blockDim.x) theta_s[j] = pow(base, -2.0 * double(j) / double(D));
   __syncthreads();
-  const int64_t total = int64_t(B) * S * half;
-  for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
-       idx += int64_t(gridDim.x) * blockDim.x) {
-    const int j = int(idx % half);
-    const int64_t bn = idx / half;
-    const int n = int(bn % S);
-    const int b = int(bn / S);
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
+  if (row < int64_t(B) * S) {
+    const int b = int(row / S), n = int(row - int64_t(b) * S);
     const SampleDev t = samples[b];
-    double x = n, y = n;
+    int x = n, y = n;
     const int im = image_of(images + t.img0, t.n_img, n);
     if (im >= 0) {  // each image on its own grid, origin at its first token
       const ImageDev g = images[t.img0 + im];
       const int i = n - g.I0;
-      x = double(g.I0 + i % g.w);
-      y = double(g.I0 + i / g.w);
+      x = g.I0 + i % g.w;
+      y = g.I0 + i / g.w;
     }
-    const double a = ((j & 1) ? y : x) * theta_s[j];
-    double sn, cs;
-    sincos(a, &sn, &cs);
-    const int64_t o = bn * D + j;
-    cos_out[o] = float(cs);
-    cos_out[o + half] = float(cs);
-    sin_out[o] = float(sn);
-    sin_out[o + half] = float(sn);
+    for (int j = lane; j < half; j += 32) {
+      const double a = double((j & 1) ? y : x) * theta_s[j];
+      double sn, cs;
+      sincos(a, &sn, &cs);
+      const int64_t o = row * D + j;
+      cos_out[o] = float(cs);
+      cos_out[o + half] = float(cs);
+      sin_out[o] = float(sn);
+      sin_out[o + half] = float(sn);
+    }
   }
 }
 
@@ -307,13 +307,11 @@ int row_grid_blocks(int64_t rows) { return int((rows + 7) / 8); }
 
 void launch_rope2d_tables(const SampleDev* samples, const ImageDev* images, int B, int S, int D, double base,
                           float* cos_out, float* sin_out, cudaStream_t st) {
-  const int64_t total = int64_t(B) * S * (D / 2);
-  if (total == 0) return;
-  const int threads = 256;
-  int64_t blocks = (total + threads - 1) / threads;
-  if (blocks > 148 * 64) blocks = 148 * 64;  // one (b, n, j) per thread up to 2.4 M entries
+  const int64_t rows = int64_t(B) * S;
+  if (rows == 0) return;
+  // one row per warp: rows < 2^31 (checked by the caller), so fewer than 2^28 blocks
   prof_begin(kRopeTables, st);
-  rope2d_tables_kernel<<<int(blocks), threads, 0, st>>>(samples, images, B, S, D, base, cos_out, sin_out);
+  rope2d_tables_kernel<<<row_grid_blocks(rows), 256, 0, st>>>(samples, images, B, S, D, base, cos_out, sin_out);
   prof_end(kRopeTables, st);
 }
 

@@ -174,36 +174,52 @@ int build(const std::vector<SampleSpec>& spec, int S, bool packed, hia_segments*
   order.assign(size_t(B) * g->bKT, 0);
   for (size_t i = 0; i < order.size(); ++i) order[i] = int(i);
   std::stable_sort(order.begin(), order.end(), [&](int a, int c) { return bwd_cost[a] > bwd_cost[c]; });
+  // Schedules: the whole list, and for parts in {2, 3, 4} and a threshold
+  // of 95, 90 or 85% of the longest query range, the list with every kv tile
+  // at or above the threshold cut into `parts` sub-ranges (of at least two
+  // query tiles each).  The launch picks one by a list-scheduling estimate.
   struct BwdJob {
     int64_t cost;
-    int32_t b, kt, lo, hi, slot, part;
+    int32_t b, kt, lo, hi, slot, part, parts;
   };
-  std::vector<BwdJob> whole, split;
   int64_t max_cost = 0;
   for (int u : order) max_cost = std::max(max_cost, bwd_cost[u]);
-  int n_slots = 0;
-  for (int u : order) {
-    const int b = u / g->bKT, kt = u % g->bKT;
-    const int32_t* e = &g->bwd_tiles[size_t(u) * 4];
-    const int64_t c = bwd_cost[u];
-    whole.push_back({c, b, kt, e[0], e[1], -1, 0});
-    if (c >= 4 && 10 * c > 9 * max_cost) {  // within 10% of the longest query range
-      const int mid = e[0] + int(c / 2);
-      split.push_back({mid - e[0], b, kt, e[0], mid, n_slots, 0});
-      split.push_back({e[1] - mid, b, kt, mid, e[1], n_slots, 1});
-      ++n_slots;
-    } else {
-      split.push_back({c, b, kt, e[0], e[1], -1, 0});
+  auto make = [&](int parts, int64_t threshold) {
+    hia_segments::BwdSched sc;
+    sc.parts = parts;
+    std::vector<BwdJob> js;
+    for (int u : order) {
+      const int b = u / g->bKT, kt = u % g->bKT;
+      const int32_t* e = &g->bwd_tiles[size_t(u) * 4];
+      const int64_t c = bwd_cost[u];
+      if (parts > 1 && c >= threshold && c >= 2 * parts) {
+        for (int j = 0; j < parts; ++j) {
+          const int lo = e[0] + int(c * j / parts), hi = e[0] + int(c * (j + 1) / parts);
+          js.push_back({hi - lo, b, kt, lo, hi, sc.n_slots, j, parts});
+        }
+        ++sc.n_slots;
+      } else {
+        js.push_back({c, b, kt, e[0], e[1], -1, 0, 1});
+      }
+    }
+    std::stable_sort(js.begin(), js.end(), [](const BwdJob& x, const BwdJob& y) { return x.cost > y.cost; });
+    for (const BwdJob& j : js) sc.work.insert(sc.work.end(), {j.b, j.kt, j.lo, j.hi, j.slot, j.part, j.parts, 0});
+    return sc;
+  };
+  g->bwd_sched.clear();
+  g->bwd_sched.push_back(make(1, 0));
+  int split_units = 0;
+  for (int parts = 2; parts <= hia::kBwdMaxParts; ++parts) {
+    int prev_slots = -1;
+    for (int pct : {95, 90, 85}) {
+      const int64_t threshold = (max_cost * pct + 99) / 100;
+      hia_segments::BwdSched sc = make(parts, threshold);
+      if (sc.n_slots == 0 || sc.n_slots == prev_slots) continue;  // nothing split, or the same tiles again
+      prev_slots = sc.n_slots;
+      if (parts == 2) split_units = std::max(split_units, sc.n_slots);
+      g->bwd_sched.push_back(std::move(sc));
     }
   }
-  std::stable_sort(split.begin(), split.end(), [](const BwdJob& a, const BwdJob& c) { return a.cost > c.cost; });
-  auto emit = [](const std::vector<BwdJob>& js, std::vector<int32_t>& out) {
-    out.clear();
-    for (const BwdJob& j : js) out.insert(out.end(), {j.b, j.kt, j.lo, j.hi, j.slot, j.part});
-  };
-  emit(whole, g->bwd_work);
-  emit(split, g->bwd_work_split);
-  g->n_split_slots = n_slots;
 
   hia_segments_info_t& in = g->info;
   in.B = B;
@@ -217,7 +233,7 @@ int build(const std::vector<SampleSpec>& spec, int S, bool packed, hia_segments*
   in.bwd_q_tiles = g->bQT;
   in.bwd_kv_tiles = g->bKT;
   in.packed = packed ? 1 : 0;
-  in.bwd_split_units = n_slots;
+  in.bwd_split_units = split_units;
   in.total_rows = g->total_rows;
   *out = g;
   return HIA_OK;
@@ -357,6 +373,16 @@ extern "C" int hia_segments_tile_classes(const hia_segments* g, uint8_t* cls) {
       }
     }
   }
+  return HIA_OK;
+}
+
+extern "C" int hia_segments_bwd_schedule(const hia_segments* g, int index, int32_t* parts, int64_t* n_entries,
+                                         int32_t* entries) {
+  if (!g || index < 0 || index >= int(g->bwd_sched.size()) || !parts || !n_entries) return HIA_ERR_INVALID_ARG;
+  const hia_segments::BwdSched& sc = g->bwd_sched[size_t(index)];
+  *parts = sc.parts;
+  *n_entries = int64_t(sc.work.size()) / hia::kBwdWorkInts;
+  if (entries && !sc.work.empty()) std::memcpy(entries, sc.work.data(), sc.work.size() * sizeof(int32_t));
   return HIA_OK;
 }
 

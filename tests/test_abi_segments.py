@@ -155,15 +155,119 @@ def test_moe_workspace_size_and_empty_batch():
 
 
 def test_bwd_split_units_and_mode():
-    """The descriptor's split schedule: kv tiles within 10% of the longest
-    query range; the mode setter refuses unknown modes."""
+    """The descriptor's split schedules cut some kv tiles (those within 15% of
+    the longest query range), never all; the mode setter takes the six modes
+    and refuses others."""
     seg = jt.hia_segments_build(synth.workload("1024px_bwd").samples, synth.workload("1024px_bwd").S,
                                 upload=False)
     assert seg.info().bwd_split_units > 0
     assert seg.info().bwd_split_units < seg.info().bwd_kv_tiles
-    for mode in (0, 1, 2):
+    for mode in range(6):
         seg.set_bwd_split(mode)
-    with pytest.raises(jt.HiaError):
-        seg.set_bwd_split(3)
+    for bad in (-1, 6):
+        with pytest.raises(jt.HiaError):
+            seg.set_bwd_split(bad)
     tiny = jt.hia_segments_build(synth.workload("tiny").samples, synth.workload("tiny").S, upload=False)
     assert tiny.info().bwd_split_units == 0  # one query range of 2 tiles: nothing worth splitting
+    assert len(tiny.bwd_schedules()) == 1
+
+
+def _schedule_layouts():
+    wl = synth.workload("1024px_bwd")
+    yield "1024px_bwd", jt.hia_segments_build(wl.samples, wl.S, upload=False)
+    wl = synth.workload("mixed")
+    yield "mixed", jt.hia_segments_build(wl.samples, wl.S, upload=False)
+    yield "mixed packed", jt.hia_segments_build_packed(wl.samples, upload=False)
+    wl = synth.workload("multi_image")
+    yield "multi_image", jt.hia_segments_build_multi(wl.samples, wl.S, upload=False)
+
+
+@pytest.mark.parametrize("which", [0, 1, 2, 3])
+def test_bwd_schedules_cover_every_query_range_once(which):
+    """Every backward schedule covers each (sample, kv tile) query range of
+    the whole schedule exactly once: unsplit, or cut into `parts` consecutive
+    sub-ranges of at least two query tiles (parts 0 .. parts-1) that share a
+    slot; slots are 0 .. n-1; entries run heaviest first; the split tiles are
+    exactly those at or above the schedule's threshold."""
+    name, seg = list(_schedule_layouts())[which]
+    sch = seg.bwd_schedules()
+    assert sch[0][0] == 1 and (sch[0][1][:, 4] == -1).all() and (sch[0][1][:, 6] == 1).all()
+    whole = {(int(e[0]), int(e[1])): (int(e[2]), int(e[3])) for e in sch[0][1]}
+    assert len(whole) == len(sch[0][1])
+    longest = max(hi - lo for lo, hi in whole.values())
+    seen_parts = set()
+    for parts, ent in sch:
+        cost = ent[:, 3] - ent[:, 2]
+        assert (np.diff(cost) <= 0).all(), name  # heaviest first
+        assert (ent[:, 7] == 0).all()
+        got = {}
+        slots = {}
+        for e in ent:
+            b, kt, lo, hi, slot, part, p = (int(x) for x in e[:7])
+            if slot < 0:
+                assert part == 0 and p == 1
+                assert (b, kt) not in got
+                got[(b, kt)] = [(lo, hi)]
+            else:
+                assert p == parts and 0 <= part < parts and hi - lo >= 2
+                slots.setdefault(slot, set()).add((b, kt))
+                got.setdefault((b, kt), []).append((part, lo, hi))
+        assert set(got) == set(whole)
+        split = set()
+        for key, rs in got.items():
+            if len(rs) == 1 and len(rs[0]) == 2:
+                assert rs[0] == whole[key]
+                continue
+            split.add(key)
+            rs = sorted(rs)
+            assert [r[0] for r in rs] == list(range(parts))
+            assert rs[0][1] == whole[key][0] and rs[-1][2] == whole[key][1]
+            assert all(rs[i][2] == rs[i + 1][1] for i in range(parts - 1))
+        assert sorted(slots) == list(range(len(slots))) and all(len(v) == 1 for v in slots.values())
+        if parts > 1:
+            assert split, name
+            # a threshold: every split tile is at least as long as every unsplit tile of 2 * parts or more
+            shortest_split = min(whole[k][1] - whole[k][0] for k in split)
+            assert all(whole[k][1] - whole[k][0] < shortest_split for k in whole
+                       if k not in split and whole[k][1] - whole[k][0] >= 2 * parts)
+            assert 100 * shortest_split >= 85 * longest
+            seen_parts.add(parts)
+    assert seen_parts == {2, 3, 4}
+
+
+def _makespan(entries, Hkv, g, n_sm):
+    """Greedy list scheduling: entries in order, each as Hkv CTAs, each CTA on
+    the SM that frees first; a CTA costs its query tiles * g + 9, a part of a
+    split kv tile its query tiles * g * 1.2 + 9, and 22.5 more for the last
+    part."""
+    import heapq
+    sms = [0.0] * n_sm
+    span = 0.0
+    for e in entries:
+        it = float(e[3] - e[2]) * g
+        c = it * 1.2 + 9.0 + (22.5 if e[5] == e[6] - 1 else 0.0) if e[4] >= 0 else it + 9.0
+        for _ in range(Hkv):
+            t = heapq.heappop(sms) + c
+            heapq.heappush(sms, t)
+            span = max(span, t)
+    return span
+
+
+@pytest.mark.parametrize("which", [0, 1, 3])
+def test_bwd_choice_follows_the_estimate(which):
+    """The schedule a launch takes: AUTO the one whose list-scheduling
+    estimate finishes first (ties to the earlier), NEVER the whole one, ALWAYS
+    the best split one, PARTS_k the best one with k parts."""
+    name, seg = list(_schedule_layouts())[which]
+    sch = seg.bwd_schedules()
+    for Hkv, g, n_sm in ((8, 4, 148), (2, 16, 132), (1, 1, 8)):
+        spans = [_makespan(e, Hkv, g, n_sm) for _, e in sch]
+        def best(admit):
+            idx = [i for i in range(len(sch)) if admit(sch[i][0])]
+            return min(idx, key=lambda i: (spans[i], i)) if idx else 0
+        expect = {0: best(lambda p: True), 1: 0, 2: best(lambda p: p > 1),
+                  3: best(lambda p: p == 2), 4: best(lambda p: p == 3), 5: best(lambda p: p == 4)}
+        for mode, want in expect.items():
+            seg.set_bwd_split(mode)
+            assert seg.bwd_choice(Hkv, g, n_sm) == want, (name, mode, Hkv, g, n_sm)
+    seg.set_bwd_split(0)

@@ -145,29 +145,42 @@ def _fwd_bwd_with_split(wl, mode, seed=0):
     return seg, (q, k, v, do), (f(dq), f(dk), f(dv))
 
 
-@pytest.mark.parametrize("name", ["256px", "mixed_small"])
-def test_bwd_split_schedule_parity(oracle_mod, name):
-    """The split schedule (the longest kv tiles' query ranges halved, the two
-    fp32 partials of dK/dV added by the half that finishes second), forced on:
-    against the oracle in full and block by block, dk/dv bitwise repeatable."""
+def _chosen_parts(seg, wl):
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    return seg.bwd_schedules()[seg.bwd_choice(wl.Hkv, wl.Hq // wl.Hkv, n_sm)][0]
+
+
+@pytest.mark.parametrize("name,mode", [("256px", 2), ("256px", 4), ("mixed_small", 3), ("mixed_small", 4),
+                                       ("mixed_small", 5)])
+def test_bwd_split_schedule_parity(oracle_mod, name, mode):
+    """A split schedule forced on: mode 2 the estimate's best split one, 3 / 4
+    / 5 the longest kv tiles' query ranges cut into 2 / 3 / 4 parts (each part
+    a CTA writing fp32 dK/dV partials, added in part order by the part that
+    finishes last): against the oracle in full and block by block, dk/dv
+    bitwise repeatable."""
     if name == "mixed_small":
         wl = synth.custom([(300, 12, 20, 5), (0, 0, 0, 0), (700, 0, 0, 0), (64, 16, 16, 2)], 8, 2, 128)
     else:
         wl = synth.workload(name)
-    seg, inputs, g1 = _fwd_bwd_with_split(wl, 2)
+    seg, inputs, g1 = _fwd_bwd_with_split(wl, mode)
     assert seg.info().bwd_split_units > 0
+    parts = _chosen_parts(seg, wl)
+    assert parts == mode - 1 if mode >= 3 else parts > 1
     check_bwd(oracle_mod, wl, inputs, g1)
-    _, _, g2 = _fwd_bwd_with_split(wl, 2)
+    _, _, g2 = _fwd_bwd_with_split(wl, mode)
     assert np.array_equal(g1[1], g2[1]) and np.array_equal(g1[2], g2[2])
 
 
-def test_bwd_split_schedule_full_size(oracle_mod):
-    """The single-sample training backward (1024px_bwd) with the split
-    schedule forced on: two complete (b, kv head) groups against the oracle,
-    one of them a kv head whose prefix tiles are split."""
+@pytest.mark.parametrize("mode", [2, 4])
+def test_bwd_split_schedule_full_size(oracle_mod, mode):
+    """The single-sample training backward (1024px_bwd) with a split schedule
+    forced on (the best split one, which cuts the longest tiles in four, and
+    the best three-part one): two complete (b, kv head) groups against the
+    oracle, one of them a kv head whose prefix tiles are split."""
     wl = synth.workload("1024px_bwd")
-    seg, inputs, grads = _fwd_bwd_with_split(wl, 2)
+    seg, inputs, grads = _fwd_bwd_with_split(wl, mode)
     assert seg.info().bwd_split_units > 0
+    assert _chosen_parts(seg, wl) == (4 if mode == 2 else 3)
     groups = np.zeros((wl.B, wl.Hkv), dtype=bool)
     groups[0, 1] = groups[0, 6] = True
     check_bwd(oracle_mod, wl, inputs, grads, groups=groups)
