@@ -44,8 +44,8 @@ def padded_inputs(wl, seed=0):
 
 # The bitwise comparisons below hold for one backward schedule: under the
 # automatic choice the two layouts (different query ranges per kv tile) may
-# pick different ones, and a split kv tile sums its two halves' fp32 partials
-# in a different order than one accumulation.  Both run the unsplit schedule.
+# pick different ones, and a split kv tile sums its parts' fp32 partials in a
+# different order than one accumulation.  Both run the unsplit schedule.
 NEVER_SPLIT = 1
 
 
