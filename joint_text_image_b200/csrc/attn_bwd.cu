@@ -378,10 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // waits on another CTA.
       const uint32_t tacc = (bf == 0 ? tdK : tdV) + lane_off;
       const int64_t unit = int64_t(slot) * p.Hkv + hkv;
+      // a partial is BK x D fp32 stored as [D / 4][BK] float4: row r's float4
+      // number q at q * BK + r, so a warp's 32 rows are 512 contiguous bytes
       const auto partial = [&](int j) {
-        return p.part + ((unit * parts + j) * 2 + bf) * int64_t(BK * D) + int64_t(r) * D;
+        return reinterpret_cast<float4*>(p.part + ((unit * parts + j) * 2 + bf) * int64_t(BK * D)) + r;
       };
-      float* mine = partial(part);
+      float4* mine = partial(part);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
@@ -392,10 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0u;
         }
-        float4* d4 = reinterpret_cast<float4*>(mine + c * 32);
+        float4* d4 = mine + c * 8 * BK;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
+          d4[i * BK] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
                               __uint_as_float(v[4 * i + 3]));
       }
       __threadfence();
@@ -422,10 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(v[i]);
             } else {
-              const float4* o4 = reinterpret_cast<const float4*>(partial(j) + c * 32);
+              const float4* o4 = partial(j) + c * 8 * BK;
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const float4 a = __ldcg(o4 + i);
+                const float4 a = __ldcg(o4 + i * BK);
                 x[4 * i] = a.x;
                 x[4 * i + 1] = a.y;
                 x[4 * i + 2] = a.z;

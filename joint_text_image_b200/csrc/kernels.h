@@ -85,7 +85,7 @@ struct BwdParams {
   const ImageDev* images;
   const int32_t* tiles;  // [B][bKT][4]: (qt_first, qt_end, full_first, full_end)
   const int32_t* work;   // [n_work][kBwdWorkInts]: (b, kt, qt_lo, qt_hi, slot, part, parts, 0)
-  float* part;           // split tiles' fp32 partials [slot][Hkv][part < parts][dK, dV][128][D]
+  float* part;           // split tiles' fp32 partials [slot][Hkv][part < parts][dK, dV][D / 4][128] float4
   int* part_cnt;         // [slot][Hkv] tickets (zeroed by bwd_pre)
   int B, S, S_pad, Hq, Hkv, g, bQT, bKT;
   const float* lse2;
