@@ -271,3 +271,28 @@ def test_bwd_choice_follows_the_estimate(which):
             seg.set_bwd_split(mode)
             assert seg.bwd_choice(Hkv, g, n_sm) == want, (name, mode, Hkv, g, n_sm)
     seg.set_bwd_split(0)
+
+
+def test_bwd_workspace_sized_for_the_chosen_schedule():
+    """The backward workspace holds the fp32 dK/dV partials of the schedule a
+    launch takes (for every part, kv head and split tile a 128 x D block for
+    dK and one for dV, plus a ticket per split tile and kv head), so it grows
+    with the forced part count and equals the unsplit size plus that much."""
+    wl = synth.workload("1024px_bwd")
+    seg = jt.hia_segments_build(wl.samples, wl.S, upload=False)
+    Hq, Hkv, D = wl.Hq, wl.Hkv, wl.D
+    align = lambda n: (n + 255) // 256 * 256
+    seg.set_bwd_split(1)
+    base = jt.hia_attn_bwd_workspace_bytes(seg, Hq, Hkv, D)
+    sch = seg.bwd_schedules()
+    sizes = {}
+    for mode in (3, 4, 5):
+        seg.set_bwd_split(mode)
+        parts, ent = sch[seg.bwd_choice(Hkv, Hq // Hkv, 148)]
+        assert parts == mode - 1
+        slots = len({int(e[4]) for e in ent if e[4] >= 0})
+        got = jt.hia_attn_bwd_workspace_bytes(seg, Hq, Hkv, D)
+        assert got == base + align(slots * Hkv * parts * 2 * 128 * D * 4) + align(slots * Hkv * 4)
+        sizes[mode] = got
+    assert base < sizes[3] and base < sizes[5]
+    seg.set_bwd_split(0)
